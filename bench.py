@@ -1,0 +1,378 @@
+"""Benchmark of one ZeRO-3 per-rank step on B200: the fused reduce-scatter
+reduction + AdamW + bf16 cast over every owned partition of a LLaMA-7B decoder
+block at D = 8 simulated ranks, then the all-gather of the 8 bf16 shards into
+the flat block (with zero-copy per-tensor views) and the host-side plan and
+memory ledger.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--e2e-steps E]
+
+One process per GPU (torchrun for N > 1).  Each rank runs its own block
+(independent replicas: the path needs no inter-GPU exchange), so the work per
+GPU is fixed as N grows.  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps between a barrier plus
+cudaDeviceSynchronize on each side, timed with CUDA events on the launching
+stream, max over ranks.  Each step streams about 9.3 GB through HBM, far more
+than the 126 MB L2, so no flush is needed between steps.  The fused kernel is
+also timed launch by launch with its own events for the roofline figure.
+
+--impl reference times the oracle (plain single-threaded C) on the host on a
+bounded sample of the same workload; it is a deliberately slow baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "owned params/s for fused reduce+AdamW+cast; achieved HBM GB/s vs ~8 TB/s"
+UNIT = "owned params/s"
+PROFILE_K1 = os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md")
+K1_SOURCE = os.path.join(ROOT, "fsdp_sharded_mixed_flat_b200", "csrc", "reduce_adamw.cu")
+SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b_d8")
+    ap.add_argument("--e2e-steps", type=int, default=12)
+    ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="elements of the oracle's sample")
+    ap.add_argument("--cpu-steps", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary of the fused kernel,
+    if that summary was taken on the current kernel source; else None."""
+    if not os.path.exists(PROFILE_K1):
+        return None
+    text = open(PROFILE_K1).read()
+    sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    tb = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not sha or not tb:
+        return None
+    cur = hashlib.sha256(open(K1_SOURCE, "rb").read()).hexdigest()
+    return float(tb.group(1)) if sha.group(1) == cur else None
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_uuid: str | None):
+        self.uuid = device_uuid
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm), "samples_under_load": len(loaded),
+                "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------- distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def aggregate(local_seconds: float, local_units: float, world: int, device=None):
+    """(max seconds over ranks, total units over ranks): the whole-job figures."""
+    if world == 1:
+        return local_seconds, local_units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([local_seconds], dtype=torch.float64, device=device)
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+# --------------------------------------------------------------- the oracle
+def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0):
+    """Time the oracle over `steps` passes of a `sample`-element slice of the
+    workload's owned elements (all D contributions, AdamW, cast).  Returns
+    (owned params/s, seconds, description)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import synth
+    w = synth.WORKLOADS[workload]
+    D = w["D"]
+    n = min(sample, synth.block_numel(w["tensors"]))
+    contribs = [synth.bf16_bits(synth.contribution(n, n, seed=seed, step=1, rank=d, sigma=w["sigma"],
+                                                   dist=w["dist"], device="cpu")) for d in range(D)]
+    p = synth.master_weights(n, n, seed=seed).numpy().copy()
+    m, v, wk = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
+    oracle.lib()
+    t0 = time.perf_counter()
+    for t in range(1, steps + 1):
+        oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED)
+    dt = time.perf_counter() - t0
+    del torch
+    desc = (f"{workload}: first {n} owned elements x {steps} steps, D={D}, one thread "
+            f"(oracle/zero3_ref.c, single-threaded C)")
+    return n * steps / dt, dt, desc
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    steps = max(1, args.steps)
+    # each step is a bounded sample (2^20 elements) so that K steps stay within minutes
+    sample = min(args.cpu_sample, 1 << 20)
+    if args.warmup > 0:
+        oracle_sample(args.workload, min(sample, 1 << 16), 1)
+    value, secs, desc = oracle_sample(args.workload, sample, steps)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": args.workload, "sample_elements": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our path
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local_rank = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from fsdp_sharded_mixed_flat_b200 import build
+    if rank == 0 or not os.path.exists(build.LIB):
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import synth
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+
+    w = synth.WORKLOADS[args.workload]
+    shapes = [s for _, s in w["tensors"]]
+    D = w["D"]
+    plan = z3.zero3_plan(shapes, D, synth.ALIGN)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    seed = 1000 + rank  # every rank runs its own block
+    contribs = synth.contributions(D, N, N_pad, seed=seed, step=1, sigma=w["sigma"], dist=w["dist"],
+                                   zero_frac=w.get("zero_frac", 0.0), device=dev)
+    master = synth.master_weights(N, N_pad, seed=seed, device=dev)
+    exp_avg, exp_avg_sq = torch.zeros_like(master), torch.zeros_like(master)
+    work = torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)
+    flat = torch.empty(N_pad, dtype=torch.bfloat16, device=dev)
+    shards = [work[r * S:(r + 1) * S] for r in range(D)]
+    stream = torch.cuda.current_stream(dev)
+    step_no = [0]
+
+    def step(k1_events=None):
+        # a1 + a2: host-side plan and ledger of the block (microseconds, overlapped with the GPU)
+        pl = z3.zero3_plan(shapes, D, synth.ALIGN)
+        z3.zero3_memory_bytes(pl.N, D, z3.Z3_STAGE_ZERO3)
+        step_no[0] += 1
+        hp = z3.adamw(lr=w_adamw["lr"], beta1=w_adamw["beta1"], beta2=w_adamw["beta2"], eps=w_adamw["eps"],
+                      weight_decay=w_adamw["weight_decay"], step=step_no[0])
+        if k1_events is not None:
+            k1_events[0].record(stream)
+        # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
+        z3.zero3_reduce_adamw(pl, -1, contribs, master, exp_avg, exp_avg_sq, work, hp, stream=stream)
+        if k1_events is not None:
+            k1_events[1].record(stream)
+        # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
+        z3.zero3_gather_block(pl, shards, flat, None, stream=stream)
+        return pl.views(flat)
+
+    w_adamw = synth.ADAMW
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else None)
+    clocks.start()
+    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(k1_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    secs = t0.elapsed_time(t1) / 1e3
+    k1_ms = [a.elapsed_time(b) for a, b in k1_ev]
+    k1_avg_s = statistics.mean(k1_ms) / 1e3
+    job_secs, job_units = aggregate(secs, float(N_pad) * args.steps, world, dev)
+    value = job_units / job_secs
+
+    # ---- end to end through the public API with host buffers
+    e2e_steps = max(1, args.e2e_steps)
+    host_c = [torch.empty(N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in range(D)]
+    for h, c in zip(host_c, contribs):
+        h.copy_(c)
+    host_flat = torch.empty(N_pad, dtype=torch.bfloat16, pin_memory=True)
+    h2d = sum(h.numel() * h.element_size() for h in host_c)
+    d2h = host_flat.numel() * host_flat.element_size()
+
+    def e2e_step():
+        for h, c in zip(host_c, contribs):
+            c.copy_(h, non_blocking=True)
+        step()
+        host_flat.copy_(flat, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_secs, e2e_units = aggregate(e0.elapsed_time(e1) / 1e3, float(N_pad) * e2e_steps, world, dev)
+
+    hbm_peak, peak_kind = measured_peaks()
+    bytes_per_param = 2 * D + 26
+    k1_gbs = bytes_per_param * N_pad / k1_avg_s / 1e9
+    step_bytes = bytes_per_param * N_pad + 4 * N_pad
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: " + describe(args.workload, N, N_pad, S, D),
+                   "D": D, "N": N, "N_pad": N_pad, "S": S, "reduce_dtype": "fp32",
+                   "launch": "all D partitions in one launch (rank=-1), full contribution layout",
+                   "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (step_bytes / 1e9),
+                   "parallelism": f"replicas x{world} (one block per GPU, no collective)"},
+        "step_hbm_gbs": step_bytes * args.steps * world / job_secs / 1e9,
+        "kernels": {"reduce_adamw_ms": 1e3 * k1_avg_s, "reduce_adamw_gbs": k1_gbs,
+                    "reduce_adamw_params_per_s": N_pad / k1_avg_s,
+                    "gather_ms_est": max(0.0, 1e3 * secs / args.steps - 1e3 * k1_avg_s)},
+        "roofline": {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind,
+                     "kernel": "k_reduce_adamw_vec<fp32, D=8>",
+                     "algorithmic_bytes_per_launch": bytes_per_param * N_pad,
+                     "traffic": profiled_traffic()},
+        "clocks": clk,
+        "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": 2 * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, secs_cpu, desc = oracle_sample(args.workload, args.cpu_sample, args.cpu_steps)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                                "seconds": secs_cpu}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def describe(name, N, N_pad, S, D):
+    import synth
+    w = synth.WORKLOADS[name]
+    return (f"{len(w['tensors'])} tensors, N={N}, N_pad={N_pad}, S={S} per rank, D={D}, "
+            f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
+            f"b=(0.9,0.95) eps=1e-8 wd=0.1")
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

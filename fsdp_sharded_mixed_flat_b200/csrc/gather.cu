@@ -1,0 +1,244 @@
+// gather.cu -- the all-gather's data movement and the unflatten, for sm_100a.
+//
+// "Building GPT from Scratch — Part 8: FSDP — When the Model Won't Fit",
+// "AllGather vs AllReduce": GPU r holds shard r; after the all-gather every GPU
+// holds the whole block [A, B, C, D].  "7.10 — Fully-sharded data parallel
+// (FSDP / ZeRO-3)", §5.1: the gathered parameters are then used as the block's
+// tensors (the unflatten).
+//
+// Both kernels are pure copies bound by HBM bandwidth (2 bytes read + 2 bytes
+// written per element).
+//   - flat copy: grid.y = rank; every thread moves 4 independent 16-byte
+//     vectors per iteration (64 bytes in flight per thread), streaming hints.
+//   - per-tensor copy: the host cuts every tensor into segments, one per rank
+//     partition it intersects, and numbers the 16-byte units of each
+//     segment's destination.  A thread takes one destination unit, finds its
+//     segment by binary search, and writes it with one 16-byte store when the
+//     unit is whole; the source run may start at any 2-byte position, so it is
+//     assembled from the two aligned 16-byte source vectors around it with
+//     funnel shifts.  Partial units at a segment's ends are written element
+//     by element.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <vector>
+
+#include "plan_impl.h"
+#include "zero3.h"
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+constexpr int kSegMax = 112;  // segments per launch; keeps the parameter block under 4 KB
+
+struct FlatArgs {
+    const uint16_t* shard[Z3_D_MAX];
+    uint16_t* flat;
+    int64_t S;
+};
+
+struct Seg {
+    const uint16_t* src;  // first source element
+    uint16_t* dst;        // first destination element
+    int64_t len;          // elements
+    int64_t unit_begin;   // index of the segment's first destination unit in this launch
+};
+
+struct SegArgs {
+    Seg seg[kSegMax];
+    int32_t nseg;
+    int32_t vec;          // 1: sources may be read as aligned 16-byte vectors
+    int64_t units;        // destination units in this launch
+};
+
+__global__ void __launch_bounds__(kThreads) k_gather_flat_vec(const __grid_constant__ FlatArgs a) {
+    const int r = blockIdx.y;
+    const uint4* src = reinterpret_cast<const uint4*>(a.shard[r]);
+    uint4* dst = reinterpret_cast<uint4*>(a.flat + int64_t(r) * a.S);
+    const int64_t n = a.S >> 3;
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    for (; i + (kUnroll - 1) * stride < n; i += kUnroll * stride) {
+        uint4 q[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) q[k] = __ldcs(src + i + k * stride);
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) __stcs(dst + i + k * stride, q[k]);
+    }
+    for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
+}
+
+__global__ void __launch_bounds__(kThreads) k_gather_flat_scalar(const __grid_constant__ FlatArgs a) {
+    const int r = blockIdx.y;
+    const uint16_t* src = a.shard[r];
+    uint16_t* dst = a.flat + int64_t(r) * a.S;
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t j = int64_t(blockIdx.x) * kThreads + threadIdx.x; j < a.S; j += stride) dst[j] = src[j];
+}
+
+// Eight consecutive bf16 values starting at element pointer s, read as aligned
+// 16-byte vectors (the caller guarantees both vectors lie inside the source).
+__device__ __forceinline__ uint4 load8_unaligned(const uint16_t* s) {
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(s);
+    const uint32_t delta = uint32_t(addr >> 1) & 7u;  // elements past the 16-byte boundary
+    const uint4* base = reinterpret_cast<const uint4*>(addr & ~uintptr_t(15));
+    const uint4 A = __ldcs(base);
+    if (delta == 0) return A;
+    const uint4 B = __ldcs(base + 1);
+    const uint32_t w[8] = {A.x, A.y, A.z, A.w, B.x, B.y, B.z, B.w};
+    const uint32_t q = delta >> 1;              // whole words to skip
+    const uint32_t sh = (delta & 1u) * 16u;     // plus half a word
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        // words k+q and k+q+1, picked without dynamic register indexing
+        uint32_t lo = w[k], hi = w[k + 1];
+#pragma unroll
+        for (int j = 1; j < 4; ++j)
+            if (q == uint32_t(j)) { lo = w[k + j]; hi = w[k + j + 1]; }
+        o[k] = __funnelshift_r(lo, hi, sh);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__global__ void __launch_bounds__(kThreads) k_gather_segments(const __grid_constant__ SegArgs a) {
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t u = int64_t(blockIdx.x) * kThreads + threadIdx.x; u < a.units; u += stride) {
+        // segment holding unit u: the last one whose unit_begin <= u
+        int lo = 0, hi = a.nseg - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.seg[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+        }
+        const Seg& s = a.seg[lo];
+        const uintptr_t d0 = reinterpret_cast<uintptr_t>(s.dst);
+        const uintptr_t unit_addr = (d0 & ~uintptr_t(15)) + uintptr_t(u - s.unit_begin) * 16u;
+        // elements of this unit inside the segment: [k0, k1) relative to s.dst
+        const int64_t k_first = (int64_t(unit_addr) - int64_t(d0)) / 2;  // may be negative
+        const int64_t k0 = k_first < 0 ? 0 : k_first;
+        const int64_t k1 = k_first + 8 < s.len ? k_first + 8 : s.len;
+        if (a.vec && k_first >= 0 && k_first + 8 <= s.len) {
+            *reinterpret_cast<uint4*>(unit_addr) = load8_unaligned(s.src + k_first);
+        } else {
+            for (int64_t k = k0; k < k1; ++k) s.dst[k] = s.src[k];
+        }
+    }
+}
+
+}  // namespace
+
+namespace z3 {
+
+int sm_count() {
+    static int cached[Z3_D_MAX * 2] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < Z3_D_MAX * 2 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    if (dev >= 0 && dev < Z3_D_MAX * 2) cached[dev] = n;
+    return n;
+}
+
+}  // namespace z3
+
+extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
+                                         uint16_t* const* tensor_out, void* cuda_stream) {
+    if (p == nullptr || shards == nullptr || (flat_out == nullptr && tensor_out == nullptr)) return Z3_EINVAL;
+    const int32_t D = p->D;
+    const int64_t S = p->S;
+    const int32_t nt = static_cast<int32_t>(p->numel.size());
+    for (int32_t r = 0; r < D; ++r) {
+        if (shards[r] == nullptr) return Z3_EINVAL;
+        if (!z3::aligned(shards[r], 2)) return Z3_EALIGN;
+    }
+    if (flat_out != nullptr && !z3::aligned(flat_out, 2)) return Z3_EALIGN;
+    if (tensor_out != nullptr)
+        for (int32_t i = 0; i < nt; ++i)
+            if (tensor_out[i] != nullptr && !z3::aligned(tensor_out[i], 2)) return Z3_EALIGN;
+    // outputs overlap neither the shards nor each other
+    for (int32_t r = 0; r < D; ++r) {
+        if (flat_out && z3::overlaps(flat_out, p->N_pad * 2, shards[r], S * 2)) return Z3_EINVAL;
+        if (tensor_out)
+            for (int32_t i = 0; i < nt; ++i)
+                if (tensor_out[i] && z3::overlaps(tensor_out[i], p->numel[i] * 2, shards[r], S * 2))
+                    return Z3_EINVAL;
+    }
+    if (tensor_out) {
+        for (int32_t i = 0; i < nt; ++i) {
+            if (!tensor_out[i]) continue;
+            if (flat_out && z3::overlaps(tensor_out[i], p->numel[i] * 2, flat_out, p->N_pad * 2))
+                return Z3_EINVAL;
+            for (int32_t k = i + 1; k < nt; ++k)
+                if (tensor_out[k] &&
+                    z3::overlaps(tensor_out[i], p->numel[i] * 2, tensor_out[k], p->numel[k] * 2))
+                    return Z3_EINVAL;
+        }
+    }
+    if (p->N_pad == 0) return Z3_OK;
+
+    const cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
+    const int sms = z3::sm_count();
+    if (sms < 1) return Z3_ECUDA;
+    bool vec_src = (S % 8) == 0;
+    for (int32_t r = 0; r < D; ++r) vec_src = vec_src && z3::aligned(shards[r], 16);
+
+    // ---- the all-gather into the flat block
+    if (flat_out != nullptr) {
+        FlatArgs a;
+        for (int32_t r = 0; r < Z3_D_MAX; ++r) a.shard[r] = r < D ? shards[r] : nullptr;
+        a.flat = flat_out;
+        a.S = S;
+        const bool vec = vec_src && z3::aligned(flat_out, 16);
+        auto fn = vec ? k_gather_flat_vec : k_gather_flat_scalar;
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const int64_t items = vec ? ((S >> 3) + kUnroll - 1) / kUnroll : S;
+        int64_t bx = (items + kThreads - 1) / kThreads;
+        const int64_t cap = std::max<int64_t>(1, (int64_t(sms) * per_sm + D - 1) / D);
+        bx = std::max<int64_t>(1, std::min(bx, cap));
+        fn<<<dim3(unsigned(bx), unsigned(D)), dim3(kThreads), 0, stream>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;
+    }
+
+    // ---- the per-tensor copies, straight from the shards
+    if (tensor_out != nullptr) {
+        std::vector<Seg> segs;
+        for (int32_t i = 0; i < nt; ++i) {
+            if (!tensor_out[i] || p->numel[i] == 0) continue;
+            const int64_t b = p->offset[i], e = b + p->numel[i];
+            for (int64_t r = b / S; r < D && r * S < e; ++r) {
+                const int64_t lo = std::max(b, r * S), hi = std::min(e, (r + 1) * S);
+                if (hi <= lo) continue;
+                segs.push_back(Seg{shards[r] + (lo - r * S), tensor_out[i] + (lo - b), hi - lo, 0});
+            }
+        }
+        for (size_t first = 0; first < segs.size(); first += kSegMax) {
+            SegArgs a;
+            a.nseg = int32_t(std::min<size_t>(kSegMax, segs.size() - first));
+            a.vec = vec_src ? 1 : 0;
+            int64_t units = 0;
+            for (int32_t k = 0; k < a.nseg; ++k) {
+                Seg s = segs[first + k];
+                const uintptr_t d0 = reinterpret_cast<uintptr_t>(s.dst);
+                const uintptr_t d1 = d0 + uintptr_t(s.len) * 2 - 1;
+                s.unit_begin = units;
+                units += int64_t((d1 >> 4) - (d0 >> 4)) + 1;
+                a.seg[k] = s;
+            }
+            a.units = units;
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gather_segments, kThreads, 0) !=
+                    cudaSuccess || per_sm < 1)
+                per_sm = 1;
+            int64_t blocks = (units + kThreads - 1) / kThreads;
+            blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(sms) * per_sm));
+            k_gather_segments<<<dim3(unsigned(blocks)), dim3(kThreads), 0, stream>>>(a);
+            if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;
+        }
+    }
+    return Z3_OK;
+}

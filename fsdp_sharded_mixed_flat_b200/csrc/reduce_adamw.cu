@@ -1,0 +1,296 @@
+// reduce_adamw.cu -- the fused per-rank optimiser pass for sm_100a:
+// reduce-scatter's reduction of the D bf16 gradient contributions for the
+// owned partition(s), AdamW on the owned fp32 master / m / v, and the cast of
+// the new master to the bf16 working shard, in one streaming pass over HBM.
+//
+// Pages: "Building GPT from Scratch — Part 8: FSDP — When the Model Won't
+// Fit", "AllGather vs AllReduce" (rank r receives the sum of the r-th slice of
+// every rank's gradient) and "Mixed Precision: Cutting Memory in Half" (fp32
+// master, bf16 params); "7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)",
+// §3 (rank r updates only P_r from its fp32 master, m, v and gradient slice)
+// and §4 (reduce-scatter replaces the all-reduce).
+//
+// The pass is bound by HBM bandwidth: per owned element it reads 2*D bytes of
+// contributions and 12 bytes of state, and writes 12 bytes of state and 2
+// bytes of bf16 weights, against about 40 floating-point operations.  There is
+// no contraction, so no tensor-core work.  Each thread owns 8 consecutive
+// elements per iteration: one 16-byte load per rank, two per state array,
+// all issued before the arithmetic so that (D + 6) x 16 bytes per thread are
+// in flight; the ranks are folded in order 0..D-1 in chunks of 8 to bound
+// registers at large D.  Loads and stores use the streaming cache hint: every
+// byte is touched exactly once.  Every arithmetic step is an explicitly
+// rounded fp32 intrinsic so that nothing is contracted into an FMA and the
+// results are fixed by the stated operation order.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "plan_impl.h"
+#include "zero3.h"
+
+namespace {
+
+struct AdamScalars {
+    float step_size;     // lr / (1 - b1^t)
+    float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
+    float decay;         // 1 - lr * wd
+    float b1, omb1, b2, omb2, eps;
+};
+
+struct K1Args {
+    const uint16_t* c[Z3_D_MAX];  // contributions, each at the launch's first element
+    float* p;                     // master
+    float* m;                     // exp_avg
+    float* v;                     // exp_avg_sq
+    uint16_t* w;                  // bf16 working weights
+    int64_t n;                    // elements in this launch
+    int32_t D;
+    float inv_D;                  // fp32 nearest to 1/D
+    AdamScalars s;
+};
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float lo_bf16(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float hi_bf16(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
+__device__ __forceinline__ float bf16_of(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// fp32 -> nearest-even bf16 -> fp32.
+__device__ __forceinline__ float round_to_bf16(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+// Two fp32 values -> two nearest-even bf16 in one 32-bit word (lo in bits 0..15).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// One AdamW element; each step a single fp32 operation rounded to nearest-even.
+__device__ __forceinline__ void adamw_elem(const AdamScalars& s, float g, float& p, float& m,
+                                           float& v) {
+    const float p1 = __fmul_rn(p, s.decay);
+    const float m1 = __fadd_rn(__fmul_rn(s.b1, m), __fmul_rn(s.omb1, g));
+    const float v1 = __fadd_rn(__fmul_rn(s.b2, v), __fmul_rn(s.omb2, __fmul_rn(g, g)));
+    const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v1), s.inv_sqrt_bc2), s.eps);
+    const float delta = __fmul_rn(s.step_size, __fdiv_rn(m1, denom));
+    p = __fsub_rn(p1, delta);
+    m = m1;
+    v = v1;
+}
+
+// Fold one rank's 8 bf16 values (one 16-byte vector) into the accumulators.
+template <int MODE>
+__device__ __forceinline__ void fold8(float (&acc)[8], const uint4& q, bool first) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float a = lo_bf16(w[k]), b = hi_bf16(w[k]);
+        if (first) {
+            acc[2 * k] = a;
+            acc[2 * k + 1] = b;
+        } else if (MODE == Z3_REDUCE_FP32) {
+            acc[2 * k] = __fadd_rn(acc[2 * k], a);
+            acc[2 * k + 1] = __fadd_rn(acc[2 * k + 1], b);
+        } else {
+            acc[2 * k] = round_to_bf16(__fadd_rn(acc[2 * k], a));
+            acc[2 * k + 1] = round_to_bf16(__fadd_rn(acc[2 * k + 1], b));
+        }
+    }
+}
+
+// Reduce ranks 0..D-1 for the 8 elements starting at e, in chunks of 8 ranks:
+// the chunk's loads are all issued before its folds.
+template <int MODE, int DT>
+__device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&acc)[8]) {
+    const int D = DT > 0 ? DT : a.D;
+#pragma unroll
+    for (int d0 = 0; d0 < (DT > 0 ? DT : Z3_D_MAX); d0 += 8) {
+        if (DT == 0 && d0 >= D) break;
+        uint4 q[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (d0 + k < D) q[k] = __ldcs(reinterpret_cast<const uint4*>(a.c[d0 + k] + e));
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (d0 + k < D) fold8<MODE>(acc, q[k], d0 + k == 0);
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ float finish(float acc, float inv_D) {
+    const float g = __fmul_rn(acc, inv_D);
+    return MODE == Z3_REDUCE_FP32 ? g : round_to_bf16(g);
+}
+
+// One element on the scalar path (tails and misaligned buffers).
+template <int MODE>
+__device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
+    float acc = bf16_of(a.c[0][i]);
+    for (int d = 1; d < a.D; ++d) {
+        const float x = bf16_of(a.c[d][i]);
+        acc = MODE == Z3_REDUCE_FP32 ? __fadd_rn(acc, x) : round_to_bf16(__fadd_rn(acc, x));
+    }
+    const float g = finish<MODE>(acc, a.inv_D);
+    float p = a.p[i], m = a.m[i], v = a.v[i];
+    adamw_elem(a.s, g, p, m, v);
+    a.p[i] = p;
+    a.m[i] = m;
+    a.v[i] = v;
+    a.w[i] = __bfloat16_as_ushort(__float2bfloat16_rn(p));
+}
+
+// Vector kernel: every pointer 16-byte aligned.  Grid-stride over 8-element
+// chunks; the last n % 8 elements go through the scalar path.
+template <int MODE, int DT>
+__global__ void __launch_bounds__(kThreads) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
+    const int64_t n8 = a.n >> 3;
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+    for (int64_t q = tid; q < n8; q += stride) {
+        const int64_t e = q << 3;
+        const float4 p0 = __ldcs(reinterpret_cast<const float4*>(a.p + e));
+        const float4 p1 = __ldcs(reinterpret_cast<const float4*>(a.p + e + 4));
+        const float4 m0 = __ldcs(reinterpret_cast<const float4*>(a.m + e));
+        const float4 m1 = __ldcs(reinterpret_cast<const float4*>(a.m + e + 4));
+        const float4 v0 = __ldcs(reinterpret_cast<const float4*>(a.v + e));
+        const float4 v1 = __ldcs(reinterpret_cast<const float4*>(a.v + e + 4));
+        float acc[8];
+        reduce8<MODE, DT>(a, e, acc);
+        float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+        float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) adamw_elem(a.s, finish<MODE>(acc[k], a.inv_D), p[k], m[k], v[k]);
+        __stcs(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
+        __stcs(reinterpret_cast<float4*>(a.p + e + 4), make_float4(p[4], p[5], p[6], p[7]));
+        __stcs(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
+        __stcs(reinterpret_cast<float4*>(a.m + e + 4), make_float4(m[4], m[5], m[6], m[7]));
+        __stcs(reinterpret_cast<float4*>(a.v + e), make_float4(v[0], v[1], v[2], v[3]));
+        __stcs(reinterpret_cast<float4*>(a.v + e + 4), make_float4(v[4], v[5], v[6], v[7]));
+        __stcs(reinterpret_cast<uint4*>(a.w + e),
+               make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                          pack_bf16x2(p[6], p[7])));
+    }
+    const int64_t tail = (n8 << 3) + tid;
+    if (tail < a.n) scalar_elem<MODE>(a, tail);
+}
+
+// Scalar kernel: any element-aligned pointers.
+template <int MODE>
+__global__ void __launch_bounds__(kThreads) k_reduce_adamw_scalar(const __grid_constant__ K1Args a) {
+    const int64_t stride = int64_t(gridDim.x) * kThreads;
+    for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < a.n; i += stride)
+        scalar_elem<MODE>(a, i);
+}
+
+using KernelFn = void (*)(K1Args);
+
+template <int MODE>
+KernelFn pick_vec(int D) {
+    switch (D) {
+    case 1: return k_reduce_adamw_vec<MODE, 1>;
+    case 2: return k_reduce_adamw_vec<MODE, 2>;
+    case 4: return k_reduce_adamw_vec<MODE, 4>;
+    case 8: return k_reduce_adamw_vec<MODE, 8>;
+    case 16: return k_reduce_adamw_vec<MODE, 16>;
+    case 32: return k_reduce_adamw_vec<MODE, 32>;
+    default: return k_reduce_adamw_vec<MODE, 0>;
+    }
+}
+
+bool is_finite(double x) { return std::isfinite(x); }
+
+}  // namespace
+
+extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                         int32_t contrib_layout, float* master, float* exp_avg,
+                                         float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
+                                         const z3_adamw* hp, void* cuda_stream) {
+    // ---- arguments
+    if (p == nullptr || contrib == nullptr || hp == nullptr) return Z3_EINVAL;
+    const int32_t D = p->D;
+    if (rank < -1 || rank >= D) return Z3_EINVAL;
+    if (contrib_layout != Z3_CONTRIB_FULL && contrib_layout != Z3_CONTRIB_OWNED) return Z3_EINVAL;
+    if (contrib_layout == Z3_CONTRIB_OWNED && rank < 0) return Z3_EINVAL;
+    if (reduce_dtype != Z3_REDUCE_FP32 && reduce_dtype != Z3_REDUCE_BF16) return Z3_EINVAL;
+    if (master == nullptr || exp_avg == nullptr || exp_avg_sq == nullptr || work_bf16 == nullptr)
+        return Z3_EINVAL;
+    for (int32_t d = 0; d < D; ++d)
+        if (contrib[d] == nullptr) return Z3_EINVAL;
+    if (hp->step < 1 || !is_finite(hp->lr) || !is_finite(hp->beta1) || !is_finite(hp->beta2) ||
+        !is_finite(hp->eps) || !is_finite(hp->weight_decay) || hp->beta1 < 0.0 || hp->beta1 >= 1.0 ||
+        hp->beta2 < 0.0 || hp->beta2 >= 1.0)
+        return Z3_EINVAL;
+    if (!z3::aligned(master, 4) || !z3::aligned(exp_avg, 4) || !z3::aligned(exp_avg_sq, 4) ||
+        !z3::aligned(work_bf16, 2))
+        return Z3_EALIGN;
+    for (int32_t d = 0; d < D; ++d)
+        if (!z3::aligned(contrib[d], 2)) return Z3_EALIGN;
+
+    const int64_t n = rank < 0 ? p->N_pad : p->S;
+    // first element of the launch inside each contribution buffer
+    const int64_t c_off = (contrib_layout == Z3_CONTRIB_FULL && rank >= 0) ? int64_t(rank) * p->S : 0;
+
+    // ---- outputs must not overlap each other or any contribution they read
+    const int64_t fb = n * 4, hb = n * 2;
+    const void* outs[4] = {master, exp_avg, exp_avg_sq, work_bf16};
+    const int64_t out_bytes[4] = {fb, fb, fb, hb};
+    for (int x = 0; x < 4; ++x) {
+        for (int y = x + 1; y < 4; ++y)
+            if (z3::overlaps(outs[x], out_bytes[x], outs[y], out_bytes[y])) return Z3_EINVAL;
+        for (int32_t d = 0; d < D; ++d)
+            if (z3::overlaps(outs[x], out_bytes[x], contrib[d] + c_off, hb)) return Z3_EINVAL;
+    }
+    if (n == 0) return Z3_OK;
+
+    // ---- host scalars: double, then rounded to fp32 once
+    K1Args a;
+    const double t = double(hp->step);
+    const double bc1 = 1.0 - std::pow(hp->beta1, t);
+    const double bc2 = 1.0 - std::pow(hp->beta2, t);
+    a.s.step_size = float(hp->lr / bc1);
+    a.s.inv_sqrt_bc2 = float(1.0 / std::sqrt(bc2));
+    a.s.decay = float(1.0 - hp->lr * hp->weight_decay);
+    a.s.b1 = float(hp->beta1);
+    a.s.omb1 = float(1.0 - hp->beta1);
+    a.s.b2 = float(hp->beta2);
+    a.s.omb2 = float(1.0 - hp->beta2);
+    a.s.eps = float(hp->eps);
+    a.inv_D = float(1.0 / double(D));
+    a.D = D;
+    a.n = n;
+    a.p = master;
+    a.m = exp_avg;
+    a.v = exp_avg_sq;
+    a.w = work_bf16;
+    bool vec = z3::aligned(master, 16) && z3::aligned(exp_avg, 16) && z3::aligned(exp_avg_sq, 16) &&
+               z3::aligned(work_bf16, 16);
+    for (int32_t d = 0; d < Z3_D_MAX; ++d) {
+        a.c[d] = d < D ? contrib[d] + c_off : nullptr;
+        if (d < D && !z3::aligned(a.c[d], 16)) vec = false;
+    }
+
+    // ---- launch: a whole number of resident waves, grid-stride inside
+    KernelFn fn;
+    if (vec)
+        fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32>(D) : pick_vec<Z3_REDUCE_BF16>(D);
+    else
+        fn = reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32>
+                                            : k_reduce_adamw_scalar<Z3_REDUCE_BF16>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int sms = z3::sm_count();
+    if (sms < 1) return Z3_ECUDA;
+    const int64_t work_items = vec ? (n >> 3) : n;
+    int64_t blocks = (work_items + kThreads - 1) / kThreads;
+    const int64_t resident = int64_t(sms) * per_sm;
+    if (blocks > resident) blocks = resident;
+    if (blocks < 1) blocks = 1;  // the vector kernel's scalar tail still needs one block
+    fn<<<dim3(unsigned(blocks)), dim3(kThreads), 0, static_cast<cudaStream_t>(cuda_stream)>>>(a);
+    return cudaGetLastError() == cudaSuccess ? Z3_OK : Z3_ECUDA;
+}

@@ -1,0 +1,237 @@
+"""Python binding of libzero3.so (the C ABI declared in include/zero3.h).
+
+Argument marshalling only: torch tensors are turned into device pointers,
+sizes are checked against the plan (the C ABI sees plain pointers and cannot
+check extents), the tensors' device is made current and the call is enqueued
+on the given (default: torch's current) stream.  Every step of the path runs
+in the library's CUDA kernels; there is no fallback.  If the library is not
+built, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libzero3.so")
+
+Z3_OK, Z3_EINVAL, Z3_EALIGN, Z3_ENOMEM, Z3_ECUDA, Z3_EOVERFLOW = 0, -1, -2, -3, -4, -5
+Z3_D_MAX = 64
+Z3_REDUCE_FP32, Z3_REDUCE_BF16 = 0, 1
+Z3_CONTRIB_FULL, Z3_CONTRIB_OWNED = 0, 1
+Z3_STAGE_DDP, Z3_STAGE_ZERO1, Z3_STAGE_ZERO2, Z3_STAGE_ZERO3 = 0, 1, 2, 3
+
+
+class TensorSpec(C.Structure):
+    _fields_ = [("numel", C.c_int64), ("ndim", C.c_int32), ("shape", C.c_int64 * 4)]
+
+
+class AdamW(C.Structure):
+    _fields_ = [("lr", C.c_double), ("beta1", C.c_double), ("beta2", C.c_double),
+                ("eps", C.c_double), ("weight_decay", C.c_double), ("step", C.c_int64)]
+
+
+class Zero3Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load() -> C.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python -m fsdp_sharded_mixed_flat_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    vp, i32, i64 = C.c_void_p, C.c_int32, C.c_int64
+    L.zero3_status_string.argtypes = [C.c_int]
+    L.zero3_status_string.restype = C.c_char_p
+    L.zero3_plan.argtypes = [C.POINTER(TensorSpec), i32, i32, i32, C.POINTER(vp)]
+    L.zero3_plan.restype = C.c_int
+    L.zero3_plan_free.argtypes = [vp]
+    L.zero3_plan_free.restype = None
+    L.zero3_plan_info.argtypes = [vp, C.POINTER(i32), C.POINTER(i32), C.POINTER(i32),
+                                  C.POINTER(i64), C.POINTER(i64), C.POINTER(i64)]
+    L.zero3_plan_info.restype = C.c_int
+    L.zero3_plan_tensor.argtypes = [vp, i32, C.POINTER(i64), C.POINTER(i64)]
+    L.zero3_plan_tensor.restype = C.c_int
+    L.zero3_plan_rank.argtypes = [vp, i32, C.POINTER(i64), C.POINTER(i64)]
+    L.zero3_plan_rank.restype = C.c_int
+    L.zero3_memory_bytes.argtypes = [i64, i32, i32, C.POINTER(i64)]
+    L.zero3_memory_bytes.restype = C.c_int
+    L.zero3_transient_bytes.argtypes = [i64, i32, C.POINTER(i64)]
+    L.zero3_transient_bytes.restype = C.c_int
+    L.zero3_reduce_adamw.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
+    L.zero3_reduce_adamw.restype = C.c_int
+    L.zero3_gather_block.argtypes = [vp, vp, vp, vp, vp]
+    L.zero3_gather_block.restype = C.c_int
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> C.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.zero3_status_string(status).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != Z3_OK:
+        raise Zero3Error(rc, what)
+
+
+# ------------------------------------------------------------------- plan
+class Plan:
+    """A flat-parameter plan (owns the C plan object)."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], D: int, align_elems: int = 128):
+        self.shapes = [tuple(int(x) for x in s) for s in shapes]
+        n = len(self.shapes)
+        specs = (TensorSpec * max(1, n))()
+        for i, s in enumerate(self.shapes):
+            if len(s) > 4:
+                raise ValueError("at most 4 dimensions per tensor")
+            numel = 1
+            for x in s:
+                numel *= x
+            specs[i].numel = numel
+            specs[i].ndim = len(s)
+            for k, x in enumerate(s):
+                specs[i].shape[k] = x
+        h = C.c_void_p()
+        _check(_lib.zero3_plan(specs, n, D, align_elems, C.byref(h)), "zero3_plan")
+        self._h = h
+        d, nt, a = C.c_int32(), C.c_int32(), C.c_int32()
+        N, N_pad, S = C.c_int64(), C.c_int64(), C.c_int64()
+        _check(_lib.zero3_plan_info(h, C.byref(d), C.byref(nt), C.byref(a), C.byref(N),
+                                    C.byref(N_pad), C.byref(S)), "zero3_plan_info")
+        self.D, self.n_tensors, self.align_elems = d.value, nt.value, a.value
+        self.N, self.N_pad, self.S = N.value, N_pad.value, S.value
+        self.offsets, self.numels = [], []
+        for i in range(n):
+            self.offsets.append(zero3_plan_tensor(self, i)[0])
+            self.numels.append(zero3_plan_tensor(self, i)[1])
+
+    @property
+    def handle(self) -> C.c_void_p:
+        return self._h
+
+    def rank_range(self, r: int):
+        return zero3_plan_rank(self, r)
+
+    def views(self, flat: torch.Tensor):
+        """Zero-copy per-tensor views of a gathered flat block (the unflatten)."""
+        if flat.numel() < self.N_pad:
+            raise ValueError("flat block smaller than N_pad")
+        return [flat[o:o + k].view(s) for o, k, s in zip(self.offsets, self.numels, self.shapes)]
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.zero3_plan_free(h)
+            self._h = None
+
+
+def zero3_plan(shapes, D: int, align_elems: int = 128) -> Plan:
+    return Plan(shapes, D, align_elems)
+
+
+def zero3_plan_tensor(plan: Plan, i: int):
+    off, n = C.c_int64(), C.c_int64()
+    _check(_lib.zero3_plan_tensor(plan.handle, i, C.byref(off), C.byref(n)), "zero3_plan_tensor")
+    return off.value, n.value
+
+
+def zero3_plan_rank(plan: Plan, r: int):
+    b, e = C.c_int64(), C.c_int64()
+    _check(_lib.zero3_plan_rank(plan.handle, r, C.byref(b), C.byref(e)), "zero3_plan_rank")
+    return b.value, e.value
+
+
+def zero3_memory_bytes(N: int, D: int, stage: int) -> int:
+    out = C.c_int64()
+    _check(_lib.zero3_memory_bytes(N, D, stage, C.byref(out)), "zero3_memory_bytes")
+    return out.value
+
+
+def zero3_transient_bytes(block_params: int, n_buffers: int = 1) -> int:
+    out = C.c_int64()
+    _check(_lib.zero3_transient_bytes(block_params, n_buffers, C.byref(out)), "zero3_transient_bytes")
+    return out.value
+
+
+# ------------------------------------------------------------- marshalling
+def adamw(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, step=1) -> AdamW:
+    return AdamW(lr, beta1, beta2, eps, weight_decay, step)
+
+
+def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < need:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {need}")
+    return t.data_ptr()
+
+
+def _stream_handle(stream, device) -> int:
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], master: torch.Tensor,
+                       exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor, work_bf16: torch.Tensor,
+                       hp: AdamW, contrib_layout: int = Z3_CONTRIB_FULL,
+                       reduce_dtype: int = Z3_REDUCE_FP32, stream=None) -> None:
+    """Fused reduce-scatter reduction + AdamW + bf16 cast (see include/zero3.h)."""
+    if len(contrib) != plan.D:
+        raise ValueError(f"need {plan.D} contributions, got {len(contrib)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * plan.D)()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    mp = _dev_tensor(master, torch.float32, n, "master")
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
+    wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
+    dev = master.device
+    with torch.cuda.device(dev):
+        rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
+                                     reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
+    _check(rc, "zero3_reduce_adamw")
+
+
+def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Optional[torch.Tensor] = None,
+                       tensor_out: Optional[Sequence[Optional[torch.Tensor]]] = None, stream=None) -> None:
+    """All-gather of the D bf16 shards into the flat block and/or per-tensor buffers."""
+    if len(shards) != plan.D:
+        raise ValueError(f"need {plan.D} shards, got {len(shards)}")
+    sp = (C.c_void_p * plan.D)()
+    for r, s in enumerate(shards):
+        sp[r] = _dev_tensor(s, torch.bfloat16, plan.S, f"shards[{r}]")
+    fp = None if flat_out is None else _dev_tensor(flat_out, torch.bfloat16, plan.N_pad, "flat_out")
+    tp = None
+    if tensor_out is not None:
+        if len(tensor_out) != plan.n_tensors:
+            raise ValueError(f"need {plan.n_tensors} tensor outputs, got {len(tensor_out)}")
+        tp = (C.c_void_p * max(1, plan.n_tensors))()
+        for i, t in enumerate(tensor_out):
+            tp[i] = None if t is None else _dev_tensor(t, torch.bfloat16, plan.numels[i], f"tensor_out[{i}]")
+    dev = shards[0].device
+    with torch.cuda.device(dev):
+        rc = _lib.zero3_gather_block(plan.handle, sp, fp, tp, _stream_handle(stream, dev))
+    _check(rc, "zero3_gather_block")

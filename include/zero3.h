@@ -1,0 +1,215 @@
+/*
+ * zero3.h -- C ABI of the B200 library for the per-rank arithmetic of one
+ * ZeRO-3 / FSDP training step, with D data-parallel ranks simulated on one GPU.
+ *
+ * Pages cited (by title and section):
+ *   [P1] "Distributed LLM Fine-Tuning at Scale: FSDP, ZeRO-3, and Multi-GPU
+ *         Orchestration"
+ *   [P2] "7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)"
+ *   [P3] "Building GPT from Scratch — Part 8: FSDP — When the Model Won't Fit"
+ *
+ * Conventions for every entry point
+ *   - Return value: Z3_OK (0) or a negative Z3_E* status.  No C++ exception
+ *     ever crosses this boundary.
+ *   - bf16 values are passed as uint16_t bit patterns.
+ *   - Device pointers are plain CUDA global-memory addresses on the current
+ *     device.  The caller owns and allocates every device buffer; the library
+ *     never allocates, frees or keeps device memory.  Host arrays of device
+ *     pointers (contrib, shards, tensor_out) are read during the call only.
+ *   - Device work is enqueued on `cuda_stream` (a cudaStream_t; NULL means the
+ *     legacy default stream) and the call returns without synchronising.
+ *     Argument and alignment errors are reported synchronously, before any
+ *     device work is enqueued; a failed launch returns Z3_ECUDA; errors that
+ *     happen while the kernels run surface at the caller's next synchronise.
+ *   - Outputs must not overlap inputs or each other unless stated (the
+ *     optimiser state is updated in place, which is the one sanctioned
+ *     input/output pairing).  Overlaps the library can see are rejected with
+ *     Z3_EINVAL.
+ *   - Element counts are int64_t; a plan may describe up to 2^62 elements.
+ *   - A plan is an immutable host object: it can be shared between threads
+ *     and streams, and must outlive the calls that use it.
+ */
+#ifndef ZERO3_H
+#define ZERO3_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define Z3_API __attribute__((visibility("default")))
+#else
+#define Z3_API
+#endif
+
+/* ----------------------------------------------------------------- status */
+enum {
+    Z3_OK = 0,
+    Z3_EINVAL = -1,    /* a NULL pointer, a value out of range, overlapping buffers */
+    Z3_EALIGN = -2,    /* a pointer not aligned to its element size */
+    Z3_ENOMEM = -3,    /* host allocation failed (the plan object) */
+    Z3_ECUDA = -4,     /* a CUDA runtime call or kernel launch failed */
+    Z3_EOVERFLOW = -5  /* a size does not fit in int64_t */
+};
+
+/* Largest number of simulated ranks D one call accepts. */
+#define Z3_D_MAX 64
+
+/* Reduce dtype, the MixedPrecision policy's reduce_dtype ([P1] §2 uses
+ * bfloat16; [P3] "Mixed Precision: Cutting Memory in Half" uses float32). */
+enum {
+    Z3_REDUCE_FP32 = 0, /* fp32 accumulator: each partial sum rounded to fp32 */
+    Z3_REDUCE_BF16 = 1  /* bf16 accumulator: each partial sum rounded to bf16 */
+};
+
+/* Layout of the D gradient contributions handed to zero3_reduce_adamw. */
+enum {
+    Z3_CONTRIB_FULL = 0, /* contrib[d] spans the whole padded block [0, N_pad);
+                            rank r's owned element j is contrib[d][r*S + j] */
+    Z3_CONTRIB_OWNED = 1 /* contrib[d] starts at rank r's partition: element j is
+                            contrib[d][j] (only with one rank per call) */
+};
+
+/* Stages of the memory ledger ([P2] §2). */
+enum { Z3_STAGE_DDP = 0, Z3_STAGE_ZERO1 = 1, Z3_STAGE_ZERO2 = 2, Z3_STAGE_ZERO3 = 3 };
+
+/* One tensor of a flat-parameter block: `ndim` sizes in `shape` (row-major,
+ * 0 <= ndim <= 4; ndim = 0 is a scalar), whose product must equal `numel`. */
+typedef struct {
+    int64_t numel;
+    int32_t ndim;
+    int64_t shape[4];
+} z3_tensor_spec;
+
+/* AdamW hyper-parameters for one optimiser step.  `step` is the 1-based step
+ * count t used for the bias corrections. */
+typedef struct {
+    double lr, beta1, beta2, eps, weight_decay;
+    int64_t step;
+} z3_adamw;
+
+/* Opaque host-side plan of one flat-parameter block. */
+typedef struct z3_plan z3_plan;
+
+/* Text for a status code (a static string; never NULL). */
+Z3_API const char* zero3_status_string(int status);
+
+/* ------------------------------------------------------------------ plan
+ * zero3_plan: lay a block's tensors out as one flat buffer and partition it
+ * over D ranks.  [P2] §3: rank r owns a partition P_r of roughly 1/D of the
+ * parameters; [P2] §5.1 and [P1] §2: the unit of sharding is one block (one
+ * wrapped transformer layer), gathered whole before it runs.
+ *   Layout: tensors packed row-major in list order with no gaps; the tail is
+ *   zero-padded so that N_pad = ceil(N / (D*A)) * D*A; every rank owns
+ *   S = N_pad / D elements, P_r = [r*S, (r+1)*S).  align_elems = A >= 1;
+ *   A = 128 keeps every partition 256-byte aligned in bf16 and 512-byte
+ *   aligned in fp32, which the vectorised kernels need (A*D % 8 == 0).
+ *   t: host array of n_tensors specs (may be NULL when n_tensors == 0).
+ *   *out: receives a new plan; release it with zero3_plan_free.
+ * Errors: Z3_EINVAL (n_tensors < 0, D outside [1, Z3_D_MAX], A < 1, a spec
+ * with numel < 0, ndim outside [0,4] or a shape product != numel, out NULL),
+ * Z3_EOVERFLOW (N_pad beyond 2^62), Z3_ENOMEM. */
+Z3_API int zero3_plan(const z3_tensor_spec* t, int32_t n_tensors, int32_t D, int32_t align_elems,
+                      z3_plan** out);
+Z3_API void zero3_plan_free(z3_plan* p);
+
+/* Sizes of a plan; any output pointer may be NULL.  N = real elements,
+ * N_pad = padded elements, S = elements per rank. */
+Z3_API int zero3_plan_info(const z3_plan* p, int32_t* D, int32_t* n_tensors, int32_t* align_elems,
+                           int64_t* N, int64_t* N_pad, int64_t* S);
+
+/* Tensor i's run in the flat block: elements [*offset, *offset + *numel).
+ * This is the unflatten of [P2] §5.1 ("full_params" used as the block's
+ * tensors): a view of tensor i is the flat block at that offset, reshaped to
+ * its row-major shape.  Errors: Z3_EINVAL (p NULL or i out of range). */
+Z3_API int zero3_plan_tensor(const z3_plan* p, int32_t i, int64_t* offset, int64_t* numel);
+
+/* Rank r's partition: *begin = r*S; *end_real = min((r+1)*S, N), never below
+ * *begin.  Elements [*end_real, *begin + S) are tail padding.
+ * Errors: Z3_EINVAL (p NULL or r outside [0, D)). */
+Z3_API int zero3_plan_rank(const z3_plan* p, int32_t r, int64_t* begin, int64_t* end_real);
+
+/* ---------------------------------------------------------- memory ledger
+ * Bytes per device for N parameters over D ranks ([P2] §2, per-stage
+ * formulas): 2 B of bf16 weights, about 6 B of gradient (bf16 with an fp32
+ * accumulator) and 12 B of fp32 master + m + v per parameter;
+ *   stage 0 (pure DP)  20 N
+ *   stage 1 (ZeRO-1)   12 N / D + 2 N + 6 N
+ *   stage 2 (ZeRO-2)   (12 + 6) N / D + 2 N
+ *   stage 3 (ZeRO-3)   20 N / D
+ * Each term that divides by D is rounded up to a whole byte.
+ * Errors: Z3_EINVAL (N < 0, D < 1, unknown stage, bytes NULL), Z3_EOVERFLOW. */
+Z3_API int zero3_memory_bytes(int64_t N, int32_t D, int32_t stage, int64_t* bytes);
+
+/* Transient bytes for gathered blocks ([P2] §5.2): one gathered block of
+ * block_params bf16 values takes 2 * block_params bytes, and n_buffers of
+ * them are live at once (two when the next block's gather overlaps).
+ * Errors: Z3_EINVAL (negative argument, bytes NULL), Z3_EOVERFLOW. */
+Z3_API int zero3_transient_bytes(int64_t block_params, int32_t n_buffers, int64_t* bytes);
+
+/* ------------------------------------------- reduce-scatter + AdamW + cast
+ * zero3_reduce_adamw: one fused pass over the owned partition(s):
+ *   1. reduce-scatter's reduction ([P3] "AllGather vs AllReduce": rank r
+ *      receives the sum of the r-th slice of every rank's gradient; [P2] §4):
+ *      g = (c_0 + c_1 + ... + c_{D-1}) * (1/D), summed left to right in rank
+ *      order in the reduce dtype (Z3_REDUCE_FP32 or Z3_REDUCE_BF16), the 1/D
+ *      factor being the fp32 constant nearest 1/D;
+ *   2. AdamW on the owned fp32 master / m / v ([P2] §3: rank r updates only
+ *      P_r from its local fp32 master, m, v and its gradient slice), in place:
+ *        p = p*(1 - lr*wd);  m = b1*m + (1-b1)*g;  v = b2*v + (1-b2)*g*g;
+ *        p = p - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps)
+ *      with each scalar factor formed in double and rounded to fp32 once and
+ *      each array operation one fp32 operation rounded to nearest-even;
+ *   3. the cast of the new master to the bf16 working shard ([P3] "Mixed
+ *      Precision"; [P1] §2 param_dtype=bfloat16), round-to-nearest-even.
+ *
+ *   p      plan of the block.
+ *   rank   r in [0, D) runs rank r's partition; -1 runs every rank in one
+ *          launch (state arrays then hold all D partitions back to back).
+ *   contrib host array of D device pointers, the ranks' bf16 gradient
+ *          contributions in `contrib_layout` (Z3_CONTRIB_OWNED needs rank >= 0).
+ *   master, exp_avg, exp_avg_sq  device fp32, S elements (N_pad if rank = -1),
+ *          read and updated in place.
+ *   work_bf16 device bf16 output, same extent as master.
+ *   reduce_dtype  Z3_REDUCE_FP32 or Z3_REDUCE_BF16.
+ *   hp     host struct; hp->step >= 1, all values finite.
+ *   cuda_stream  stream to enqueue on.
+ * Pad elements are processed like real ones: a zero master with zero
+ * contributions stays exactly zero.
+ * Alignment: every pointer must be aligned to its element size (Z3_EALIGN
+ * otherwise).  When every contribution (at its partition offset), master,
+ * m, v and work_bf16 is 16-byte aligned the kernel moves 16-byte vectors;
+ * otherwise it falls back to a scalar kernel with the same results.
+ * Errors: Z3_EINVAL, Z3_EALIGN, Z3_ECUDA (launch failed). */
+Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                              int32_t contrib_layout, float* master, float* exp_avg,
+                              float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
+                              const z3_adamw* hp, void* cuda_stream);
+
+/* ------------------------------------------------ all-gather + unflatten
+ * zero3_gather_block: the all-gather's data movement ([P3] "AllGather vs
+ * AllReduce": GPU r holds shard r; afterwards every GPU holds [A, B, C, D];
+ * [P2] §5.1: full_params = all_gather(local_shard) before the block runs) and
+ * the optional unflatten into separate per-tensor buffers.
+ *   shards     host array of D device pointers, shard r = rank r's S bf16
+ *              working weights.
+ *   flat_out   device bf16, N_pad elements: flat_out[r*S + j] = shards[r][j].
+ *              May be NULL when tensor_out is given.
+ *   tensor_out host array of n_tensors device pointers, or NULL: tensor i's
+ *              buffer receives its numel elements (flat elements
+ *              [offset_i, offset_i + numel_i)), read straight from the shards.
+ *              An entry may be NULL to skip that tensor.
+ * Zero-copy views need no call: zero3_plan_tensor gives each tensor's offset
+ * in flat_out.  The vector path needs S % 8 == 0 and 16-byte aligned
+ * pointers; otherwise a scalar kernel gives the same bytes.
+ * Errors: Z3_EINVAL (both outputs NULL, a NULL shard), Z3_EALIGN, Z3_ECUDA. */
+Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
+                              uint16_t* const* tensor_out, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO3_H */

@@ -1,0 +1,224 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads and exports
+every entry point include/zero3.h declares, the planner and the memory ledger
+agree with the oracle, and every argument error is reported before any device
+work.  No call here reaches a CUDA API: each one either fails validation or
+has nothing to do (an empty plan)."""
+import ctypes as C
+import math
+import os
+import random
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from fsdp_sharded_mixed_flat_b200 import build as pkg_build
+
+pkg_build.build()
+from fsdp_sharded_mixed_flat_b200 import zero3 as z3  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zero3.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"Z3_API\s+[\w\s\*]+?\b(zero3_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
+                            "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
+                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_gather_block"]), names
+    out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(z3.lib(), n)
+    # nothing else of ours (and none of the static CUDA runtime) leaks out
+    leaked = sorted(s for s in exported if s.startswith("cuda") or s.startswith("_ZN"))
+    assert not leaked, leaked[:10]
+
+
+def test_status_strings():
+    for s in (0, -1, -2, -3, -4, -5):
+        assert z3.status_string(s) and z3.status_string(s) != "unknown status"
+    assert z3.status_string(-99) == "unknown status"
+
+
+# ------------------------------------------------------------------ planner
+def test_plan_matches_oracle_brute_force():
+    rnd = random.Random(5)
+    for _ in range(300):
+        shapes = [tuple(rnd.randint(1, 9) for _ in range(rnd.randint(0, 4))) for _ in range(rnd.randint(0, 8))]
+        D = rnd.randint(1, 64)
+        A = rnd.choice([1, 2, 3, 8, 16, 128, 1000])
+        p = z3.zero3_plan(shapes, D, A)
+        numels = [int(np.prod(s)) if s else 1 for s in shapes]
+        offs, N, N_pad, S = oracle.plan(numels, D, A)
+        assert (p.N, p.N_pad, p.S, p.D, p.align_elems, p.n_tensors) == (N, N_pad, S, D, A, len(shapes))
+        assert p.offsets == list(offs) and p.numels == numels
+        for r in range(D):
+            assert p.rank_range(r) == oracle.rank_range(N, S, r)
+
+
+def test_plan_workloads_match_oracle():
+    for name, w in synth.WORKLOADS.items():
+        D = w["D"]
+        p = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
+        offs, N, N_pad, S = oracle.plan([synth.numel(s) for _, s in w["tensors"]], D, synth.ALIGN)
+        assert (p.N, p.N_pad, p.S) == (N, N_pad, S) and p.offsets == list(offs)
+
+
+def test_plan_errors():
+    with pytest.raises(z3.Zero3Error) as e:
+        z3.zero3_plan([(3,)], 0)
+    assert e.value.status == z3.Z3_EINVAL
+    for bad in [dict(D=65), dict(D=1, align_elems=0), dict(D=-1)]:
+        with pytest.raises(z3.Zero3Error):
+            z3.zero3_plan([(3,)], **bad)
+    # shape product must equal numel
+    spec = (z3.TensorSpec * 1)()
+    spec[0].numel, spec[0].ndim = 7, 2
+    spec[0].shape[0], spec[0].shape[1] = 2, 3
+    h = C.c_void_p()
+    assert z3.lib().zero3_plan(spec, 1, 2, 1, C.byref(h)) == z3.Z3_EINVAL
+    spec[0].numel, spec[0].ndim = 6, 5
+    assert z3.lib().zero3_plan(spec, 1, 2, 1, C.byref(h)) == z3.Z3_EINVAL
+    spec[0].numel, spec[0].ndim = -1, 0
+    assert z3.lib().zero3_plan(spec, 1, 2, 1, C.byref(h)) == z3.Z3_EINVAL
+    assert z3.lib().zero3_plan(spec, 1, 2, 1, None) == z3.Z3_EINVAL
+    # overflow: N itself beyond 2^62, and a padded size beyond 2^62 (2^62 - 1 = 3 mod 7)
+    two = (z3.TensorSpec * 2)()
+    for k in range(2):
+        two[k].numel, two[k].ndim, two[k].shape[0] = 2 ** 61 + 1, 1, 2 ** 61 + 1
+    assert z3.lib().zero3_plan(two, 2, 1, 1, C.byref(h)) == z3.Z3_EOVERFLOW
+    spec[0].numel, spec[0].ndim = 2 ** 62 - 1, 1
+    spec[0].shape[0] = 2 ** 62 - 1
+    assert z3.lib().zero3_plan(spec, 1, 7, 1, C.byref(h)) == z3.Z3_EOVERFLOW
+    assert z3.lib().zero3_plan(spec, 1, 3, 1, C.byref(h)) == z3.Z3_OK
+    z3.lib().zero3_plan_free(h)
+    p = z3.zero3_plan([(3,)], 2)
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_plan_tensor(p, 1)
+    with pytest.raises(z3.Zero3Error):
+        p.rank_range(2)
+
+
+def test_plan_scalar_and_empty():
+    p = z3.zero3_plan([(), (4,)], 2, 1)
+    assert p.numels == [1, 4] and p.N == 5 and p.N_pad == 6 and p.S == 3
+    e = z3.zero3_plan([], 4, 128)
+    assert (e.N, e.N_pad, e.S) == (0, 0, 0)
+
+
+# ------------------------------------------------------------------- ledger
+def test_memory_bytes_matches_oracle():
+    rnd = random.Random(9)
+    cases = [(7_000_000_000, 32), (70_000_000_000, 8), (202_383_360, 8), (1, 1), (0, 5)]
+    cases += [(rnd.randint(0, 10 ** 13), rnd.randint(1, 4096)) for _ in range(200)]
+    for N, D in cases:
+        for stage in range(4):
+            got = z3.zero3_memory_bytes(N, D, stage)
+            ref = oracle.memory_bytes(N, D, stage)
+            # the ABI rounds each sharded term up to a whole byte; the oracle is real-valued
+            assert ref - 1e-6 * max(1.0, ref) <= got <= ref + 1 + 1e-6 * max(1.0, ref), (N, D, stage)
+            if (20 * N) % D == 0 and (12 * N) % D == 0 and (18 * N) % D == 0:
+                assert got == round(ref)
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_memory_bytes(10, 2, 4)
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_memory_bytes(-1, 2, 3)
+    with pytest.raises(z3.Zero3Error) as e:
+        z3.zero3_memory_bytes(2 ** 62, 2, 0)
+    assert e.value.status == z3.Z3_EOVERFLOW
+
+
+def test_transient_bytes_matches_oracle():
+    for block in (0, 1, 12 * 4096 * 4096, 855_654_400):
+        for nb in (0, 1, 2):
+            assert z3.zero3_transient_bytes(block, nb) == oracle.transient_bytes(block, nb)
+
+
+# ------------------------------------------- argument errors, no device work
+P16 = 0x10000  # fake, 16-byte aligned device addresses: never dereferenced here
+
+
+def call_reduce(plan, rank=-1, contrib=None, layout=0, ptrs=None, mode=0, hp=None):
+    D = plan.D
+    if contrib is None:
+        contrib = [P16 * (100 + d) for d in range(D)]
+    arr = (C.c_void_p * max(1, D))(*contrib)
+    ptrs = ptrs or [P16 * 1, P16 * 2, P16 * 3, P16 * 4]
+    hp = hp or z3.adamw(step=1)
+    return z3.lib().zero3_reduce_adamw(plan.handle, rank, arr, layout, *[C.c_void_p(x) for x in ptrs],
+                                       mode, C.byref(hp), None)
+
+
+def test_reduce_adamw_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)   # S = 256 elements = 1 KiB fp32
+    E = z3.Z3_EINVAL
+    assert call_reduce(p, rank=4) == E
+    assert call_reduce(p, rank=-2) == E
+    assert call_reduce(p, layout=1) == E                     # owned layout needs one rank
+    assert call_reduce(p, layout=7, rank=0) == E
+    assert call_reduce(p, mode=2) == E
+    assert call_reduce(p, contrib=[P16, 0, P16 * 3, P16 * 4]) == E
+    assert call_reduce(p, ptrs=[0, P16 * 2, P16 * 3, P16 * 4]) == E
+    assert call_reduce(p, hp=z3.adamw(step=0)) == E
+    assert call_reduce(p, hp=z3.adamw(beta1=1.0)) == E
+    assert call_reduce(p, hp=z3.adamw(lr=float("nan"))) == E
+    assert call_reduce(p, hp=z3.adamw(eps=float("inf"))) == E
+    assert z3.lib().zero3_reduce_adamw(None, 0, None, 0, None, None, None, None, 0, None, None) == E
+    # misaligned: fp32 state off a 4-byte boundary, bf16 off a 2-byte boundary
+    assert call_reduce(p, ptrs=[P16 + 2, P16 * 2, P16 * 3, P16 * 4]) == z3.Z3_EALIGN
+    assert call_reduce(p, ptrs=[P16, P16 * 2, P16 * 3, P16 * 4 + 1]) == z3.Z3_EALIGN
+    assert call_reduce(p, contrib=[P16 * 100 + 1] + [P16 * 101] * 3) == z3.Z3_EALIGN
+    # overlapping outputs, and an output over a contribution it reads
+    n_bytes = p.N_pad * 4
+    assert call_reduce(p, ptrs=[P16 * 10, P16 * 10 + n_bytes - 4, P16 * 30, P16 * 40]) == E
+    assert call_reduce(p, contrib=[P16 * 40] * 4, ptrs=[P16 * 10, P16 * 20, P16 * 30, P16 * 40]) == E
+    # rank 1 reads contributions at [S, 2S): an output over that range is rejected
+    S = p.S
+    base = P16 * 1000
+    assert call_reduce(p, rank=1, contrib=[base] * 4, ptrs=[base + 2 * S, P16 * 20, P16 * 30, P16 * 40]) == E
+
+
+def test_reduce_adamw_empty_plan_is_a_no_op():
+    p = z3.zero3_plan([], 4, 128)
+    assert call_reduce(p) == z3.Z3_OK
+    assert call_reduce(p, rank=2) == z3.Z3_OK
+
+
+def call_gather(plan, shards=None, flat=P16 * 500, tensor_out=None):
+    D = plan.D
+    shards = shards if shards is not None else [P16 * (100 + 10 * r) for r in range(D)]
+    sa = (C.c_void_p * max(1, D))(*shards)
+    ta = None
+    if tensor_out is not None:
+        ta = (C.c_void_p * max(1, len(tensor_out)))(*tensor_out)
+    return z3.lib().zero3_gather_block(plan.handle, sa, None if flat is None else C.c_void_p(flat), ta, None)
+
+
+def test_gather_block_argument_errors():
+    p = z3.zero3_plan([(64,), (64,)], 4, 8)
+    E = z3.Z3_EINVAL
+    assert call_gather(p, flat=None) == E
+    assert call_gather(p, shards=[P16, 0, P16 * 3, P16 * 4]) == E
+    assert call_gather(p, shards=[P16 + 1, P16 * 2, P16 * 3, P16 * 4]) == z3.Z3_EALIGN
+    assert call_gather(p, flat=P16 * 500 + 1) == z3.Z3_EALIGN
+    assert call_gather(p, flat=None, tensor_out=[P16 * 700 + 1, 0]) == z3.Z3_EALIGN
+    assert call_gather(p, flat=P16 * 100) == E                    # flat over shard 0
+    assert call_gather(p, flat=None, tensor_out=[P16 * 700, P16 * 700 + 2]) == E   # tensors overlap
+    assert call_gather(p, tensor_out=[P16 * 500, 0]) == E         # tensor over flat
+    assert z3.lib().zero3_gather_block(None, None, None, None, None) == E
+
+
+def test_gather_empty_plan_is_a_no_op():
+    p = z3.zero3_plan([(0,)], 2, 8)
+    assert call_gather(p) == z3.Z3_OK

@@ -1,0 +1,240 @@
+"""GPU parity of the fused reduce-scatter + AdamW + bf16-cast kernel against the
+oracle, called through the C ABI, on the same seeded inputs.
+
+Small cases (seconds for the oracle) span several 8-element chunks, thread
+blocks and ragged tails, every rank count class (1, powers of two, odd, the
+maximum 64), both contribution layouts, both reduce dtypes, single ranks and
+all ranks in one launch, and misaligned buffers (scalar path); every buffer
+sits between canary bands that must come back untouched.  Full-size cases run
+the workloads in the launch configuration the benchmark times and compare
+sampled elements (every element is independent of the others, so the oracle
+run on the gathered sample equals the full run at those indices).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from parity_util import (Guarded, assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp,
+                         state_init)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def z3():
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    from fsdp_sharded_mixed_flat_b200 import build
+    build.build()
+    from fsdp_sharded_mixed_flat_b200 import zero3
+    return zero3
+
+
+def run_small(z3, numels, D, A, rank, layout, mode, steps=10, seed=0, skew=(0, 0, 0, 0, 0),
+              dist="normal", sigma=1e-3, zero_frac=0.0):
+    plan = z3.zero3_plan([(k,) for k in numels], D, A)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    n = N_pad if rank < 0 else S
+    p_full, _, _ = state_init(N, N_pad, seed)
+    p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
+    gp = Guarded(n, torch.float32, skew[0], fill=p0)
+    gm = Guarded(n, torch.float32, skew[1], fill=torch.zeros(n, device="cuda"))
+    gv = Guarded(n, torch.float32, skew[2], fill=torch.zeros(n, device="cuda"))
+    gw = Guarded(n, torch.bfloat16, skew[3], fill=torch.zeros(n, device="cuda", dtype=torch.bfloat16))
+    hp_, hm, hv = f32_host(p0).copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+    hw = np.zeros(n, np.uint16)
+    for t in range(1, steps + 1):
+        contribs = synth.contributions(D, N, N_pad, seed=seed, step=t, sigma=sigma, dist=dist,
+                                       zero_frac=zero_frac, device="cuda")
+        if layout == z3.Z3_CONTRIB_OWNED:
+            contribs = [c[rank * S:(rank + 1) * S].clone() for c in contribs]
+        gc = [Guarded(c.numel(), torch.bfloat16, skew[4], fill=c) for c in contribs]
+        z3.zero3_reduce_adamw(plan, rank, [g.t for g in gc], gp.t, gm.t, gv.t, gw.t, z3.adamw(**hp_for(t)),
+                              contrib_layout=layout, reduce_dtype=mode)
+        oracle.reduce_adamw([synth.bf16_bits(c) for c in contribs], S, rank, hp_, hm, hv, hw, oracle_hp(t),
+                            layout=layout, reduce_dtype=mode)
+        torch.cuda.synchronize()
+        what = f"numels={numels} D={D} A={A} rank={rank} layout={layout} mode={mode} step={t}"
+        assert_f32_parity(f32_host(gp.t), hp_, "master " + what)
+        assert_f32_parity(f32_host(gm.t), hm, "exp_avg " + what)
+        assert_f32_parity(f32_host(gv.t), hv, "exp_avg_sq " + what)
+        assert_bf16_parity(synth.bf16_bits(gw.t), hw, "work_bf16 " + what)
+        for g in (gp, gm, gv, gw, *gc):
+            assert g.guards_intact(), "canary overwritten: " + what
+        for g, c in zip(gc, contribs):
+            assert torch.equal(g.t.view(torch.int16), c.view(torch.int16)), "contribution modified"
+    return plan
+
+
+SMALL = [
+    ([13], 1, 1), ([1], 8, 1), ([5, 7, 1], 4, 1), ([13], 3, 1), ([999], 5, 1),
+    ([300, 77, 1000], 4, 8), ([1000, 2000], 3, 8), ([4097, 33], 32, 128), ([123457], 8, 128),
+    ([2 ** 16 + 3], 64, 8), ([50000], 16, 1), ([70001], 2, 128), ([6000, 1, 2], 7, 16),
+]
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("numels,D,A", SMALL)
+def test_all_ranks_one_launch(z3, numels, D, A, mode):
+    run_small(z3, numels, D, A, -1, z3.Z3_CONTRIB_FULL, mode)
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("numels,D,A", SMALL)
+def test_single_rank_full_and_owned(z3, numels, D, A, mode):
+    run_small(z3, numels, D, A, D // 2, z3.Z3_CONTRIB_FULL, mode, steps=4)
+    run_small(z3, numels, D, A, D - 1, z3.Z3_CONTRIB_OWNED, mode, steps=4)
+
+
+@pytest.mark.parametrize("skew", [(1, 0, 0, 0, 0), (0, 0, 0, 1, 0), (0, 0, 0, 0, 1), (1, 1, 1, 1, 1),
+                                  (2, 0, 2, 0, 0)])
+def test_misaligned_buffers_take_the_scalar_path(z3, skew):
+    run_small(z3, [3000, 17], 4, 8, -1, z3.Z3_CONTRIB_FULL, 0, steps=3, skew=skew)
+    run_small(z3, [3000, 17], 4, 8, 1, z3.Z3_CONTRIB_OWNED, 1, steps=2, skew=skew)
+
+
+def test_heavy_tails_and_exact_zeros(z3):
+    for mode in (0, 1):
+        run_small(z3, [40000, 123], 8, 128, -1, z3.Z3_CONTRIB_FULL, mode, steps=5, dist="student_t",
+                  zero_frac=0.01)
+
+
+def test_integer_contributions_give_the_same_step_in_both_reduce_dtypes(z3):
+    """Exact partial sums: the bf16 and fp32 reductions must coincide."""
+    out = []
+    for mode in (0, 1):
+        plan = z3.zero3_plan([(4096,)], 8, 8)
+        p, m, v = state_init(plan.N, plan.N_pad, 1)
+        w = torch.zeros(plan.N_pad, dtype=torch.bfloat16, device="cuda")
+        c = synth.contributions(8, plan.N, plan.N_pad, seed=2, step=1, sigma=0, dist="integers", device="cuda")
+        z3.zero3_reduce_adamw(plan, -1, c, p, m, v, w, z3.adamw(step=1), reduce_dtype=mode)
+        out.append((p, m, v, w))
+    for a, b in zip(*out):
+        assert torch.equal(a.view(torch.int16 if a.dtype == torch.bfloat16 else torch.int32),
+                           b.view(torch.int16 if b.dtype == torch.bfloat16 else torch.int32))
+
+
+def test_pad_stays_exactly_zero(z3):
+    plan = run_small(z3, [1000 * 32 + 1], 32, 128, -1, z3.Z3_CONTRIB_FULL, 0, steps=3)
+    assert plan.N_pad - plan.N == 4095
+
+
+def test_empty_plan_and_stream_argument(z3):
+    plan = z3.zero3_plan([], 4, 128)
+    z = torch.zeros(16, device="cuda")
+    zb = torch.zeros(16, device="cuda", dtype=torch.bfloat16)
+    z3.zero3_reduce_adamw(plan, -1, [zb] * 4, z, z.clone(), z.clone(), zb.clone(), z3.adamw(step=1))
+    s = torch.cuda.Stream()
+    run_on = z3.zero3_plan([(4096,)], 2, 8)
+    p, m, v = state_init(run_on.N, run_on.N_pad, 3)
+    w = torch.zeros(run_on.N_pad, dtype=torch.bfloat16, device="cuda")
+    c = synth.contributions(2, run_on.N, run_on.N_pad, seed=3, step=1, sigma=1e-3, device="cuda")
+    torch.cuda.synchronize()
+    ref = [p.clone(), m.clone(), v.clone(), w.clone()]
+    with torch.cuda.stream(s):
+        z3.zero3_reduce_adamw(run_on, -1, c, p, m, v, w, z3.adamw(step=1))
+    z3.zero3_reduce_adamw(run_on, -1, c, *ref, z3.adamw(step=1), stream=torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert torch.equal(p, ref[0]) and torch.equal(w.view(torch.int16), ref[3].view(torch.int16))
+
+
+# ------------------------------------------------------------- full sizes
+def sample_indices(n: int, S: int, D: int, k: int, seed: int) -> torch.Tensor:
+    rng = np.random.default_rng(seed)
+    picks = [rng.choice(n, size=min(k, n), replace=False), np.arange(min(64, n)), np.arange(max(0, n - 64), n)]
+    for r in range(1, D):
+        picks.append(np.arange(max(0, r * S - 16), min(n, r * S + 16)))
+    return torch.from_numpy(np.unique(np.concatenate(picks))).cuda()
+
+
+def run_sampled(z3, workload: str, D: int, rank: int, layout: int, mode: int, steps: int,
+                k: int = 200_000, seed: int = 0):
+    w = synth.WORKLOADS[workload]
+    plan = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    n = N_pad if rank < 0 else S
+    p_full, _, _ = state_init(N, N_pad, seed)
+    p = (p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]).contiguous()
+    del p_full
+    m, v = torch.zeros_like(p), torch.zeros_like(p)
+    wk = torch.zeros(n, dtype=torch.bfloat16, device="cuda")
+    idx = sample_indices(n, S if rank < 0 else n, D if rank < 0 else 1, k, seed + 1)
+    hp_, hm, hv = f32_host(p[idx]).copy(), np.zeros(idx.numel(), np.float32), np.zeros(idx.numel(), np.float32)
+    hw = np.zeros(idx.numel(), np.uint16)
+    for t in range(1, steps + 1):
+        if layout == z3.Z3_CONTRIB_OWNED:
+            c = [synth.contribution(min(S, max(0, N - rank * S)), S, seed=seed, step=t, rank=d,
+                                    sigma=w["sigma"], dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
+                                    device="cuda") for d in range(D)]
+        else:
+            c = synth.contributions(D, N, N_pad, seed=seed, step=t, sigma=w["sigma"], dist=w["dist"],
+                                    zero_frac=w.get("zero_frac", 0.0), device="cuda")
+        z3.zero3_reduce_adamw(plan, rank, c, p, m, v, wk, z3.adamw(**hp_for(t)), contrib_layout=layout,
+                              reduce_dtype=mode)
+        base = 0 if (rank < 0 or layout == z3.Z3_CONTRIB_OWNED) else rank * S
+        sub = [synth.bf16_bits(x[idx + base]) for x in c]
+        oracle.reduce_adamw(sub, idx.numel(), 0, hp_, hm, hv, hw, oracle_hp(t), layout=oracle.LAYOUT_OWNED,
+                            reduce_dtype=mode)
+        del c
+    torch.cuda.synchronize()
+    what = f"{workload} D={D} rank={rank} mode={mode}"
+    assert_f32_parity(f32_host(p[idx]), hp_, "master " + what)
+    assert_f32_parity(f32_host(m[idx]), hm, "exp_avg " + what)
+    assert_f32_parity(f32_host(v[idx]), hv, "exp_avg_sq " + what)
+    assert_bf16_parity(synth.bf16_bits(wk[idx]), hw, "work_bf16 " + what)
+    return plan, p, m, v, wk
+
+
+def test_llama7b_block_d8_bench_configuration(z3):
+    """The benchmark's launch: all 8 ranks in one launch, full layout, fp32 reduce, 10 steps."""
+    run_sampled(z3, "llama7b_d8", 8, -1, z3.Z3_CONTRIB_FULL, 0, steps=10)
+
+
+def test_llama7b_block_d32_padded(z3):
+    plan, p, m, v, wk = run_sampled(z3, "llama7b_d32", 32, -1, z3.Z3_CONTRIB_FULL, 0, steps=10)
+    assert plan.N_pad - plan.N == 4095
+    for t in (p, m, v):
+        assert not t[plan.N:].any()
+    assert not wk[plan.N:].view(torch.int16).any()
+
+
+@pytest.mark.parametrize("D", [2, 4, 8, 16])
+def test_llama7b_policy_sweep_bf16_reduce(z3, D):
+    run_sampled(z3, "llama7b_policy", D, -1, z3.Z3_CONTRIB_FULL, 1, steps=3, k=100_000)
+
+
+def test_llama70b_layer_owned_rank(z3):
+    """One 70B layer's owned shard of rank 3 at D = 8, contributions in the owned layout."""
+    run_sampled(z3, "llama70b_layer", 8, 3, z3.Z3_CONTRIB_OWNED, 0, steps=2, k=100_000)
+
+
+def test_tiny_gpt_full_ten_steps_then_gather(z3):
+    """Config of the 3.3M-parameter GPT, every element compared, then the gather."""
+    w = synth.WORKLOADS["tiny_gpt"]
+    shapes = [s for _, s in w["tensors"]]
+    plan = z3.zero3_plan(shapes, w["D"], synth.ALIGN)
+    N, N_pad, S, D = plan.N, plan.N_pad, plan.S, plan.D
+    p, m, v = state_init(N, N_pad, 0)
+    wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
+        np.zeros(N_pad, np.uint16)
+    for t in range(1, 11):
+        c = synth.contributions(D, N, N_pad, seed=0, step=t, sigma=w["sigma"], device="cuda")
+        z3.zero3_reduce_adamw(plan, -1, c, p, m, v, wk, z3.adamw(**hp_for(t)))
+        oracle.reduce_adamw([synth.bf16_bits(x) for x in c], S, -1, hp_, hm, hv, hw, oracle_hp(t))
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(p), hp_, "master")
+    assert_f32_parity(f32_host(m), hm, "exp_avg")
+    assert_f32_parity(f32_host(v), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(wk), hw, "work_bf16")
+    flat = torch.empty(N_pad, dtype=torch.bfloat16, device="cuda")
+    outs = [torch.empty(s, dtype=torch.bfloat16, device="cuda") for s in shapes]
+    z3.zero3_gather_block(plan, [wk[r * S:(r + 1) * S] for r in range(D)], flat, outs)
+    torch.cuda.synchronize()
+    ref_flat = oracle.all_gather([hw[r * S:(r + 1) * S] for r in range(D)], S)
+    assert np.array_equal(synth.bf16_bits(flat), ref_flat)
+    ref_t = oracle.unflatten(ref_flat, plan.offsets, plan.numels)
+    for o, r, view in zip(outs, ref_t, plan.views(flat)):
+        assert np.array_equal(synth.bf16_bits(o).ravel(), r)
+        assert np.array_equal(synth.bf16_bits(view).ravel(), r)
