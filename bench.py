@@ -52,7 +52,7 @@ def parse_args():
     ap.add_argument("--workload", default="llama7b_d8")
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="elements of the oracle's sample")
-    ap.add_argument("--cpu-steps", type=int, default=8)
+    ap.add_argument("--cpu-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
