@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="elements of the oracle's sample")
     ap.add_argument("--cpu-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
+    ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
     return ap.parse_args()
 
 
@@ -161,7 +163,7 @@ def aggregate(local_seconds: float, local_units: float, world: int, device=None)
 
 
 # --------------------------------------------------------------- the oracle
-def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0):
+def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int = 0, reduce_dtype: int = 0):
     """Time the oracle over `steps` passes of a `sample`-element slice of the
     workload's owned elements (all D contributions, AdamW, cast).  Returns
     (owned params/s, seconds, description)."""
@@ -170,20 +172,25 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0):
 
     import oracle
     import synth
+    if workload == "llama70b_shard":
+        workload = "llama70b_layer"
     w = synth.WORKLOADS[workload]
-    D = w["D"]
+    D = D or w["D"]
     n = min(sample, synth.block_numel(w["tensors"]))
     contribs = [synth.bf16_bits(synth.contribution(n, n, seed=seed, step=1, rank=d, sigma=w["sigma"],
-                                                   dist=w["dist"], device="cpu")) for d in range(D)]
+                                                   dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
+                                                   device="cpu")) for d in range(D)]
     p = synth.master_weights(n, n, seed=seed).numpy().copy()
     m, v, wk = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
     oracle.lib()
     t0 = time.perf_counter()
     for t in range(1, steps + 1):
-        oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED)
+        oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED,
+                            reduce_dtype=reduce_dtype)
     dt = time.perf_counter() - t0
     del torch
-    desc = (f"{workload}: first {n} owned elements x {steps} steps, D={D}, one thread "
+    desc = (f"{workload}: first {n} owned elements x {steps} steps, D={D}, "
+            f"{'bf16' if reduce_dtype else 'fp32'} reduce, one thread "
             f"(oracle/zero3_ref.c, single-threaded C)")
     return n * steps / dt, dt, desc
 
@@ -195,13 +202,15 @@ def run_reference(args):
     steps = max(1, args.steps)
     # each step is a bounded sample (2^20 elements) so that K steps stay within minutes
     sample = min(args.cpu_sample, 1 << 20)
+    mode = 1 if args.reduce_dtype == "bf16" else 0
     if args.warmup > 0:
-        oracle_sample(args.workload, min(sample, 1 << 16), 1)
-    value, secs, desc = oracle_sample(args.workload, sample, steps)
+        oracle_sample(args.workload, min(sample, 1 << 16), 1, D=args.D, reduce_dtype=mode)
+    value, secs, desc = oracle_sample(args.workload, sample, steps, D=args.D, reduce_dtype=mode)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": {"workload": args.workload, "sample_elements": sample},
+            "data": "synthetic", "config": {"workload": args.workload, "sample_elements": sample,
+                                                      "D": args.D or None, "reduce_dtype": args.reduce_dtype},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -209,6 +218,139 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- our path
+class BlockRunner:
+    """One block, every rank's partition in one launch: plan + ledger (host),
+    fused reduce + AdamW + cast, gather into the flat block, zero-copy views."""
+
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev):
+        import torch
+        w = synth.WORKLOADS[workload]
+        self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
+        self.shapes = [s for _, s in w["tensors"]]
+        plan = z3.zero3_plan(self.shapes, D, synth.ALIGN)
+        self.N, self.N_pad, self.S = plan.N, plan.N_pad, plan.S
+        self.contribs = synth.contributions(D, self.N, self.N_pad, seed=seed, step=1, sigma=w["sigma"],
+                                            dist=w["dist"], zero_frac=w.get("zero_frac", 0.0), device=dev)
+        self.master = synth.master_weights(self.N, self.N_pad, seed=seed, device=dev)
+        self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
+        self.work = torch.zeros(self.N_pad, dtype=torch.bfloat16, device=dev)
+        self.flat = torch.empty(self.N_pad, dtype=torch.bfloat16, device=dev)
+        self.shards = [self.work[r * self.S:(r + 1) * self.S] for r in range(D)]
+        self.stream = torch.cuda.current_stream(dev)
+        self.step_no = 0
+        self.units_per_step = self.N_pad                       # owned params, all ranks
+        self.k1_launches_per_step = 1
+        self.k1_bytes_per_launch = (2 * D + 26) * self.N_pad
+        self.step_bytes = self.k1_bytes_per_launch + 4 * self.N_pad
+        self.launches_per_step = 2
+        self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}>"
+        self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
+                     f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
+                     f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + fused reduce/AdamW/cast over all "
+                     f"{D} partitions + gather into the flat block")
+
+    def hp(self):
+        a = self.synth.ADAMW
+        self.step_no += 1
+        return self.z3.adamw(lr=a["lr"], beta1=a["beta1"], beta2=a["beta2"], eps=a["eps"],
+                             weight_decay=a["weight_decay"], step=self.step_no)
+
+    def step(self, k1_events=None):
+        z3 = self.z3
+        # a1 + a2: host-side plan and ledger of the block (microseconds, overlapped with the GPU)
+        pl = z3.zero3_plan(self.shapes, self.D, self.synth.ALIGN)
+        z3.zero3_memory_bytes(pl.N, self.D, z3.Z3_STAGE_ZERO3)
+        hp = self.hp()
+        if k1_events is not None:
+            k1_events[0][0].record(self.stream)
+        # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
+        z3.zero3_reduce_adamw(pl, -1, self.contribs, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
+                              reduce_dtype=self.mode, stream=self.stream)
+        if k1_events is not None:
+            k1_events[0][1].record(self.stream)
+        # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
+        z3.zero3_gather_block(pl, self.shards, self.flat, None, stream=self.stream)
+        return pl.views(self.flat)
+
+    def e2e_setup(self):
+        import torch
+        self.host_c = [torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in range(self.D)]
+        for h, c in zip(self.host_c, self.contribs):
+            h.copy_(c)
+        self.host_flat = torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True)
+        return (sum(h.numel() * h.element_size() for h in self.host_c),
+                self.host_flat.numel() * self.host_flat.element_size())
+
+    def e2e_step(self):
+        for h, c in zip(self.host_c, self.contribs):
+            c.copy_(h, non_blocking=True)
+        self.step()
+        self.host_flat.copy_(self.flat, non_blocking=True)
+
+
+class ShardRunner:
+    """One rank's resident 70B shard (80 layers at D = 8): per step, the layers'
+    owned contributions stream in last to first through two transient buffers
+    (copy stream) while the fused kernel runs on the other buffer."""
+
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev):
+        import torch
+        from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
+        w = synth.WORKLOADS["llama70b_layer"]
+        self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
+        self.L = w["layers"]
+        plan = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
+        self.plan, self.S = plan, plan.S
+        S, L = self.S, self.L
+        self.master = torch.empty(L * S, dtype=torch.float32, device=dev)
+        for l in range(L):
+            self.master[l * S:(l + 1) * S] = synth.master_weights(S, S, seed=seed * 100 + l, device=dev)
+        self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
+        self.work = torch.zeros(L * S, dtype=torch.bfloat16, device=dev)
+        # the refill source: two layers' worth of owned contributions (what the reduce-scatter delivers)
+        self.pool = [torch.cat([synth.contribution(S, S, seed=seed, step=1, rank=d, sigma=w["sigma"], device=dev)
+                                for d in range(D)]) for _ in range(2)]
+        self.streamer = LayerStreamer(plan, L, 0, self.master, self.exp_avg, self.exp_avg_sq, self.work,
+                                      reduce_dtype=reduce_dtype)
+        self.stream = torch.cuda.current_stream(dev)
+        self.step_no = 0
+        self.units_per_step = L * S                            # owned params of this rank
+        self.k1_launches_per_step = L
+        self.k1_bytes_per_launch = (2 * D + 26) * S
+        self.refill_bytes = L * 2 * D * S * 2                  # D2D copy: read + write
+        self.step_bytes = L * self.k1_bytes_per_launch + self.refill_bytes
+        self.launches_per_step = L
+        self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}> (owned layout)"
+        self.source = lambda l: self.pool[l & 1]
+        self.desc = (f"rank 0's resident shard of 80 LLaMA-70B-shaped layers ({len(w['tensors'])} tensors, "
+                     f"855,654,400 params each), D={D}, S={S} per layer, {L * S} owned params "
+                     f"({L * S * 14 / 1e9:.1f} GB of master+m+v+bf16); per step the 80 layers' owned bf16 "
+                     f"contributions ({2 * D * S / 1e9:.2f} GB each) stream 79->0 through two transient buffers "
+                     f"(device-to-device refill on a copy stream) while the fused kernel runs")
+
+    def hp(self):
+        a = self.synth.ADAMW
+        self.step_no += 1
+        return self.z3.adamw(lr=a["lr"], beta1=a["beta1"], beta2=a["beta2"], eps=a["eps"],
+                             weight_decay=a["weight_decay"], step=self.step_no)
+
+    def step(self, k1_events=None):
+        self.streamer.step(self.source, self.hp(), k1_events)
+
+    def e2e_setup(self):
+        import torch
+        self.host_pool = [torch.empty_like(p, device="cpu").pin_memory() for p in self.pool]
+        for h, p in zip(self.host_pool, self.pool):
+            h.copy_(p)
+        self.host_out = torch.empty(self.S, dtype=torch.bfloat16, pin_memory=True)
+        return self.L * self.host_pool[0].numel() * 2, self.S * 2
+
+    def e2e_step(self):
+        # contributions come from pinned host memory layer by layer; layer 0's bf16 shard goes back
+        self.streamer.step(lambda l: self.host_pool[l & 1], self.hp())
+        self.host_out.copy_(self.work[:self.S], non_blocking=True)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -230,125 +372,86 @@ def run_ours(args):
     import synth
     from fsdp_sharded_mixed_flat_b200 import zero3 as z3
 
-    w = synth.WORKLOADS[args.workload]
-    shapes = [s for _, s in w["tensors"]]
-    D = w["D"]
-    plan = z3.zero3_plan(shapes, D, synth.ALIGN)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
     seed = 1000 + rank  # every rank runs its own block
-    contribs = synth.contributions(D, N, N_pad, seed=seed, step=1, sigma=w["sigma"], dist=w["dist"],
-                                   zero_frac=w.get("zero_frac", 0.0), device=dev)
-    master = synth.master_weights(N, N_pad, seed=seed, device=dev)
-    exp_avg, exp_avg_sq = torch.zeros_like(master), torch.zeros_like(master)
-    work = torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)
-    flat = torch.empty(N_pad, dtype=torch.bfloat16, device=dev)
-    shards = [work[r * S:(r + 1) * S] for r in range(D)]
-    stream = torch.cuda.current_stream(dev)
-    step_no = [0]
+    if args.workload == "llama70b_shard":
+        R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev)
+    else:
+        R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev)
+    stream = R.stream
 
-    def step(k1_events=None):
-        # a1 + a2: host-side plan and ledger of the block (microseconds, overlapped with the GPU)
-        pl = z3.zero3_plan(shapes, D, synth.ALIGN)
-        z3.zero3_memory_bytes(pl.N, D, z3.Z3_STAGE_ZERO3)
-        step_no[0] += 1
-        hp = z3.adamw(lr=w_adamw["lr"], beta1=w_adamw["beta1"], beta2=w_adamw["beta2"], eps=w_adamw["eps"],
-                      weight_decay=w_adamw["weight_decay"], step=step_no[0])
-        if k1_events is not None:
-            k1_events[0].record(stream)
-        # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
-        z3.zero3_reduce_adamw(pl, -1, contribs, master, exp_avg, exp_avg_sq, work, hp, stream=stream)
-        if k1_events is not None:
-            k1_events[1].record(stream)
-        # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
-        z3.zero3_gather_block(pl, shards, flat, None, stream=stream)
-        return pl.views(flat)
-
-    w_adamw = synth.ADAMW
     for _ in range(args.warmup):
-        step()
+        R.step()
     torch.cuda.synchronize(dev)
 
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else None)
     clocks.start()
-    k1_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-             for _ in range(args.steps)]
+    k1_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(R.k1_launches_per_step)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t0.record(stream)
     for i in range(args.steps):
-        step(k1_ev[i])
+        R.step(k1_ev[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
     secs = t0.elapsed_time(t1) / 1e3
-    k1_ms = [a.elapsed_time(b) for a, b in k1_ev]
+    k1_ms = [a.elapsed_time(b) for step_ev in k1_ev for a, b in step_ev]
     k1_avg_s = statistics.mean(k1_ms) / 1e3
-    job_secs, job_units = aggregate(secs, float(N_pad) * args.steps, world, dev)
+    job_secs, job_units = aggregate(secs, float(R.units_per_step) * args.steps, world, dev)
     value = job_units / job_secs
 
     # ---- end to end through the public API with host buffers
     e2e_steps = max(1, args.e2e_steps)
-    host_c = [torch.empty(N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in range(D)]
-    for h, c in zip(host_c, contribs):
-        h.copy_(c)
-    host_flat = torch.empty(N_pad, dtype=torch.bfloat16, pin_memory=True)
-    h2d = sum(h.numel() * h.element_size() for h in host_c)
-    d2h = host_flat.numel() * host_flat.element_size()
-
-    def e2e_step():
-        for h, c in zip(host_c, contribs):
-            c.copy_(h, non_blocking=True)
-        step()
-        host_flat.copy_(flat, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
+    h2d, d2h = R.e2e_setup()
+    for _ in range(1):
+        R.e2e_step()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        e2e_step()
+        R.e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_secs, e2e_units = aggregate(e0.elapsed_time(e1) / 1e3, float(N_pad) * e2e_steps, world, dev)
+    e2e_secs, e2e_units = aggregate(e0.elapsed_time(e1) / 1e3, float(R.units_per_step) * e2e_steps, world, dev)
 
     hbm_peak, peak_kind = measured_peaks()
-    bytes_per_param = 2 * D + 26
-    k1_gbs = bytes_per_param * N_pad / k1_avg_s / 1e9
-    step_bytes = bytes_per_param * N_pad + 4 * N_pad
+    k1_gbs = R.k1_bytes_per_launch / k1_avg_s / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: " + describe(args.workload, N, N_pad, S, D),
-                   "D": D, "N": N, "N_pad": N_pad, "S": S, "reduce_dtype": "fp32",
-                   "launch": "all D partitions in one launch (rank=-1), full contribution layout",
-                   "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (step_bytes / 1e9),
+        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D,
+                   "reduce_dtype": "bf16" if mode == z3.Z3_REDUCE_BF16 else "fp32",
+                   "owned_params_per_step": R.units_per_step,
+                   "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (R.step_bytes / 1e9),
                    "parallelism": f"replicas x{world} (one block per GPU, no collective)"},
-        "step_hbm_gbs": step_bytes * args.steps * world / job_secs / 1e9,
+        "step_hbm_gbs": R.step_bytes * args.steps * world / job_secs / 1e9,
         "kernels": {"reduce_adamw_ms": 1e3 * k1_avg_s, "reduce_adamw_gbs": k1_gbs,
-                    "reduce_adamw_params_per_s": N_pad / k1_avg_s,
-                    "gather_ms_est": max(0.0, 1e3 * secs / args.steps - 1e3 * k1_avg_s)},
+                    "reduce_adamw_params_per_s": (R.k1_bytes_per_launch / (2 * R.D + 26)) / k1_avg_s,
+                    "reduce_adamw_launches_per_step": R.k1_launches_per_step,
+                    "rest_of_step_ms": max(0.0, 1e3 * secs / args.steps - 1e3 * k1_avg_s * R.k1_launches_per_step)},
         "roofline": {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind,
-                     "kernel": "k_reduce_adamw_vec<fp32, D=8>",
-                     "algorithmic_bytes_per_launch": bytes_per_param * N_pad,
-                     "traffic": profiled_traffic()},
+                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
+                     "frac_of_nominal_8000": k1_gbs / 8000.0, "kernel": R.k1_name,
+                     "algorithmic_bytes_per_launch": R.k1_bytes_per_launch,
+                     "traffic": profiled_traffic() if args.workload == "llama7b_d8" and mode == 0 else None},
         "clocks": clk,
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": R.launches_per_step * args.steps,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, secs_cpu, desc = oracle_sample(args.workload, args.cpu_sample, args.cpu_steps)
+        v, secs_cpu, desc = oracle_sample(args.workload, args.cpu_sample, args.cpu_steps, D=R.D, reduce_dtype=mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                 "seconds": secs_cpu}
     if rank == 0:
@@ -357,14 +460,6 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
-
-
-def describe(name, N, N_pad, S, D):
-    import synth
-    w = synth.WORKLOADS[name]
-    return (f"{len(w['tensors'])} tensors, N={N}, N_pad={N_pad}, S={S} per rank, D={D}, "
-            f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
-            f"b=(0.9,0.95) eps=1e-8 wd=0.1")
 
 
 def main():

@@ -14,11 +14,14 @@
 // contributions and 12 bytes of state, and writes 12 bytes of state and 2
 // bytes of bf16 weights, against about 40 floating-point operations.  There is
 // no contraction, so no tensor-core work.  Each thread owns 8 consecutive
-// elements per iteration: one 16-byte load per rank, two per state array,
-// all issued before the arithmetic so that (D + 6) x 16 bytes per thread are
-// in flight; the ranks are folded in order 0..D-1 in chunks of 8 to bound
-// registers at large D.  Loads and stores use the streaming cache hint: every
-// byte is touched exactly once.  Every arithmetic step is an explicitly
+// elements: one 16-byte load per rank, two per state array, all issued before
+// the arithmetic so that (D + 6) x 16 bytes per thread are in flight; the
+// ranks are folded in order 0..D-1 in chunks of 8 to bound registers at large
+// D.  The grid covers the whole range rather than looping over a resident
+// grid: HBM bandwidth does not divide evenly over the SMs, and a resident grid
+// leaves the SMs that finish first idle, while the block scheduler keeps
+// every SM fed until the end.  Stores carry the streaming cache hint: every
+// byte is written exactly once.  Every arithmetic step is an explicitly
 // rounded fp32 intrinsic so that nothing is contracted into an FMA and the
 // results are fixed by the stated operation order.
 #include <cuda_bf16.h>
@@ -52,10 +55,21 @@ struct K1Args {
 };
 
 constexpr int kThreads = 256;
+constexpr int kChunks = 1;                  // 8-element chunks per thread
+constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
 
 __device__ __forceinline__ float lo_bf16(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
 __device__ __forceinline__ float bf16_of(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
+
+// 16-byte load (default caching) and streaming store.  Among the cache hints
+// measured on B200 for this kernel (streaming, read-only, last-use and
+// default loads; streaming and default stores), default loads with streaming
+// stores moved the most bytes per second at every D.
+template <class T>
+__device__ __forceinline__ T ld16(const T* p) { return *p; }
+template <class T>
+__device__ __forceinline__ void st16(T* p, const T& v) { __stcs(p, v); }
 
 // fp32 -> nearest-even bf16 -> fp32.
 __device__ __forceinline__ float round_to_bf16(float x) {
@@ -112,7 +126,7 @@ __device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&acc)
         uint4 q[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-            if (d0 + k < D) q[k] = __ldcs(reinterpret_cast<const uint4*>(a.c[d0 + k] + e));
+            if (d0 + k < D) q[k] = ld16(reinterpret_cast<const uint4*>(a.c[d0 + k] + e));
 #pragma unroll
         for (int k = 0; k < 8; ++k)
             if (d0 + k < D) fold8<MODE>(acc, q[k], d0 + k == 0);
@@ -142,39 +156,52 @@ __device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
     a.w[i] = __bfloat16_as_ushort(__float2bfloat16_rn(p));
 }
 
-// Vector kernel: every pointer 16-byte aligned.  Grid-stride over 8-element
-// chunks; the last n % 8 elements go through the scalar path.
+// The 8 elements starting at e: state loads, the rank fold, AdamW, stores.
+template <int MODE, int DT>
+__device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
+    const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
+    const float4 p1 = ld16(reinterpret_cast<const float4*>(a.p + e + 4));
+    const float4 m0 = ld16(reinterpret_cast<const float4*>(a.m + e));
+    const float4 m1 = ld16(reinterpret_cast<const float4*>(a.m + e + 4));
+    const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
+    const float4 v1 = ld16(reinterpret_cast<const float4*>(a.v + e + 4));
+    float acc[8];
+    reduce8<MODE, DT>(a, e, acc);
+    float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) adamw_elem(a.s, finish<MODE>(acc[k], a.inv_D), p[k], m[k], v[k]);
+    st16(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
+    st16(reinterpret_cast<float4*>(a.p + e + 4), make_float4(p[4], p[5], p[6], p[7]));
+    st16(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
+    st16(reinterpret_cast<float4*>(a.m + e + 4), make_float4(m[4], m[5], m[6], m[7]));
+    st16(reinterpret_cast<float4*>(a.v + e), make_float4(v[0], v[1], v[2], v[3]));
+    st16(reinterpret_cast<float4*>(a.v + e + 4), make_float4(v[4], v[5], v[6], v[7]));
+    st16(reinterpret_cast<uint4*>(a.w + e),
+         make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                    pack_bf16x2(p[6], p[7])));
+}
+
+// Vector kernel: every pointer 16-byte aligned.  The grid covers the whole
+// range (kChunks 8-element chunks per thread, consecutive threads on
+// consecutive chunks), so the block scheduler hands blocks to whichever SM is
+// free and every SM keeps streaming to the end; the outer loop only runs more
+// than once when the range exceeds the largest grid.  The last n % 8 elements
+// go through the scalar path.
 template <int MODE, int DT>
 __global__ void __launch_bounds__(kThreads) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
     const int64_t n8 = a.n >> 3;
-    const int64_t stride = int64_t(gridDim.x) * kThreads;
-    const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    for (int64_t q = tid; q < n8; q += stride) {
-        const int64_t e = q << 3;
-        const float4 p0 = __ldcs(reinterpret_cast<const float4*>(a.p + e));
-        const float4 p1 = __ldcs(reinterpret_cast<const float4*>(a.p + e + 4));
-        const float4 m0 = __ldcs(reinterpret_cast<const float4*>(a.m + e));
-        const float4 m1 = __ldcs(reinterpret_cast<const float4*>(a.m + e + 4));
-        const float4 v0 = __ldcs(reinterpret_cast<const float4*>(a.v + e));
-        const float4 v1 = __ldcs(reinterpret_cast<const float4*>(a.v + e + 4));
-        float acc[8];
-        reduce8<MODE, DT>(a, e, acc);
-        float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-        float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    const int64_t span = int64_t(kThreads) * kChunks;
+    const int64_t step = int64_t(gridDim.x) * span;
+    for (int64_t first = int64_t(blockIdx.x) * span + threadIdx.x; first < n8; first += step) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) adamw_elem(a.s, finish<MODE>(acc[k], a.inv_D), p[k], m[k], v[k]);
-        __stcs(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
-        __stcs(reinterpret_cast<float4*>(a.p + e + 4), make_float4(p[4], p[5], p[6], p[7]));
-        __stcs(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
-        __stcs(reinterpret_cast<float4*>(a.m + e + 4), make_float4(m[4], m[5], m[6], m[7]));
-        __stcs(reinterpret_cast<float4*>(a.v + e), make_float4(v[0], v[1], v[2], v[3]));
-        __stcs(reinterpret_cast<float4*>(a.v + e + 4), make_float4(v[4], v[5], v[6], v[7]));
-        __stcs(reinterpret_cast<uint4*>(a.w + e),
-               make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                          pack_bf16x2(p[6], p[7])));
+        for (int k = 0; k < kChunks; ++k) {
+            const int64_t q = first + int64_t(k) * kThreads;
+            if (q < n8) process8<MODE, DT>(a, q << 3);
+        }
     }
-    const int64_t tail = (n8 << 3) + tid;
+    const int64_t tail = (n8 << 3) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
     if (tail < a.n) scalar_elem<MODE>(a, tail);
 }
 
@@ -273,23 +300,30 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
         if (d < D && !z3::aligned(a.c[d], 16)) vec = false;
     }
 
-    // ---- launch: a whole number of resident waves, grid-stride inside
+    // ---- launch: the vector kernel's grid covers the range; the scalar kernel
+    // runs a whole number of resident waves with a grid-stride loop
     KernelFn fn;
     if (vec)
         fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32>(D) : pick_vec<Z3_REDUCE_BF16>(D);
     else
         fn = reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32>
                                             : k_reduce_adamw_scalar<Z3_REDUCE_BF16>;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    const int sms = z3::sm_count();
-    if (sms < 1) return Z3_ECUDA;
-    const int64_t work_items = vec ? (n >> 3) : n;
-    int64_t blocks = (work_items + kThreads - 1) / kThreads;
-    const int64_t resident = int64_t(sms) * per_sm;
-    if (blocks > resident) blocks = resident;
+    int64_t blocks;
+    if (vec) {
+        const int64_t span = int64_t(kThreads) * kChunks;
+        blocks = ((n >> 3) + span - 1) / span;
+        if (blocks > kMaxBlocks) blocks = kMaxBlocks;
+    } else {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        const int sms = z3::sm_count();
+        if (sms < 1) return Z3_ECUDA;
+        blocks = (n + kThreads - 1) / kThreads;
+        const int64_t resident = int64_t(sms) * per_sm;
+        if (blocks > resident) blocks = resident;
+    }
     if (blocks < 1) blocks = 1;  // the vector kernel's scalar tail still needs one block
     fn<<<dim3(unsigned(blocks)), dim3(kThreads), 0, static_cast<cudaStream_t>(cuda_stream)>>>(a);
     return cudaGetLastError() == cudaSuccess ? Z3_OK : Z3_ECUDA;

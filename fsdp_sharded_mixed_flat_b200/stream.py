@@ -57,10 +57,12 @@ class LayerStreamer:
 
     def step(self, source: Callable[[int], torch.Tensor], hp: "z3.AdamW",
              k1_events: Optional[Sequence] = None) -> None:
-        """One optimiser step over every block, last to first.  source(layer) gives the
-        device tensor (D * S bf16, the D owned contributions back to back) to copy in
-        for that block.  k1_events, if given, is a list of L (start, end) CUDA event
-        pairs recorded around each fused-kernel launch on the compute stream."""
+        """One optimiser step over every block, last to first.
+
+        source(layer) gives the tensor to copy in for that block: D * S bf16, the D
+        owned contributions back to back, on the device or in pinned host memory.
+        k1_events, if given, is a list of L (start, end) CUDA event pairs recorded
+        around each fused-kernel launch on the compute stream."""
         caller = torch.cuda.current_stream(self.device)
         self.copy.wait_stream(caller)
         self.compute.wait_stream(caller)
@@ -70,7 +72,8 @@ class LayerStreamer:
                 self.copy.wait_event(self.free[b])          # the kernel two blocks back is done with it
                 src = source(layer)
                 self.buf[b].copy_(src, non_blocking=True)
-                src.record_stream(self.copy)
+                if src.is_cuda:
+                    src.record_stream(self.copy)
                 self.filled[b].record(self.copy)
             self.compute.wait_event(self.filled[b])
             p, m, v, w = self.layer_views(layer)
