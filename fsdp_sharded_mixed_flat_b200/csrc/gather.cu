@@ -8,8 +8,9 @@
 //
 // Both kernels are pure copies bound by HBM bandwidth (2 bytes read + 2 bytes
 // written per element).
-//   - flat copy: grid.y = rank; every thread moves 4 independent 16-byte
-//     vectors per iteration (64 bytes in flight per thread), streaming hints.
+//   - flat copy: grid.y = rank, grid.x covering the shard (2 independent
+//     16-byte vectors per thread, consecutive threads on consecutive vectors),
+//     so the block scheduler balances the SMs; streaming stores.
 //   - per-tensor copy: the host cuts every tensor into segments, one per rank
 //     partition it intersects, and numbers the 16-byte units of each
 //     segment's destination.  A thread takes one destination unit, finds its
@@ -30,7 +31,8 @@
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 2;                 // 16-byte vectors per thread in the flat copy
+constexpr int64_t kMaxBlocks = 1 << 30;   // grid.x cap; beyond it the kernels loop
 constexpr int kSegMax = 112;  // segments per launch; keeps the parameter block under 4 KB
 
 struct FlatArgs {
@@ -58,16 +60,16 @@ __global__ void __launch_bounds__(kThreads) k_gather_flat_vec(const __grid_const
     const uint4* src = reinterpret_cast<const uint4*>(a.shard[r]);
     uint4* dst = reinterpret_cast<uint4*>(a.flat + int64_t(r) * a.S);
     const int64_t n = a.S >> 3;
-    const int64_t stride = int64_t(gridDim.x) * kThreads;
-    int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    for (; i + (kUnroll - 1) * stride < n; i += kUnroll * stride) {
+    const int64_t span = int64_t(kThreads) * kUnroll;
+    for (int64_t i = int64_t(blockIdx.x) * span + threadIdx.x; i < n; i += int64_t(gridDim.x) * span) {
         uint4 q[kUnroll];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) q[k] = __ldcs(src + i + k * stride);
+        for (int k = 0; k < kUnroll; ++k)
+            if (i + k * kThreads < n) q[k] = src[i + k * kThreads];
 #pragma unroll
-        for (int k = 0; k < kUnroll; ++k) __stcs(dst + i + k * stride, q[k]);
+        for (int k = 0; k < kUnroll; ++k)
+            if (i + k * kThreads < n) __stcs(dst + i + k * kThreads, q[k]);
     }
-    for (; i < n; i += stride) __stcs(dst + i, __ldcs(src + i));
 }
 
 __global__ void __launch_bounds__(kThreads) k_gather_flat_scalar(const __grid_constant__ FlatArgs a) {
@@ -193,13 +195,18 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
         a.S = S;
         const bool vec = vec_src && z3::aligned(flat_out, 16);
         auto fn = vec ? k_gather_flat_vec : k_gather_flat_scalar;
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess || per_sm < 1)
-            per_sm = 1;
-        const int64_t items = vec ? ((S >> 3) + kUnroll - 1) / kUnroll : S;
-        int64_t bx = (items + kThreads - 1) / kThreads;
-        const int64_t cap = std::max<int64_t>(1, (int64_t(sms) * per_sm + D - 1) / D);
-        bx = std::max<int64_t>(1, std::min(bx, cap));
+        int64_t bx;
+        if (vec) {
+            bx = ((S >> 3) + int64_t(kThreads) * kUnroll - 1) / (int64_t(kThreads) * kUnroll);
+            bx = std::max<int64_t>(1, std::min(bx, kMaxBlocks));
+        } else {
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess || per_sm < 1)
+                per_sm = 1;
+            bx = (S + kThreads - 1) / kThreads;
+            const int64_t cap = std::max<int64_t>(1, (int64_t(sms) * per_sm + D - 1) / D);
+            bx = std::max<int64_t>(1, std::min(bx, cap));
+        }
         fn<<<dim3(unsigned(bx), unsigned(D)), dim3(kThreads), 0, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;
     }
@@ -230,12 +237,8 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
                 a.seg[k] = s;
             }
             a.units = units;
-            int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gather_segments, kThreads, 0) !=
-                    cudaSuccess || per_sm < 1)
-                per_sm = 1;
             int64_t blocks = (units + kThreads - 1) / kThreads;
-            blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, int64_t(sms) * per_sm));
+            blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, kMaxBlocks));
             k_gather_segments<<<dim3(unsigned(blocks)), dim3(kThreads), 0, stream>>>(a);
             if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;
         }

@@ -21,7 +21,15 @@
 // grid: HBM bandwidth does not divide evenly over the SMs, and a resident grid
 // leaves the SMs that finish first idle, while the block scheduler keeps
 // every SM fed until the end.  Stores carry the streaming cache hint: every
-// byte is written exactly once.  Every arithmetic step is an explicitly
+// byte is written exactly once.  Asking for three resident blocks per SM caps
+// the registers at 85 (left alone the compiler takes up to 128 at D >= 16 and
+// spills at D = 4 and 8 in bf16 mode); measured on B200 this never loses and
+// gains up to 12 % (bf16 reduce at D = 16).
+//
+// Measured ceilings of HBM on the B200s used here, for a full-grid kernel with
+// two or more independent 16-byte vectors per thread: read-only 7.54 TB/s,
+// write-only 7.56 TB/s, copy 6.94 TB/s, two reads per write 7.16 TB/s.  This
+// pass reads 28 B and writes 14 B per element at D = 8, the two-to-one mix.  Every arithmetic step is an explicitly
 // rounded fp32 intrinsic so that nothing is contracted into an FMA and the
 // results are fixed by the stated operation order.
 #include <cuda_bf16.h>
@@ -55,6 +63,7 @@ struct K1Args {
 };
 
 constexpr int kThreads = 256;
+constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: caps registers at 85 per thread
 constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
 
@@ -95,31 +104,45 @@ __device__ __forceinline__ void adamw_elem(const AdamScalars& s, float g, float&
     v = v1;
 }
 
-// Fold one rank's 8 bf16 values (one 16-byte vector) into the accumulators.
-template <int MODE>
-__device__ __forceinline__ void fold8(float (&acc)[8], const uint4& q, bool first) {
+// Two bf16 values added pairwise by the packed hardware add, which rounds the
+// exact sum to the nearest-even bf16.  That equals rounding the fp32 sum to
+// bf16: double rounding through a format with more than 2p + 2 significand
+// bits is innocuous (Figueroa, "When is double rounding innocuous?", 1995),
+// and fp32's 24 bits exceed 18 for bf16's p = 8, also in the shared subnormal
+// range, where both formats lose the same number of leading bits.
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Fold one rank's 8 bf16 values (one 16-byte vector) into fp32 accumulators.
+__device__ __forceinline__ void fold8_fp32(float (&acc)[8], const uint4& q, bool first) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const float a = lo_bf16(w[k]), b = hi_bf16(w[k]);
-        if (first) {
-            acc[2 * k] = a;
-            acc[2 * k + 1] = b;
-        } else if (MODE == Z3_REDUCE_FP32) {
-            acc[2 * k] = __fadd_rn(acc[2 * k], a);
-            acc[2 * k + 1] = __fadd_rn(acc[2 * k + 1], b);
-        } else {
-            acc[2 * k] = round_to_bf16(__fadd_rn(acc[2 * k], a));
-            acc[2 * k + 1] = round_to_bf16(__fadd_rn(acc[2 * k + 1], b));
-        }
+        acc[2 * k] = first ? a : __fadd_rn(acc[2 * k], a);
+        acc[2 * k + 1] = first ? b : __fadd_rn(acc[2 * k + 1], b);
     }
 }
 
-// Reduce ranks 0..D-1 for the 8 elements starting at e, in chunks of 8 ranks:
-// the chunk's loads are all issued before its folds.
+// Fold one rank's 8 bf16 values into packed bf16 accumulators (element 2k in
+// the low half of word k).
+__device__ __forceinline__ void fold8_bf16(uint32_t (&acc)[4], const uint4& q, bool first) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = first ? w[k] : add_bf16x2(acc[k], w[k]);
+}
+
+// Reduce ranks 0..D-1 for the 8 elements starting at e, left to right, in
+// chunks of 8 ranks (the chunk's loads are all issued before its folds), and
+// return the averaged gradient g = sum * (1/D) in the reduce dtype.
 template <int MODE, int DT>
-__device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&acc)[8]) {
+__device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8]) {
     const int D = DT > 0 ? DT : a.D;
+    float acc[8];
+    uint32_t accw[4];
 #pragma unroll
     for (int d0 = 0; d0 < (DT > 0 ? DT : Z3_D_MAX); d0 += 8) {
         if (DT == 0 && d0 >= D) break;
@@ -128,8 +151,23 @@ __device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&acc)
         for (int k = 0; k < 8; ++k)
             if (d0 + k < D) q[k] = ld16(reinterpret_cast<const uint4*>(a.c[d0 + k] + e));
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            if (d0 + k < D) fold8<MODE>(acc, q[k], d0 + k == 0);
+        for (int k = 0; k < 8; ++k) {
+            if (d0 + k >= D) continue;
+            if constexpr (MODE == Z3_REDUCE_FP32)
+                fold8_fp32(acc, q[k], d0 + k == 0);
+            else
+                fold8_bf16(accw, q[k], d0 + k == 0);
+        }
+    }
+    if constexpr (MODE == Z3_REDUCE_FP32) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) g[k] = __fmul_rn(acc[k], a.inv_D);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            g[2 * k] = round_to_bf16(__fmul_rn(lo_bf16(accw[k]), a.inv_D));
+            g[2 * k + 1] = round_to_bf16(__fmul_rn(hi_bf16(accw[k]), a.inv_D));
+        }
     }
 }
 
@@ -165,13 +203,13 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
     const float4 m1 = ld16(reinterpret_cast<const float4*>(a.m + e + 4));
     const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
     const float4 v1 = ld16(reinterpret_cast<const float4*>(a.v + e + 4));
-    float acc[8];
-    reduce8<MODE, DT>(a, e, acc);
+    float g[8];
+    reduce8<MODE, DT>(a, e, g);
     float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
     float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) adamw_elem(a.s, finish<MODE>(acc[k], a.inv_D), p[k], m[k], v[k]);
+    for (int k = 0; k < 8; ++k) adamw_elem(a.s, g[k], p[k], m[k], v[k]);
     st16(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
     st16(reinterpret_cast<float4*>(a.p + e + 4), make_float4(p[4], p[5], p[6], p[7]));
     st16(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
@@ -190,7 +228,7 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
 // than once when the range exceeds the largest grid.  The last n % 8 elements
 // go through the scalar path.
 template <int MODE, int DT>
-__global__ void __launch_bounds__(kThreads) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
     const int64_t n8 = a.n >> 3;
     const int64_t span = int64_t(kThreads) * kChunks;
     const int64_t step = int64_t(gridDim.x) * span;

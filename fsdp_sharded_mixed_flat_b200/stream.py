@@ -56,18 +56,33 @@ class LayerStreamer:
         return [self.buf[b][d * S:(d + 1) * S] for d in range(self.plan.D)]
 
     def step(self, source: Callable[[int], torch.Tensor], hp: "z3.AdamW",
-             k1_events: Optional[Sequence] = None) -> None:
+             k1_events: Optional[Sequence] = None, copy_in: bool = True) -> None:
         """One optimiser step over every block, last to first.
 
         source(layer) gives the tensor to copy in for that block: D * S bf16, the D
         owned contributions back to back, on the device or in pinned host memory.
         k1_events, if given, is a list of L (start, end) CUDA event pairs recorded
-        around each fused-kernel launch on the compute stream."""
+        around each fused-kernel launch on the compute stream.  With copy_in=False
+        the kernel reads each block's contributions where source(layer) holds them
+        (a device tensor that stays valid for the step) and nothing is copied."""
         caller = torch.cuda.current_stream(self.device)
         self.copy.wait_stream(caller)
         self.compute.wait_stream(caller)
+        S, D = self.plan.S, self.plan.D
         for i, layer in enumerate(range(self.L - 1, -1, -1)):
             b = i & 1
+            if not copy_in:
+                src = source(layer)
+                contribs = [src[d * S:(d + 1) * S] for d in range(D)]
+                p, m, v, w = self.layer_views(layer)
+                if k1_events is not None:
+                    k1_events[i][0].record(self.compute)
+                z3.zero3_reduce_adamw(self.plan, self.rank, contribs, p, m, v, w, hp,
+                                      contrib_layout=z3.Z3_CONTRIB_OWNED, reduce_dtype=self.reduce_dtype,
+                                      stream=self.compute)
+                if k1_events is not None:
+                    k1_events[i][1].record(self.compute)
+                continue
             with torch.cuda.stream(self.copy):
                 self.copy.wait_event(self.free[b])          # the kernel two blocks back is done with it
                 src = source(layer)

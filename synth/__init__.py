@@ -116,6 +116,9 @@ def contribution(n_real: int, n_total: int, *, seed: int, step: int, rank: int,
             chi2 += e * e
         x = z / torch.sqrt(chi2 / 3.0) * sigma
         del z, chi2
+    elif dist == "subnormal":
+        # scaled so that most values and partial sums are bf16 / fp32 subnormals
+        x = torch.randn(n_real, generator=g, device=device, dtype=torch.float32) * 2.0 ** -130
     elif dist == "integers":
         # small integers, exactly representable in bf16 and in every partial sum
         x = torch.randint(-8, 9, (n_real,), generator=g, device=device).to(torch.float32)

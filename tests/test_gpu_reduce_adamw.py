@@ -100,6 +100,14 @@ def test_heavy_tails_and_exact_zeros(z3):
                   zero_frac=0.01)
 
 
+def test_subnormal_contributions(z3):
+    """Gradients in the bf16 / fp32 subnormal range: the packed bf16 add and the
+    fp32 path keep subnormals exactly as the oracle does (no flush to zero)."""
+    for mode in (0, 1):
+        run_small(z3, [20000, 77], 8, 8, -1, z3.Z3_CONTRIB_FULL, mode, steps=3, dist="subnormal")
+        run_small(z3, [20000, 77], 16, 8, 3, z3.Z3_CONTRIB_OWNED, mode, steps=2, dist="subnormal")
+
+
 def test_integer_contributions_give_the_same_step_in_both_reduce_dtypes(z3):
     """Exact partial sums: the bf16 and fp32 reductions must coincide."""
     out = []

@@ -27,8 +27,9 @@ def owned_contribs(D, S, n_real, seed, step, layer, sigma=1e-3):
                                          device="cuda") for d in range(D)])
 
 
+@pytest.mark.parametrize("copy_in", [True, False], ids=["double_buffer", "in_place"])
 @pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
-def test_streamed_layers_match_oracle(z3, mode):
+def test_streamed_layers_match_oracle(z3, mode, copy_in):
     from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
     L, D, rank = 7, 4, 2
     plan = z3.zero3_plan([(300,), (77, 5), (1000,)], D, 8)
@@ -42,7 +43,7 @@ def test_streamed_layers_match_oracle(z3, mode):
         np.zeros(L * S, np.uint16)
     for t in range(1, 4):
         src = {l: owned_contribs(D, S, n_real, 9, t, l) for l in range(L)}
-        st.step(lambda l: src[l], z3.adamw(**hp_for(t)))
+        st.step(lambda l: src[l], z3.adamw(**hp_for(t)), copy_in=copy_in)
         for l in range(L):
             host = synth.bf16_bits(src[l])
             sl = slice(l * S, (l + 1) * S)
