@@ -56,6 +56,12 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
+    ap.add_argument("--drift", action="store_true",
+                    help="report the drift of the bf16-reduce path against the fp32-reduce path")
+    ap.add_argument("--drift-elements", type=int, default=1 << 24)
+    ap.add_argument("--stage", type=int, choices=[1, 2, 3], default=3,
+                    help="3: ZeRO-3 step (fused reduce/AdamW/cast, then the gather of the shards); "
+                         "1 or 2: the fused kernel also all-gathers into the replicated bf16 weights")
     return ap.parse_args()
 
 
@@ -220,9 +226,11 @@ def run_reference(args):
 # ---------------------------------------------------------------- our path
 class BlockRunner:
     """One block, every rank's partition in one launch: plan + ledger (host),
-    fused reduce + AdamW + cast, gather into the flat block, zero-copy views."""
+    fused reduce + AdamW + cast, gather into the flat block, zero-copy views.
+    stage 1 or 2: one kernel does the reduce, AdamW, cast and the all-gather into
+    the replicated bf16 weights (the flat block), with no separate shard."""
 
-    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev):
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
@@ -238,16 +246,20 @@ class BlockRunner:
         self.shards = [self.work[r * self.S:(r + 1) * self.S] for r in range(D)]
         self.stream = torch.cuda.current_stream(dev)
         self.step_no = 0
+        self.stage = stage
         self.units_per_step = self.N_pad                       # owned params, all ranks
         self.k1_launches_per_step = 1
-        self.k1_bytes_per_launch = (2 * D + 26) * self.N_pad
-        self.step_bytes = self.k1_bytes_per_launch + 4 * self.N_pad
-        self.launches_per_step = 2
-        self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}>"
+        self.k1_bytes_per_launch = (2 * D + 26) * self.N_pad   # stage 1/2: the bf16 goes to the block instead
+        self.step_bytes = self.k1_bytes_per_launch + (4 * self.N_pad if stage == 3 else 0)
+        self.launches_per_step = 2 if stage == 3 else 1
+        self.k1_name = (f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}"
+                        f"{', gather' if stage != 3 else ''}>")
+        what = ("fused reduce/AdamW/cast over all %d partitions + gather into the flat block" % D if stage == 3
+                else "one kernel: reduce/AdamW/cast over all %d partitions writing the replicated bf16 "
+                     "weights in place of the gather (ZeRO-%d)" % (D, stage))
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
                      f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
-                     f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + fused reduce/AdamW/cast over all "
-                     f"{D} partitions + gather into the flat block")
+                     f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + {what}")
 
     def hp(self):
         a = self.synth.ADAMW
@@ -259,10 +271,17 @@ class BlockRunner:
         z3 = self.z3
         # a1 + a2: host-side plan and ledger of the block (microseconds, overlapped with the GPU)
         pl = z3.zero3_plan(self.shapes, self.D, self.synth.ALIGN)
-        z3.zero3_memory_bytes(pl.N, self.D, z3.Z3_STAGE_ZERO3)
+        z3.zero3_memory_bytes(pl.N, self.D, self.stage)
         hp = self.hp()
         if k1_events is not None:
             k1_events[0][0].record(self.stream)
+        if self.stage != 3:
+            # ZeRO-1/2: the kernel writes each new bf16 weight into the replicated block
+            z3.zero3_reduce_adamw_gather(pl, -1, self.contribs, self.master, self.exp_avg, self.exp_avg_sq, None,
+                                         [self.flat], hp, reduce_dtype=self.mode, stream=self.stream)
+            if k1_events is not None:
+                k1_events[0][1].record(self.stream)
+            return pl.views(self.flat)
         # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
         z3.zero3_reduce_adamw(pl, -1, self.contribs, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
                               reduce_dtype=self.mode, stream=self.stream)
@@ -381,7 +400,8 @@ def run_ours(args):
     if args.workload == "llama70b_shard":
         R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev)
     else:
-        R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev)
+        R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
+                        stage=args.stage)
     stream = R.stream
 
     for _ in range(args.warmup):
@@ -454,7 +474,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D,
+        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D, "stage": getattr(R, "stage", 3),
                    "reduce_dtype": "bf16" if mode == z3.Z3_REDUCE_BF16 else "fp32",
                    "owned_params_per_step": R.units_per_step,
                    "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (R.step_bytes / 1e9),
@@ -487,8 +507,55 @@ def run_ours(args):
     return 0
 
 
+def run_drift(args):
+    """The policy sweep's drift: the same heavy-tailed contributions (Student-t nu=3,
+    1% exact zeros, fresh every step) drive two copies of the same master, one
+    reduced in bf16 and one in fp32, for --steps steps at each D; report how far
+    the bf16 path's master and bf16 weights end up from the fp32 path's."""
+    import torch
+
+    import synth
+    from fsdp_sharded_mixed_flat_b200 import build
+    build.build()
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    dev = torch.device("cuda", 0)
+    w = synth.WORKLOADS["llama7b_policy"]
+    n = args.drift_elements
+    out = {"drift": {}, "steps": args.steps, "elements": n,
+           "workload": "first %d elements of the LLaMA-7B block, Student-t nu=3 x %g, %g%% exact zeros, "
+                       "fresh contributions every step" % (n, w["sigma"], 100 * w["zero_frac"])}
+    for D in w["Ds"]:
+        plan = z3.zero3_plan([(n,)], D, synth.ALIGN)
+        N_pad = plan.N_pad
+        p0 = synth.master_weights(n, N_pad, seed=11, device=dev)
+        state = {mode: [p0.clone(), torch.zeros_like(p0), torch.zeros_like(p0),
+                        torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)] for mode in (0, 1)}
+        for t in range(1, args.steps + 1):
+            c = synth.contributions(D, n, N_pad, seed=11, step=t, sigma=w["sigma"], dist=w["dist"],
+                                    zero_frac=w["zero_frac"], device=dev)
+            for mode in (0, 1):
+                z3.zero3_reduce_adamw(plan, -1, c, *state[mode], z3.adamw(step=t), reduce_dtype=mode)
+        torch.cuda.synchronize(dev)
+        pf, pb = state[0][0][:n].double(), state[1][0][:n].double()
+        upd = (pf - p0[:n].double())
+        diff = (pb - pf)
+        rel = diff.abs() / pf.abs().clamp_min(1e-30)
+        upd_rms = upd.pow(2).mean().sqrt()
+        wf, wb = state[0][3][:n].view(torch.int16), state[1][3][:n].view(torch.int16)
+        out["drift"][f"D={D}"] = {
+            "master_median_rel": rel.median().item(),
+            "max_abs_diff_over_update_rms": (diff.abs().max() / upd_rms).item(),
+            "diff_rms_over_update_rms": (diff.pow(2).mean().sqrt() / upd_rms).item(),
+            "bf16_weights_differing": (wf != wb).double().mean().item(),
+        }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
+    if args.drift:
+        return run_drift(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

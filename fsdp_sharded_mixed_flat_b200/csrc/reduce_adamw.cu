@@ -55,7 +55,9 @@ struct K1Args {
     float* p;                     // master
     float* m;                     // exp_avg
     float* v;                     // exp_avg_sq
-    uint16_t* w;                  // bf16 working weights
+    uint16_t* w;                  // bf16 working weights (may be null when gathering)
+    uint16_t* g[Z3_GATHER_MAX];   // gathered blocks, each at the launch's first element
+    int32_t ng;                   // number of gathered blocks
     int64_t n;                    // elements in this launch
     int32_t D;
     float inv_D;                  // fp32 nearest to 1/D
@@ -178,7 +180,7 @@ __device__ __forceinline__ float finish(float acc, float inv_D) {
 }
 
 // One element on the scalar path (tails and misaligned buffers).
-template <int MODE>
+template <int MODE, bool GATHER>
 __device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
     float acc = bf16_of(a.c[0][i]);
     for (int d = 1; d < a.D; ++d) {
@@ -191,11 +193,16 @@ __device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
     a.p[i] = p;
     a.m[i] = m;
     a.v[i] = v;
-    a.w[i] = __bfloat16_as_ushort(__float2bfloat16_rn(p));
+    const uint16_t w = __bfloat16_as_ushort(__float2bfloat16_rn(p));
+    if (!GATHER || a.w != nullptr) a.w[i] = w;
+    if (GATHER)
+        for (int k = 0; k < a.ng; ++k) a.g[k][i] = w;
 }
 
 // The 8 elements starting at e: state loads, the rank fold, AdamW, stores.
-template <int MODE, int DT>
+// GATHER: the bf16 result also goes to every gathered block (the all-gather's
+// data movement done by the producer of the data).
+template <int MODE, int DT, bool GATHER>
 __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
     const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
     const float4 p1 = ld16(reinterpret_cast<const float4*>(a.p + e + 4));
@@ -216,9 +223,14 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
     st16(reinterpret_cast<float4*>(a.m + e + 4), make_float4(m[4], m[5], m[6], m[7]));
     st16(reinterpret_cast<float4*>(a.v + e), make_float4(v[0], v[1], v[2], v[3]));
     st16(reinterpret_cast<float4*>(a.v + e + 4), make_float4(v[4], v[5], v[6], v[7]));
-    st16(reinterpret_cast<uint4*>(a.w + e),
-         make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
-                    pack_bf16x2(p[6], p[7])));
+    const uint4 w = make_uint4(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3]), pack_bf16x2(p[4], p[5]),
+                               pack_bf16x2(p[6], p[7]));
+    if (!GATHER || a.w != nullptr) st16(reinterpret_cast<uint4*>(a.w + e), w);
+    if (GATHER) {
+#pragma unroll
+        for (int k = 0; k < Z3_GATHER_MAX; ++k)
+            if (k < a.ng) st16(reinterpret_cast<uint4*>(a.g[k] + e), w);
+    }
 }
 
 // Vector kernel: every pointer 16-byte aligned.  The grid covers the whole
@@ -227,7 +239,7 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
 // free and every SM keeps streaming to the end; the outer loop only runs more
 // than once when the range exceeds the largest grid.  The last n % 8 elements
 // go through the scalar path.
-template <int MODE, int DT>
+template <int MODE, int DT, bool GATHER>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
     const int64_t n8 = a.n >> 3;
     const int64_t span = int64_t(kThreads) * kChunks;
@@ -236,44 +248,54 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const
 #pragma unroll
         for (int k = 0; k < kChunks; ++k) {
             const int64_t q = first + int64_t(k) * kThreads;
-            if (q < n8) process8<MODE, DT>(a, q << 3);
+            if (q < n8) process8<MODE, DT, GATHER>(a, q << 3);
         }
     }
     const int64_t tail = (n8 << 3) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    if (tail < a.n) scalar_elem<MODE>(a, tail);
+    if (tail < a.n) scalar_elem<MODE, GATHER>(a, tail);
 }
 
 // Scalar kernel: any element-aligned pointers.
-template <int MODE>
+template <int MODE, bool GATHER>
 __global__ void __launch_bounds__(kThreads) k_reduce_adamw_scalar(const __grid_constant__ K1Args a) {
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < a.n; i += stride)
-        scalar_elem<MODE>(a, i);
+        scalar_elem<MODE, GATHER>(a, i);
 }
 
 using KernelFn = void (*)(K1Args);
 
-template <int MODE>
+template <int MODE, bool GATHER>
 KernelFn pick_vec(int D) {
     switch (D) {
-    case 1: return k_reduce_adamw_vec<MODE, 1>;
-    case 2: return k_reduce_adamw_vec<MODE, 2>;
-    case 4: return k_reduce_adamw_vec<MODE, 4>;
-    case 8: return k_reduce_adamw_vec<MODE, 8>;
-    case 16: return k_reduce_adamw_vec<MODE, 16>;
-    case 32: return k_reduce_adamw_vec<MODE, 32>;
-    default: return k_reduce_adamw_vec<MODE, 0>;
+    case 1: return k_reduce_adamw_vec<MODE, 1, GATHER>;
+    case 2: return k_reduce_adamw_vec<MODE, 2, GATHER>;
+    case 4: return k_reduce_adamw_vec<MODE, 4, GATHER>;
+    case 8: return k_reduce_adamw_vec<MODE, 8, GATHER>;
+    case 16: return k_reduce_adamw_vec<MODE, 16, GATHER>;
+    case 32: return k_reduce_adamw_vec<MODE, 32, GATHER>;
+    default: return k_reduce_adamw_vec<MODE, 0, GATHER>;
     }
+}
+
+template <bool GATHER>
+KernelFn pick(bool vec, int32_t reduce_dtype, int D) {
+    if (vec)
+        return reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32, GATHER>(D)
+                                              : pick_vec<Z3_REDUCE_BF16, GATHER>(D);
+    return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, GATHER>
+                                          : k_reduce_adamw_scalar<Z3_REDUCE_BF16, GATHER>;
 }
 
 bool is_finite(double x) { return std::isfinite(x); }
 
-}  // namespace
-
-extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
-                                         int32_t contrib_layout, float* master, float* exp_avg,
-                                         float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
-                                         const z3_adamw* hp, void* cuda_stream) {
+// Validation and launch shared by both entry points.  `gathered` holds
+// n_gathered whole padded blocks (0 for the plain entry point); `work_bf16`
+// may be null only when n_gathered > 0.
+int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, int32_t contrib_layout,
+              float* master, float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
+              uint16_t* const* gathered, int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
+              void* cuda_stream) {
     // ---- arguments
     if (p == nullptr || contrib == nullptr || hp == nullptr) return Z3_EINVAL;
     const int32_t D = p->D;
@@ -281,10 +303,15 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
     if (contrib_layout != Z3_CONTRIB_FULL && contrib_layout != Z3_CONTRIB_OWNED) return Z3_EINVAL;
     if (contrib_layout == Z3_CONTRIB_OWNED && rank < 0) return Z3_EINVAL;
     if (reduce_dtype != Z3_REDUCE_FP32 && reduce_dtype != Z3_REDUCE_BF16) return Z3_EINVAL;
-    if (master == nullptr || exp_avg == nullptr || exp_avg_sq == nullptr || work_bf16 == nullptr)
+    if (n_gathered < 0 || n_gathered > Z3_GATHER_MAX || (n_gathered > 0 && gathered == nullptr))
+        return Z3_EINVAL;
+    if (master == nullptr || exp_avg == nullptr || exp_avg_sq == nullptr ||
+        (work_bf16 == nullptr && n_gathered == 0))
         return Z3_EINVAL;
     for (int32_t d = 0; d < D; ++d)
         if (contrib[d] == nullptr) return Z3_EINVAL;
+    for (int32_t k = 0; k < n_gathered; ++k)
+        if (gathered[k] == nullptr) return Z3_EINVAL;
     if (hp->step < 1 || !is_finite(hp->lr) || !is_finite(hp->beta1) || !is_finite(hp->beta2) ||
         !is_finite(hp->eps) || !is_finite(hp->weight_decay) || hp->beta1 < 0.0 || hp->beta1 >= 1.0 ||
         hp->beta2 < 0.0 || hp->beta2 >= 1.0)
@@ -294,17 +321,25 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
         return Z3_EALIGN;
     for (int32_t d = 0; d < D; ++d)
         if (!z3::aligned(contrib[d], 2)) return Z3_EALIGN;
+    for (int32_t k = 0; k < n_gathered; ++k)
+        if (!z3::aligned(gathered[k], 2)) return Z3_EALIGN;
 
     const int64_t n = rank < 0 ? p->N_pad : p->S;
-    // first element of the launch inside each contribution buffer
+    // first element of the launch inside each contribution buffer and gathered block
     const int64_t c_off = (contrib_layout == Z3_CONTRIB_FULL && rank >= 0) ? int64_t(rank) * p->S : 0;
+    const int64_t g_off = rank >= 0 ? int64_t(rank) * p->S : 0;
 
     // ---- outputs must not overlap each other or any contribution they read
     const int64_t fb = n * 4, hb = n * 2;
-    const void* outs[4] = {master, exp_avg, exp_avg_sq, work_bf16};
-    const int64_t out_bytes[4] = {fb, fb, fb, hb};
-    for (int x = 0; x < 4; ++x) {
-        for (int y = x + 1; y < 4; ++y)
+    const void* outs[4 + Z3_GATHER_MAX] = {master, exp_avg, exp_avg_sq, work_bf16};
+    int64_t out_bytes[4 + Z3_GATHER_MAX] = {fb, fb, fb, work_bf16 ? hb : 0};
+    for (int32_t k = 0; k < n_gathered; ++k) {
+        outs[4 + k] = gathered[k];
+        out_bytes[4 + k] = p->N_pad * 2;  // the whole block is the caller's buffer
+    }
+    const int n_out = 4 + n_gathered;
+    for (int x = 0; x < n_out; ++x) {
+        for (int y = x + 1; y < n_out; ++y)
             if (z3::overlaps(outs[x], out_bytes[x], outs[y], out_bytes[y])) return Z3_EINVAL;
         for (int32_t d = 0; d < D; ++d)
             if (z3::overlaps(outs[x], out_bytes[x], contrib[d] + c_off, hb)) return Z3_EINVAL;
@@ -331,21 +366,21 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
     a.m = exp_avg;
     a.v = exp_avg_sq;
     a.w = work_bf16;
+    a.ng = n_gathered;
     bool vec = z3::aligned(master, 16) && z3::aligned(exp_avg, 16) && z3::aligned(exp_avg_sq, 16) &&
                z3::aligned(work_bf16, 16);
     for (int32_t d = 0; d < Z3_D_MAX; ++d) {
         a.c[d] = d < D ? contrib[d] + c_off : nullptr;
         if (d < D && !z3::aligned(a.c[d], 16)) vec = false;
     }
+    for (int32_t k = 0; k < Z3_GATHER_MAX; ++k) {
+        a.g[k] = k < n_gathered ? gathered[k] + g_off : nullptr;
+        if (k < n_gathered && !z3::aligned(a.g[k], 16)) vec = false;
+    }
 
     // ---- launch: the vector kernel's grid covers the range; the scalar kernel
     // runs a whole number of resident waves with a grid-stride loop
-    KernelFn fn;
-    if (vec)
-        fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32>(D) : pick_vec<Z3_REDUCE_BF16>(D);
-    else
-        fn = reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32>
-                                            : k_reduce_adamw_scalar<Z3_REDUCE_BF16>;
+    const KernelFn fn = n_gathered > 0 ? pick<true>(vec, reduce_dtype, D) : pick<false>(vec, reduce_dtype, D);
     int64_t blocks;
     if (vec) {
         const int64_t span = int64_t(kThreads) * kChunks;
@@ -365,4 +400,24 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
     if (blocks < 1) blocks = 1;  // the vector kernel's scalar tail still needs one block
     fn<<<dim3(unsigned(blocks)), dim3(kThreads), 0, static_cast<cudaStream_t>(cuda_stream)>>>(a);
     return cudaGetLastError() == cudaSuccess ? Z3_OK : Z3_ECUDA;
+}
+
+}  // namespace
+
+extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                         int32_t contrib_layout, float* master, float* exp_avg,
+                                         float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
+                                         const z3_adamw* hp, void* cuda_stream) {
+    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, nullptr, 0,
+                     reduce_dtype, hp, cuda_stream);
+}
+
+extern "C" Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                                int32_t contrib_layout, float* master, float* exp_avg,
+                                                float* exp_avg_sq, uint16_t* work_bf16,
+                                                uint16_t* const* gathered, int32_t n_gathered,
+                                                int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream) {
+    if (n_gathered < 1) return Z3_EINVAL;
+    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
+                     n_gathered, reduce_dtype, hp, cuda_stream);
 }

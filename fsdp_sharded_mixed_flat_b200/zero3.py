@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(HERE, "libzero3.so")
 
 Z3_OK, Z3_EINVAL, Z3_EALIGN, Z3_ENOMEM, Z3_ECUDA, Z3_EOVERFLOW = 0, -1, -2, -3, -4, -5
 Z3_D_MAX = 64
+Z3_GATHER_MAX = 8
 Z3_REDUCE_FP32, Z3_REDUCE_BF16 = 0, 1
 Z3_CONTRIB_FULL, Z3_CONTRIB_OWNED = 0, 1
 Z3_STAGE_DDP, Z3_STAGE_ZERO1, Z3_STAGE_ZERO2, Z3_STAGE_ZERO3 = 0, 1, 2, 3
@@ -64,6 +65,9 @@ def _load() -> C.CDLL:
     L.zero3_transient_bytes.restype = C.c_int
     L.zero3_reduce_adamw.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw.restype = C.c_int
+    L.zero3_reduce_adamw_gather.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
+                                            C.POINTER(AdamW), vp]
+    L.zero3_reduce_adamw_gather.restype = C.c_int
     L.zero3_gather_block.argtypes = [vp, vp, vp, vp, vp]
     L.zero3_gather_block.restype = C.c_int
     return L
@@ -213,6 +217,37 @@ def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], m
         rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                      reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw")
+
+
+def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], master: torch.Tensor,
+                              exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
+                              work_bf16: Optional[torch.Tensor], gathered: Sequence[torch.Tensor], hp: AdamW,
+                              contrib_layout: int = Z3_CONTRIB_FULL, reduce_dtype: int = Z3_REDUCE_FP32,
+                              stream=None) -> None:
+    """zero3_reduce_adamw whose kernel also writes every new bf16 weight into its place
+    in each gathered block (N_pad bf16 each); work_bf16 may be None (see include/zero3.h)."""
+    if len(contrib) != plan.D:
+        raise ValueError(f"need {plan.D} contributions, got {len(contrib)}")
+    if not 1 <= len(gathered) <= Z3_GATHER_MAX:
+        raise ValueError(f"need 1..{Z3_GATHER_MAX} gathered blocks, got {len(gathered)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * plan.D)()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    gp = (C.c_void_p * len(gathered))()
+    for k, g in enumerate(gathered):
+        gp[k] = _dev_tensor(g, torch.bfloat16, plan.N_pad, f"gathered[{k}]")
+    mp = _dev_tensor(master, torch.float32, n, "master")
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
+    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
+    dev = master.device
+    with torch.cuda.device(dev):
+        rc = _lib.zero3_reduce_adamw_gather(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp, gp,
+                                            len(gathered), reduce_dtype, C.byref(hp),
+                                            _stream_handle(stream, dev))
+    _check(rc, "zero3_reduce_adamw_gather")
 
 
 def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Optional[torch.Tensor] = None,

@@ -15,7 +15,8 @@
  *   - Device pointers are plain CUDA global-memory addresses on the current
  *     device.  The caller owns and allocates every device buffer; the library
  *     never allocates, frees or keeps device memory.  Host arrays of device
- *     pointers (contrib, shards, tensor_out) are read during the call only.
+ *     pointers (contrib, gathered, shards, tensor_out) are read during the
+ *     call only.
  *   - Device work is enqueued on `cuda_stream` (a cudaStream_t; NULL means the
  *     legacy default stream) and the call returns without synchronising.
  *     Argument and alignment errors are reported synchronously, before any
@@ -56,6 +57,9 @@ enum {
 
 /* Largest number of simulated ranks D one call accepts. */
 #define Z3_D_MAX 64
+
+/* Largest number of gathered blocks zero3_reduce_adamw_gather writes in one call. */
+#define Z3_GATHER_MAX 8
 
 /* Reduce dtype, the MixedPrecision policy's reduce_dtype ([P1] §2 uses
  * bfloat16; [P3] "Mixed Precision: Cutting Memory in Half" uses float32). */
@@ -187,6 +191,37 @@ Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const uint16_t* co
                               int32_t contrib_layout, float* master, float* exp_avg,
                               float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
                               const z3_adamw* hp, void* cuda_stream);
+
+/* ------------------------ reduce-scatter + AdamW + cast + all-gather, fused
+ * zero3_reduce_adamw_gather: zero3_reduce_adamw whose kernel also stores each
+ * new bf16 working weight straight into its place in n_gathered whole padded
+ * blocks: the value of rank r's owned element j goes to gathered[k][r*S + j]
+ * for every k.  This is the all-gather's data movement ([P3] "AllGather vs
+ * AllReduce": afterwards every GPU holds [A, B, C, D]; [P2] §3: rank r sends
+ * its updated P_r slice to all other ranks) done by the kernel that produces
+ * the data, so no separate pass reads the shards back.  It is the per-rank
+ * step of ZeRO-1 and ZeRO-2, which keep the bf16 working weights replicated
+ * and all-gather them at the end of every step ([P2] §3, §4); ZeRO-3 instead
+ * gathers each block just before it runs (zero3_gather_block, [P2] §5.1).
+ *   gathered    host array of n_gathered (1..Z3_GATHER_MAX) device pointers,
+ *               each a bf16 block of N_pad elements.  Only the positions of
+ *               the partitions this call updates are written (all of them for
+ *               rank = -1, [r*S, (r+1)*S) for rank r).  A pointer may address
+ *               any memory this device can store to with plain stores (its
+ *               own, or another GPU's mapped through peer access).
+ *   work_bf16   as in zero3_reduce_adamw, or NULL to write the gathered blocks
+ *               only.
+ * Every other argument, the arithmetic and the results are those of
+ * zero3_reduce_adamw; the vector path also needs every gathered pointer at
+ * its partition offset 16-byte aligned.
+ * Errors: those of zero3_reduce_adamw, plus Z3_EINVAL for n_gathered outside
+ * [1, Z3_GATHER_MAX], a NULL gathered pointer, or a gathered block that
+ * overlaps another output or a contribution. */
+Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                     int32_t contrib_layout, float* master, float* exp_avg,
+                                     float* exp_avg_sq, uint16_t* work_bf16, uint16_t* const* gathered,
+                                     int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
+                                     void* cuda_stream);
 
 /* ------------------------------------------------ all-gather + unflatten
  * zero3_gather_block: the all-gather's data movement ([P3] "AllGather vs

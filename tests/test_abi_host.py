@@ -33,7 +33,8 @@ def test_library_exports_every_declared_symbol():
     names = declared_symbols()
     assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
                             "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
-                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_gather_block"]), names
+                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_reduce_adamw_gather",
+                            "zero3_gather_block"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -187,6 +188,31 @@ def test_reduce_adamw_argument_errors():
     S = p.S
     base = P16 * 1000
     assert call_reduce(p, rank=1, contrib=[base] * 4, ptrs=[base + 2 * S, P16 * 20, P16 * 30, P16 * 40]) == E
+
+
+def call_fused(plan, gathered, work=P16 * 4, rank=-1, n=None):
+    D = plan.D
+    arr = (C.c_void_p * D)(*[P16 * (100 + d) for d in range(D)])
+    ga = (C.c_void_p * max(1, len(gathered)))(*gathered)
+    hp = z3.adamw(step=1)
+    return z3.lib().zero3_reduce_adamw_gather(plan.handle, rank, arr, 0, C.c_void_p(P16 * 1), C.c_void_p(P16 * 2),
+                                              C.c_void_p(P16 * 3), None if work is None else C.c_void_p(work), ga,
+                                              len(gathered) if n is None else n, 0, C.byref(hp), None)
+
+
+def test_reduce_adamw_gather_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)
+    E = z3.Z3_EINVAL
+    far = P16 * 5000
+    assert call_fused(p, [far], n=0) == E                         # at least one gathered block
+    assert call_fused(p, [far] * 9) == E                          # at most Z3_GATHER_MAX
+    assert call_fused(p, [far, 0]) == E                           # a NULL gathered block
+    assert call_fused(p, [far + 1]) == z3.Z3_EALIGN
+    assert call_fused(p, [far, far + 2]) == E                     # gathered blocks overlap
+    assert call_fused(p, [P16 * 3]) == E                          # over exp_avg_sq
+    assert call_fused(p, [P16 * 100]) == E                        # over a contribution
+    e = z3.zero3_plan([], 4, 8)
+    assert call_fused(e, [far], work=None) == z3.Z3_OK            # empty plan, work may be NULL
 
 
 def test_reduce_adamw_empty_plan_is_a_no_op():

@@ -147,6 +147,71 @@ def test_empty_plan_and_stream_argument(z3):
     assert torch.equal(p, ref[0]) and torch.equal(w.view(torch.int16), ref[3].view(torch.int16))
 
 
+# ------------------------------------------- fused all-gather (ZeRO-1/2 step)
+SENTINEL = 0x7FAB  # a bf16 NaN pattern the kernel never produces
+
+
+def run_fused(z3, numels, D, A, rank, layout, mode, n_gathered, with_work, steps=3, skew=0, seed=5):
+    plan = z3.zero3_plan([(k,) for k in numels], D, A)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    n = N_pad if rank < 0 else S
+    p_full, _, _ = state_init(N, N_pad, seed)
+    p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
+    gp = Guarded(n, torch.float32, skew, fill=p0)
+    gm = Guarded(n, torch.float32, 0, fill=torch.zeros(n, device="cuda"))
+    gv = Guarded(n, torch.float32, 0, fill=torch.zeros(n, device="cuda"))
+    gw = Guarded(n, torch.bfloat16, skew, fill=torch.zeros(n, device="cuda", dtype=torch.bfloat16)) \
+        if with_work else None
+    gg = []
+    for k in range(n_gathered):
+        g = Guarded(N_pad, torch.bfloat16, skew if k == 0 else 0)
+        g.t.view(torch.int16).fill_(SENTINEL)
+        gg.append(g)
+    hp_, hm, hv = f32_host(p0).copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+    hw = np.zeros(n, np.uint16)
+    lo = 0 if rank < 0 else rank * S
+    for t in range(1, steps + 1):
+        contribs = synth.contributions(D, N, N_pad, seed=seed, step=t, sigma=1e-3, device="cuda")
+        if layout == z3.Z3_CONTRIB_OWNED:
+            contribs = [c[rank * S:(rank + 1) * S].clone() for c in contribs]
+        z3.zero3_reduce_adamw_gather(plan, rank, contribs, gp.t, gm.t, gv.t, None if gw is None else gw.t,
+                                     [g.t for g in gg], z3.adamw(**hp_for(t)), contrib_layout=layout,
+                                     reduce_dtype=mode)
+        oracle.reduce_adamw([synth.bf16_bits(c) for c in contribs], S, rank, hp_, hm, hv, hw, oracle_hp(t),
+                            layout=layout, reduce_dtype=mode)
+        torch.cuda.synchronize()
+        what = f"fused numels={numels} D={D} rank={rank} layout={layout} mode={mode} ng={n_gathered} step={t}"
+        assert_f32_parity(f32_host(gp.t), hp_, "master " + what)
+        assert_f32_parity(f32_host(gm.t), hm, "exp_avg " + what)
+        assert_f32_parity(f32_host(gv.t), hv, "exp_avg_sq " + what)
+        if gw is not None:
+            assert_bf16_parity(synth.bf16_bits(gw.t), hw, "work_bf16 " + what)
+            assert gw.guards_intact()
+        for k, g in enumerate(gg):
+            bits = synth.bf16_bits(g.t)
+            assert_bf16_parity(bits[lo:lo + n], hw, f"gathered[{k}] " + what)
+            rest = np.concatenate([bits[:lo], bits[lo + n:]])
+            assert (rest == SENTINEL).all(), "a gathered position outside the updated partitions was written"
+            assert g.guards_intact(), f"canary of gathered[{k}] " + what
+        for g in (gp, gm, gv):
+            assert g.guards_intact()
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("numels,D,A", [([300, 77, 1000], 4, 8), ([123457], 8, 128), ([13], 3, 1),
+                                        ([4097, 33], 32, 128)])
+def test_fused_gather_matches_oracle(z3, numels, D, A, mode):
+    run_fused(z3, numels, D, A, -1, z3.Z3_CONTRIB_FULL, mode, 1, with_work=False)
+    run_fused(z3, numels, D, A, -1, z3.Z3_CONTRIB_FULL, mode, 3, with_work=True)
+    run_fused(z3, numels, D, A, D - 1, z3.Z3_CONTRIB_FULL, mode, 2, with_work=True)
+    run_fused(z3, numels, D, A, D // 2, z3.Z3_CONTRIB_OWNED, mode, 8, with_work=False)
+
+
+def test_fused_gather_misaligned_scalar_path(z3):
+    run_fused(z3, [3000, 17], 4, 8, -1, z3.Z3_CONTRIB_FULL, 0, 2, with_work=True, skew=1)
+    run_fused(z3, [3000, 17], 4, 8, 2, z3.Z3_CONTRIB_OWNED, 1, 1, with_work=False, skew=1)
+
+
 # ------------------------------------------------------------- full sizes
 def sample_indices(n: int, S: int, D: int, k: int, seed: int) -> torch.Tensor:
     rng = np.random.default_rng(seed)
