@@ -33,7 +33,7 @@
  *         Fit", sections "AllGather vs AllReduce" and "Mixed Precision:
  *         Cutting Memory in Half".
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - flat layout: tensors packed row-major in list order, no padding between
  *     tensors, zero padding at the tail to a multiple of D*A elements;
  *   - the reduction sums ranks 0..D-1 left to right, starting from rank 0's
