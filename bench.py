@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
+    ap.add_argument("--unflatten-copy", action="store_true",
+                    help="the gather also copies every tensor into its own buffer (straight from the shards)")
     ap.add_argument("--drift", action="store_true",
                     help="report the drift of the bf16-reduce path against the fp32-reduce path")
     ap.add_argument("--drift-elements", type=int, default=1 << 24)
@@ -230,7 +232,7 @@ class BlockRunner:
     stage 1 or 2: one kernel does the reduce, AdamW, cast and the all-gather into
     the replicated bf16 weights (the flat block), with no separate shard."""
 
-    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3):
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
@@ -247,14 +249,18 @@ class BlockRunner:
         self.stream = torch.cuda.current_stream(dev)
         self.step_no = 0
         self.stage = stage
+        self.tensor_out = ([torch.empty(shape, dtype=torch.bfloat16, device=dev) for shape in self.shapes]
+                           if unflatten_copy and stage == 3 else None)
         self.units_per_step = self.N_pad                       # owned params, all ranks
         self.k1_launches_per_step = 1
         self.k1_bytes_per_launch = (2 * D + 26) * self.N_pad   # stage 1/2: the bf16 goes to the block instead
-        self.step_bytes = self.k1_bytes_per_launch + (4 * self.N_pad if stage == 3 else 0)
-        self.launches_per_step = 2 if stage == 3 else 1
+        self.step_bytes = self.k1_bytes_per_launch + (4 * self.N_pad if stage == 3 else 0) + \
+            (4 * self.N if self.tensor_out is not None else 0)
+        self.launches_per_step = (2 + (1 if self.tensor_out is not None else 0)) if stage == 3 else 1
         self.k1_name = (f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}"
                         f"{', gather' if stage != 3 else ''}>")
-        what = ("fused reduce/AdamW/cast over all %d partitions + gather into the flat block" % D if stage == 3
+        what = ("fused reduce/AdamW/cast over all %d partitions + gather into the flat block%s" %
+                (D, " and into one buffer per tensor" if self.tensor_out is not None else "") if stage == 3
                 else "one kernel: reduce/AdamW/cast over all %d partitions writing the replicated bf16 "
                      "weights in place of the gather (ZeRO-%d)" % (D, stage))
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
@@ -290,7 +296,7 @@ class BlockRunner:
         if k1_events is not None:
             k1_events[0][1].record(self.stream)
         # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
-        z3.zero3_gather_block(pl, self.shards, flat, None, stream=self.stream)
+        z3.zero3_gather_block(pl, self.shards, flat, self.tensor_out, stream=self.stream)
         return pl.views(flat)
 
     def e2e_setup(self):
@@ -436,7 +442,7 @@ def run_ours(args):
         R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev)
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
-                        stage=args.stage)
+                        stage=args.stage, unflatten_copy=args.unflatten_copy)
     stream = R.stream
 
     for _ in range(args.warmup):
