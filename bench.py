@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step's launches in a CUDA graph once and replay it every step")
     ap.add_argument("--unflatten-copy", action="store_true",
                     help="the gather also copies every tensor into its own buffer (straight from the shards)")
     ap.add_argument("--drift", action="store_true",
@@ -232,11 +234,13 @@ class BlockRunner:
     stage 1 or 2: one kernel does the reduce, AdamW, cast and the all-gather into
     the replicated bf16 weights (the flat block), with no separate shard."""
 
-    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False):
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
+                 graph=False):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
         self.shapes = [s for _, s in w["tensors"]]
+        self.specs = z3.tensor_specs(self.shapes)       # the step's input: the block's tensor list
         plan = z3.zero3_plan(self.shapes, D, synth.ALIGN)
         self.N, self.N_pad, self.S = plan.N, plan.N_pad, plan.S
         self.contribs = synth.contributions(D, self.N, self.N_pad, seed=seed, step=1, sigma=w["sigma"],
@@ -263,6 +267,16 @@ class BlockRunner:
                 (D, " and into one buffer per tensor" if self.tensor_out is not None else "") if stage == 3
                 else "one kernel: reduce/AdamW/cast over all %d partitions writing the replicated bf16 "
                      "weights in place of the gather (ZeRO-%d)" % (D, stage))
+        self.graphed = None
+        if graph:
+            from fsdp_sharded_mixed_flat_b200.graph import GraphedStep
+            self.graphed = GraphedStep(plan, self.contribs, self.master, self.exp_avg, self.exp_avg_sq,
+                                       self.work if stage == 3 else None, self.flat, stage=stage,
+                                       reduce_dtype=reduce_dtype)
+            what += "; captured once in a CUDA graph and replayed (scalars from device memory)"
+            # events around the replay time every kernel of the graph
+            self.k1_bytes_per_launch = self.step_bytes
+            self.k1_name = "CUDA graph of the step (%s)" % ("fused kernel + gather" if stage == 3 else "fused kernel")
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
                      f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
                      f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + {what}")
@@ -278,9 +292,16 @@ class BlockRunner:
         contribs = self.contribs if contribs is None else contribs
         flat = self.flat if flat is None else flat
         # a1 + a2: host-side plan and ledger of the block (microseconds, overlapped with the GPU)
-        pl = z3.zero3_plan(self.shapes, self.D, self.synth.ALIGN)
+        pl = z3.Plan(self.shapes, self.D, self.synth.ALIGN, specs=self.specs)
         z3.zero3_memory_bytes(pl.N, self.D, self.stage)
         hp = self.hp()
+        if self.graphed is not None and contribs is self.contribs and flat is self.flat:
+            if k1_events is not None:
+                k1_events[0][0].record(self.stream)
+            self.graphed.step(hp)
+            if k1_events is not None:
+                k1_events[0][1].record(self.stream)
+            return self.views(pl, flat)
         if k1_events is not None:
             k1_events[0][0].record(self.stream)
         if self.stage != 3:
@@ -289,7 +310,7 @@ class BlockRunner:
                                          [flat], hp, reduce_dtype=self.mode, stream=self.stream)
             if k1_events is not None:
                 k1_events[0][1].record(self.stream)
-            return pl.views(flat)
+            return self.views(pl, flat)
         # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
         z3.zero3_reduce_adamw(pl, -1, contribs, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
                               reduce_dtype=self.mode, stream=self.stream)
@@ -297,7 +318,16 @@ class BlockRunner:
             k1_events[0][1].record(self.stream)
         # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
         z3.zero3_gather_block(pl, self.shards, flat, self.tensor_out, stream=self.stream)
-        return pl.views(flat)
+        return self.views(pl, flat)
+
+    def views(self, pl, flat):
+        """a6: the zero-copy per-tensor views of the gathered block.  They alias the
+        same buffer every step, so they are built once per buffer."""
+        key = flat.data_ptr()
+        cache = self.__dict__.setdefault("_views", {})
+        if key not in cache:
+            cache[key] = pl.views(flat)
+        return cache[key]
 
     def e2e_setup(self):
         """Pinned host copies of the contributions and of the gathered block, and a
@@ -437,12 +467,14 @@ def run_ours(args):
     from fsdp_sharded_mixed_flat_b200 import zero3 as z3
 
     mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
+    if args.graph and (args.unflatten_copy or args.workload == "llama70b_shard"):
+        raise SystemExit("--graph covers the block step without --unflatten-copy")
     seed = 1000 + rank  # every rank runs its own block
     if args.workload == "llama70b_shard":
         R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev)
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
-                        stage=args.stage, unflatten_copy=args.unflatten_copy)
+                        stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph)
     stream = R.stream
 
     for _ in range(args.warmup):
@@ -526,7 +558,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world} (one block per GPU, no collective)"},
         "step_hbm_gbs": R.step_bytes * args.steps * world / job_secs / 1e9,
         "kernels": {"reduce_adamw_ms": 1e3 * k1_avg_s, "reduce_adamw_gbs": k1_gbs,
-                    "reduce_adamw_params_per_s": (R.k1_bytes_per_launch / (2 * R.D + 26)) / k1_avg_s,
+                    "reduce_adamw_params_per_s": R.units_per_step / R.k1_launches_per_step / k1_avg_s,
                     "reduce_adamw_launches_per_step": R.k1_launches_per_step,
                     "rest_of_step_ms": max(0.0, 1e3 * secs / args.steps - 1e3 * k1_avg_s * R.k1_launches_per_step)},
         "roofline": {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",

@@ -37,12 +37,15 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 
 #include "plan_impl.h"
 #include "zero3.h"
 
 namespace {
 
+// The eight fp32 scalars of one AdamW step, in the order the C ABI documents
+// for zero3_step_scalars.
 struct AdamScalars {
     float step_size;     // lr / (1 - b1^t)
     float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
@@ -61,8 +64,28 @@ struct K1Args {
     int64_t n;                    // elements in this launch
     int32_t D;
     float inv_D;                  // fp32 nearest to 1/D
-    AdamScalars s;
+    AdamScalars s;                // this step's scalars (unless s_dev is used)
+    const AdamScalars* s_dev;     // device copy of the scalars (the DEVS kernels)
 };
+
+static_assert(sizeof(AdamScalars) == Z3_SCALARS * sizeof(float), "scalar layout");
+
+// Host computation of one step's scalars: binary64, each rounded to fp32 once.
+AdamScalars step_scalars(const z3_adamw* hp) {
+    AdamScalars s;
+    const double t = double(hp->step);
+    const double bc1 = 1.0 - std::pow(hp->beta1, t);
+    const double bc2 = 1.0 - std::pow(hp->beta2, t);
+    s.step_size = float(hp->lr / bc1);
+    s.inv_sqrt_bc2 = float(1.0 / std::sqrt(bc2));
+    s.decay = float(1.0 - hp->lr * hp->weight_decay);
+    s.b1 = float(hp->beta1);
+    s.omb1 = float(1.0 - hp->beta1);
+    s.b2 = float(hp->beta2);
+    s.omb2 = float(1.0 - hp->beta2);
+    s.eps = float(hp->eps);
+    return s;
+}
 
 constexpr int kThreads = 256;
 constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: caps registers at 85 per thread
@@ -181,7 +204,7 @@ __device__ __forceinline__ float finish(float acc, float inv_D) {
 
 // One element on the scalar path (tails and misaligned buffers).
 template <int MODE, bool GATHER>
-__device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
+__device__ __forceinline__ void scalar_elem(const K1Args& a, const AdamScalars& sc, int64_t i) {
     float acc = bf16_of(a.c[0][i]);
     for (int d = 1; d < a.D; ++d) {
         const float x = bf16_of(a.c[d][i]);
@@ -189,7 +212,7 @@ __device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
     }
     const float g = finish<MODE>(acc, a.inv_D);
     float p = a.p[i], m = a.m[i], v = a.v[i];
-    adamw_elem(a.s, g, p, m, v);
+    adamw_elem(sc, g, p, m, v);
     a.p[i] = p;
     a.m[i] = m;
     a.v[i] = v;
@@ -203,7 +226,7 @@ __device__ __forceinline__ void scalar_elem(const K1Args& a, int64_t i) {
 // GATHER: the bf16 result also goes to every gathered block (the all-gather's
 // data movement done by the producer of the data).
 template <int MODE, int DT, bool GATHER>
-__device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
+__device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc, int64_t e) {
     const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
     const float4 p1 = ld16(reinterpret_cast<const float4*>(a.p + e + 4));
     const float4 m0 = ld16(reinterpret_cast<const float4*>(a.m + e));
@@ -216,7 +239,7 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
     float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
     float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-    for (int k = 0; k < 8; ++k) adamw_elem(a.s, g[k], p[k], m[k], v[k]);
+    for (int k = 0; k < 8; ++k) adamw_elem(sc, g[k], p[k], m[k], v[k]);
     st16(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
     st16(reinterpret_cast<float4*>(a.p + e + 4), make_float4(p[4], p[5], p[6], p[7]));
     st16(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
@@ -233,14 +256,23 @@ __device__ __forceinline__ void process8(const K1Args& a, int64_t e) {
     }
 }
 
-// Vector kernel: every pointer 16-byte aligned.  The grid covers the whole
-// range (kChunks 8-element chunks per thread, consecutive threads on
+// The scalars of this step, (DEVS) read from device memory, so that a captured
+// CUDA graph can be replayed step after step with only the 32-byte scalar
+// buffer rewritten in between.
+__device__ __forceinline__ AdamScalars load_scalars(const AdamScalars* p) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    return AdamScalars{x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+}
+
+// Vector kernel body: every pointer 16-byte aligned.  The grid covers the
+// whole range (kChunks 8-element chunks per thread, consecutive threads on
 // consecutive chunks), so the block scheduler hands blocks to whichever SM is
 // free and every SM keeps streaming to the end; the outer loop only runs more
 // than once when the range exceeds the largest grid.  The last n % 8 elements
 // go through the scalar path.
 template <int MODE, int DT, bool GATHER>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
+__device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc) {
     const int64_t n8 = a.n >> 3;
     const int64_t span = int64_t(kThreads) * kChunks;
     const int64_t step = int64_t(gridDim.x) * span;
@@ -248,56 +280,92 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const
 #pragma unroll
         for (int k = 0; k < kChunks; ++k) {
             const int64_t q = first + int64_t(k) * kThreads;
-            if (q < n8) process8<MODE, DT, GATHER>(a, q << 3);
+            if (q < n8) process8<MODE, DT, GATHER>(a, sc, q << 3);
         }
     }
     const int64_t tail = (n8 << 3) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    if (tail < a.n) scalar_elem<MODE, GATHER>(a, tail);
+    if (tail < a.n) scalar_elem<MODE, GATHER>(a, sc, tail);
+}
+
+template <int MODE, int DT, bool GATHER, bool DEVS>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
+    if constexpr (DEVS) {
+        const AdamScalars sc = load_scalars(a.s_dev);
+        vec_body<MODE, DT, GATHER>(a, sc);
+    } else {
+        vec_body<MODE, DT, GATHER>(a, a.s);   // the scalars stay in the parameter block
+    }
 }
 
 // Scalar kernel: any element-aligned pointers.
 template <int MODE, bool GATHER>
-__global__ void __launch_bounds__(kThreads) k_reduce_adamw_scalar(const __grid_constant__ K1Args a) {
+__device__ __forceinline__ void scalar_body(const K1Args& a, const AdamScalars& sc) {
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < a.n; i += stride)
-        scalar_elem<MODE, GATHER>(a, i);
+        scalar_elem<MODE, GATHER>(a, sc, i);
+}
+
+template <int MODE, bool GATHER, bool DEVS>
+__global__ void __launch_bounds__(kThreads) k_reduce_adamw_scalar(const __grid_constant__ K1Args a) {
+    if constexpr (DEVS) {
+        const AdamScalars sc = load_scalars(a.s_dev);
+        scalar_body<MODE, GATHER>(a, sc);
+    } else {
+        scalar_body<MODE, GATHER>(a, a.s);
+    }
 }
 
 using KernelFn = void (*)(K1Args);
 
-template <int MODE, bool GATHER>
+template <int MODE, bool GATHER, bool DEVS>
 KernelFn pick_vec(int D) {
     switch (D) {
-    case 1: return k_reduce_adamw_vec<MODE, 1, GATHER>;
-    case 2: return k_reduce_adamw_vec<MODE, 2, GATHER>;
-    case 4: return k_reduce_adamw_vec<MODE, 4, GATHER>;
-    case 8: return k_reduce_adamw_vec<MODE, 8, GATHER>;
-    case 16: return k_reduce_adamw_vec<MODE, 16, GATHER>;
-    case 32: return k_reduce_adamw_vec<MODE, 32, GATHER>;
-    default: return k_reduce_adamw_vec<MODE, 0, GATHER>;
+    case 1: return k_reduce_adamw_vec<MODE, 1, GATHER, DEVS>;
+    case 2: return k_reduce_adamw_vec<MODE, 2, GATHER, DEVS>;
+    case 4: return k_reduce_adamw_vec<MODE, 4, GATHER, DEVS>;
+    case 8: return k_reduce_adamw_vec<MODE, 8, GATHER, DEVS>;
+    case 16: return k_reduce_adamw_vec<MODE, 16, GATHER, DEVS>;
+    case 32: return k_reduce_adamw_vec<MODE, 32, GATHER, DEVS>;
+    default: return k_reduce_adamw_vec<MODE, 0, GATHER, DEVS>;
     }
 }
 
-template <bool GATHER>
+template <bool GATHER, bool DEVS>
 KernelFn pick(bool vec, int32_t reduce_dtype, int D) {
     if (vec)
-        return reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32, GATHER>(D)
-                                              : pick_vec<Z3_REDUCE_BF16, GATHER>(D);
-    return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, GATHER>
-                                          : k_reduce_adamw_scalar<Z3_REDUCE_BF16, GATHER>;
+        return reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32, GATHER, DEVS>(D)
+                                              : pick_vec<Z3_REDUCE_BF16, GATHER, DEVS>(D);
+    return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, GATHER, DEVS>
+                                          : k_reduce_adamw_scalar<Z3_REDUCE_BF16, GATHER, DEVS>;
 }
 
+KernelFn pick_any(bool gather, bool devs, bool vec, int32_t reduce_dtype, int D) {
+    if (gather)
+        return devs ? pick<true, true>(vec, reduce_dtype, D) : pick<true, false>(vec, reduce_dtype, D);
+    return devs ? pick<false, true>(vec, reduce_dtype, D) : pick<false, false>(vec, reduce_dtype, D);
+}
+
+bool hp_valid(const z3_adamw* hp);
+
 bool is_finite(double x) { return std::isfinite(x); }
+
+bool hp_valid(const z3_adamw* hp) {
+    return hp != nullptr && hp->step >= 1 && is_finite(hp->lr) && is_finite(hp->beta1) &&
+           is_finite(hp->beta2) && is_finite(hp->eps) && is_finite(hp->weight_decay) && hp->beta1 >= 0.0 &&
+           hp->beta1 < 1.0 && hp->beta2 >= 0.0 && hp->beta2 < 1.0;
+}
 
 // Validation and launch shared by both entry points.  `gathered` holds
 // n_gathered whole padded blocks (0 for the plain entry point); `work_bf16`
 // may be null only when n_gathered > 0.
+// Exactly one of hp (scalars computed here, passed by value) and dev_scalars
+// (read by the kernel from device memory) is non-null.
 int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, int32_t contrib_layout,
               float* master, float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
               uint16_t* const* gathered, int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
-              void* cuda_stream) {
+              const float* dev_scalars, void* cuda_stream) {
     // ---- arguments
-    if (p == nullptr || contrib == nullptr || hp == nullptr) return Z3_EINVAL;
+    if (p == nullptr || contrib == nullptr || (hp == nullptr) == (dev_scalars == nullptr)) return Z3_EINVAL;
     const int32_t D = p->D;
     if (rank < -1 || rank >= D) return Z3_EINVAL;
     if (contrib_layout != Z3_CONTRIB_FULL && contrib_layout != Z3_CONTRIB_OWNED) return Z3_EINVAL;
@@ -312,10 +380,8 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
         if (contrib[d] == nullptr) return Z3_EINVAL;
     for (int32_t k = 0; k < n_gathered; ++k)
         if (gathered[k] == nullptr) return Z3_EINVAL;
-    if (hp->step < 1 || !is_finite(hp->lr) || !is_finite(hp->beta1) || !is_finite(hp->beta2) ||
-        !is_finite(hp->eps) || !is_finite(hp->weight_decay) || hp->beta1 < 0.0 || hp->beta1 >= 1.0 ||
-        hp->beta2 < 0.0 || hp->beta2 >= 1.0)
-        return Z3_EINVAL;
+    if (hp != nullptr && !hp_valid(hp)) return Z3_EINVAL;
+    if (dev_scalars != nullptr && !z3::aligned(dev_scalars, 16)) return Z3_EALIGN;
     if (!z3::aligned(master, 4) || !z3::aligned(exp_avg, 4) || !z3::aligned(exp_avg_sq, 4) ||
         !z3::aligned(work_bf16, 2))
         return Z3_EALIGN;
@@ -348,17 +414,8 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
 
     // ---- host scalars: double, then rounded to fp32 once
     K1Args a;
-    const double t = double(hp->step);
-    const double bc1 = 1.0 - std::pow(hp->beta1, t);
-    const double bc2 = 1.0 - std::pow(hp->beta2, t);
-    a.s.step_size = float(hp->lr / bc1);
-    a.s.inv_sqrt_bc2 = float(1.0 / std::sqrt(bc2));
-    a.s.decay = float(1.0 - hp->lr * hp->weight_decay);
-    a.s.b1 = float(hp->beta1);
-    a.s.omb1 = float(1.0 - hp->beta1);
-    a.s.b2 = float(hp->beta2);
-    a.s.omb2 = float(1.0 - hp->beta2);
-    a.s.eps = float(hp->eps);
+    a.s = hp != nullptr ? step_scalars(hp) : AdamScalars{};
+    a.s_dev = reinterpret_cast<const AdamScalars*>(dev_scalars);
     a.inv_D = float(1.0 / double(D));
     a.D = D;
     a.n = n;
@@ -380,7 +437,7 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
 
     // ---- launch: the vector kernel's grid covers the range; the scalar kernel
     // runs a whole number of resident waves with a grid-stride loop
-    const KernelFn fn = n_gathered > 0 ? pick<true>(vec, reduce_dtype, D) : pick<false>(vec, reduce_dtype, D);
+    const KernelFn fn = pick_any(n_gathered > 0, dev_scalars != nullptr, vec, reduce_dtype, D);
     int64_t blocks;
     if (vec) {
         const int64_t span = int64_t(kThreads) * kChunks;
@@ -408,8 +465,9 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
                                          int32_t contrib_layout, float* master, float* exp_avg,
                                          float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
                                          const z3_adamw* hp, void* cuda_stream) {
+    if (hp == nullptr) return Z3_EINVAL;
     return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, nullptr, 0,
-                     reduce_dtype, hp, cuda_stream);
+                     reduce_dtype, hp, nullptr, cuda_stream);
 }
 
 extern "C" Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
@@ -417,7 +475,24 @@ extern "C" Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, 
                                                 float* exp_avg_sq, uint16_t* work_bf16,
                                                 uint16_t* const* gathered, int32_t n_gathered,
                                                 int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream) {
-    if (n_gathered < 1) return Z3_EINVAL;
+    if (n_gathered < 1 || hp == nullptr) return Z3_EINVAL;
     return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
-                     n_gathered, reduce_dtype, hp, cuda_stream);
+                     n_gathered, reduce_dtype, hp, nullptr, cuda_stream);
+}
+
+extern "C" Z3_API int zero3_step_scalars(const z3_adamw* hp, float* out) {
+    if (out == nullptr || !hp_valid(hp)) return Z3_EINVAL;
+    const AdamScalars s = step_scalars(hp);
+    std::memcpy(out, &s, sizeof s);
+    return Z3_OK;
+}
+
+extern "C" Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                             int32_t contrib_layout, float* master, float* exp_avg,
+                                             float* exp_avg_sq, uint16_t* work_bf16, uint16_t* const* gathered,
+                                             int32_t n_gathered, int32_t reduce_dtype, const float* scalars,
+                                             void* cuda_stream) {
+    if (scalars == nullptr) return Z3_EINVAL;
+    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
+                     n_gathered, reduce_dtype, nullptr, scalars, cuda_stream);
 }

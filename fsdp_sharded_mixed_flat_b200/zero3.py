@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(HERE, "libzero3.so")
 Z3_OK, Z3_EINVAL, Z3_EALIGN, Z3_ENOMEM, Z3_ECUDA, Z3_EOVERFLOW = 0, -1, -2, -3, -4, -5
 Z3_D_MAX = 64
 Z3_GATHER_MAX = 8
+Z3_SCALARS = 8
 Z3_REDUCE_FP32, Z3_REDUCE_BF16 = 0, 1
 Z3_CONTRIB_FULL, Z3_CONTRIB_OWNED = 0, 1
 Z3_STAGE_DDP, Z3_STAGE_ZERO1, Z3_STAGE_ZERO2, Z3_STAGE_ZERO3 = 0, 1, 2, 3
@@ -68,6 +69,10 @@ def _load() -> C.CDLL:
     L.zero3_reduce_adamw_gather.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
                                             C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw_gather.restype = C.c_int
+    L.zero3_step_scalars.argtypes = [C.POINTER(AdamW), vp]
+    L.zero3_step_scalars.restype = C.c_int
+    L.zero3_reduce_adamw_dev.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+    L.zero3_reduce_adamw_dev.restype = C.c_int
     L.zero3_gather_block.argtypes = [vp, vp, vp, vp, vp]
     L.zero3_gather_block.restype = C.c_int
     return L
@@ -90,23 +95,32 @@ def _check(rc: int, what: str) -> None:
 
 
 # ------------------------------------------------------------------- plan
-class Plan:
-    """A flat-parameter plan (owns the C plan object)."""
+def tensor_specs(shapes: Sequence[Sequence[int]]):
+    """A host array of z3_tensor_spec for the given row-major shapes."""
+    shapes = [tuple(int(x) for x in s) for s in shapes]
+    specs = (TensorSpec * max(1, len(shapes)))()
+    for i, s in enumerate(shapes):
+        if len(s) > 4:
+            raise ValueError("at most 4 dimensions per tensor")
+        numel = 1
+        for x in s:
+            numel *= x
+        specs[i].numel = numel
+        specs[i].ndim = len(s)
+        for k, x in enumerate(s):
+            specs[i].shape[k] = x
+    return specs
 
-    def __init__(self, shapes: Sequence[Sequence[int]], D: int, align_elems: int = 128):
+
+class Plan:
+    """A flat-parameter plan (owns the C plan object).  `specs` may be passed in,
+    prebuilt by tensor_specs(shapes), to re-plan the same block cheaply."""
+
+    def __init__(self, shapes: Sequence[Sequence[int]], D: int, align_elems: int = 128, specs=None):
         self.shapes = [tuple(int(x) for x in s) for s in shapes]
         n = len(self.shapes)
-        specs = (TensorSpec * max(1, n))()
-        for i, s in enumerate(self.shapes):
-            if len(s) > 4:
-                raise ValueError("at most 4 dimensions per tensor")
-            numel = 1
-            for x in s:
-                numel *= x
-            specs[i].numel = numel
-            specs[i].ndim = len(s)
-            for k, x in enumerate(s):
-                specs[i].shape[k] = x
+        if specs is None:
+            specs = tensor_specs(self.shapes)
         h = C.c_void_p()
         _check(_lib.zero3_plan(specs, n, D, align_elems, C.byref(h)), "zero3_plan")
         self._h = h
@@ -116,10 +130,21 @@ class Plan:
                                     C.byref(N_pad), C.byref(S)), "zero3_plan_info")
         self.D, self.n_tensors, self.align_elems = d.value, nt.value, a.value
         self.N, self.N_pad, self.S = N.value, N_pad.value, S.value
-        self.offsets, self.numels = [], []
-        for i in range(n):
-            self.offsets.append(zero3_plan_tensor(self, i)[0])
-            self.numels.append(zero3_plan_tensor(self, i)[1])
+        self._runs = None
+
+    def _tensor_runs(self):
+        if self._runs is None:
+            runs = [zero3_plan_tensor(self, i) for i in range(self.n_tensors)]
+            self._runs = ([o for o, _ in runs], [k for _, k in runs])
+        return self._runs
+
+    @property
+    def offsets(self):
+        return self._tensor_runs()[0]
+
+    @property
+    def numels(self):
+        return self._tensor_runs()[1]
 
     @property
     def handle(self) -> C.c_void_p:
@@ -248,6 +273,51 @@ def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Ten
                                             len(gathered), reduce_dtype, C.byref(hp),
                                             _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw_gather")
+
+
+def zero3_step_scalars(hp: AdamW, out: Optional[int] = None):
+    """The Z3_SCALARS fp32 scalars of one AdamW step.  With `out` (a host address of
+    Z3_SCALARS floats, e.g. a pinned tensor's data_ptr()) they are written there;
+    otherwise they are returned as a list."""
+    if out is not None:
+        _check(_lib.zero3_step_scalars(C.byref(hp), out), "zero3_step_scalars")
+        return None
+    buf = (C.c_float * Z3_SCALARS)()
+    _check(_lib.zero3_step_scalars(C.byref(hp), buf), "zero3_step_scalars")
+    return list(buf)
+
+
+def zero3_reduce_adamw_dev(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], master: torch.Tensor,
+                           exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor, work_bf16: Optional[torch.Tensor],
+                           gathered: Sequence[torch.Tensor], scalars: torch.Tensor,
+                           contrib_layout: int = Z3_CONTRIB_FULL, reduce_dtype: int = Z3_REDUCE_FP32,
+                           stream=None) -> None:
+    """The fused kernel reading the step's scalars from `scalars` (a CUDA float32
+    tensor of Z3_SCALARS elements), so that the launch can be captured in a CUDA
+    graph (see include/zero3.h)."""
+    if len(contrib) != plan.D:
+        raise ValueError(f"need {plan.D} contributions, got {len(contrib)}")
+    if len(gathered) > Z3_GATHER_MAX:
+        raise ValueError(f"at most {Z3_GATHER_MAX} gathered blocks")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * plan.D)()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    gp = (C.c_void_p * max(1, len(gathered)))()
+    for k, g in enumerate(gathered):
+        gp[k] = _dev_tensor(g, torch.bfloat16, plan.N_pad, f"gathered[{k}]")
+    sp = _dev_tensor(scalars, torch.float32, Z3_SCALARS, "scalars")
+    mp = _dev_tensor(master, torch.float32, n, "master")
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
+    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
+    dev = master.device
+    with torch.cuda.device(dev):
+        rc = _lib.zero3_reduce_adamw_dev(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
+                                         gp if gathered else None, len(gathered), reduce_dtype, sp,
+                                         _stream_handle(stream, dev))
+    _check(rc, "zero3_reduce_adamw_dev")
 
 
 def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Optional[torch.Tensor] = None,

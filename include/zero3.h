@@ -61,6 +61,9 @@ enum {
 /* Largest number of gathered blocks zero3_reduce_adamw_gather writes in one call. */
 #define Z3_GATHER_MAX 8
 
+/* Number of fp32 scalars zero3_step_scalars writes. */
+#define Z3_SCALARS 8
+
 /* Reduce dtype, the MixedPrecision policy's reduce_dtype ([P1] §2 uses
  * bfloat16; [P3] "Mixed Precision: Cutting Memory in Half" uses float32). */
 enum {
@@ -222,6 +225,33 @@ Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint1
                                      float* exp_avg_sq, uint16_t* work_bf16, uint16_t* const* gathered,
                                      int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
                                      void* cuda_stream);
+
+/* ------------------------------------- scalars in device memory (graphs)
+ * zero3_step_scalars: the Z3_SCALARS fp32 scalars of one AdamW step, formed in
+ * binary64 from *hp and rounded to fp32 once, exactly as zero3_reduce_adamw
+ * forms them, in this order:
+ *   [0] lr / (1 - beta1^t)    [1] 1 / sqrt(1 - beta2^t)   [2] 1 - lr * weight_decay
+ *   [3] beta1   [4] 1 - beta1   [5] beta2   [6] 1 - beta2   [7] eps
+ *   out: host array of Z3_SCALARS floats.
+ * Errors: Z3_EINVAL (out or hp NULL, hp->step < 1, a value not finite, a beta
+ * outside [0, 1)).
+ *
+ * zero3_reduce_adamw_dev: zero3_reduce_adamw (n_gathered = 0) or
+ * zero3_reduce_adamw_gather (n_gathered >= 1, up to Z3_GATHER_MAX) whose kernel
+ * reads the step's scalars from `scalars`, a device array of Z3_SCALARS floats
+ * (16-byte aligned) laid out as above, instead of taking them as launch
+ * arguments.  Nothing else in the launch depends on the step, so the launch can
+ * be captured into a CUDA graph once and the graph replayed every step, with
+ * only the scalars rewritten (stream-ordered) before each replay.  The
+ * arithmetic and results are those of zero3_reduce_adamw.  work_bf16 may be
+ * NULL only when n_gathered >= 1.
+ * Errors: those of zero3_reduce_adamw_gather, Z3_EINVAL (scalars NULL),
+ * Z3_EALIGN (scalars not 16-byte aligned). */
+Z3_API int zero3_step_scalars(const z3_adamw* hp, float* out);
+Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                  int32_t contrib_layout, float* master, float* exp_avg, float* exp_avg_sq,
+                                  uint16_t* work_bf16, uint16_t* const* gathered, int32_t n_gathered,
+                                  int32_t reduce_dtype, const float* scalars, void* cuda_stream);
 
 /* ------------------------------------------------ all-gather + unflatten
  * zero3_gather_block: the all-gather's data movement ([P3] "AllGather vs

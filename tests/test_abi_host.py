@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
     assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
                             "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
                             "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_reduce_adamw_gather",
-                            "zero3_gather_block"]), names
+                            "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -213,6 +213,46 @@ def test_reduce_adamw_gather_argument_errors():
     assert call_fused(p, [P16 * 100]) == E                        # over a contribution
     e = z3.zero3_plan([], 4, 8)
     assert call_fused(e, [far], work=None) == z3.Z3_OK            # empty plan, work may be NULL
+
+
+def test_step_scalars_match_the_oracle():
+    """The scalars a graph-captured step reads equal the oracle's, bit for bit."""
+    rnd = random.Random(17)
+    cases = [dict(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, step=t) for t in (1, 2, 10, 1000)]
+    cases += [dict(lr=rnd.uniform(1e-6, 1e-2), beta1=rnd.uniform(0, 0.999), beta2=rnd.uniform(0, 0.9999),
+                   eps=10 ** rnd.uniform(-12, -4), weight_decay=rnd.uniform(0, 0.3), step=rnd.randint(1, 10 ** 6))
+              for _ in range(200)]
+    for c in cases:
+        got = np.array(z3.zero3_step_scalars(z3.adamw(**c)), dtype=np.float32)
+        ref = oracle.adamw_consts(oracle.hp(**c))
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32)), c
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_step_scalars(z3.adamw(step=0))
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_step_scalars(z3.adamw(beta2=1.0))
+
+
+def test_reduce_adamw_dev_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)
+    D = p.D
+    arr = (C.c_void_p * D)(*[P16 * (100 + d) for d in range(D)])
+    L = z3.lib()
+
+    def call(scalars, work=P16 * 4, gathered=(), rank=-1):
+        ga = (C.c_void_p * max(1, len(gathered)))(*gathered)
+        return L.zero3_reduce_adamw_dev(p.handle, rank, arr, 0, C.c_void_p(P16), C.c_void_p(P16 * 2),
+                                        C.c_void_p(P16 * 3), None if work is None else C.c_void_p(work),
+                                        ga if gathered else None, len(gathered), 0,
+                                        None if scalars is None else C.c_void_p(scalars), None)
+    assert call(None) == z3.Z3_EINVAL
+    assert call(P16 * 9000 + 4) == z3.Z3_EALIGN                # 16-byte alignment of the scalars
+    assert call(P16 * 9000, work=None) == z3.Z3_EINVAL          # no shard and no gathered block
+    assert call(P16 * 9000, gathered=[P16 * 5000] * 9) == z3.Z3_EINVAL
+    assert call(P16 * 9000, rank=7) == z3.Z3_EINVAL
+    e = z3.zero3_plan([], 4, 8)
+    assert L.zero3_reduce_adamw_dev(e.handle, -1, arr, 0, C.c_void_p(P16), C.c_void_p(P16 * 2),
+                                    C.c_void_p(P16 * 3), C.c_void_p(P16 * 4), None, 0, 0,
+                                    C.c_void_p(P16 * 9000), None) == z3.Z3_OK
 
 
 def test_reduce_adamw_empty_plan_is_a_no_op():
