@@ -56,6 +56,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
+    ap.add_argument("--refill", choices=["copy", "fill"], default="copy",
+                    help="70B shard: each layer's contributions arrive by a device-to-device copy from a "
+                         "pool (read + write) or by a write-only fill of the transient buffer")
     ap.add_argument("--graph", action="store_true",
                     help="capture the step's launches in a CUDA graph once and replay it every step")
     ap.add_argument("--unflatten-copy", action="store_true",
@@ -380,7 +383,7 @@ class ShardRunner:
     owned contributions stream in last to first through two transient buffers
     (copy stream) while the fused kernel runs on the other buffer."""
 
-    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev):
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, refill="copy"):
         import torch
         from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
         w = synth.WORKLOADS["llama70b_layer"]
@@ -404,16 +407,20 @@ class ShardRunner:
         self.units_per_step = L * S                            # owned params of this rank
         self.k1_launches_per_step = L
         self.k1_bytes_per_launch = (2 * D + 26) * S
-        self.refill_bytes = L * 2 * D * S * 2                  # D2D copy: read + write
+        self.refill = refill
+        self.refill_bytes = L * 2 * D * S * (2 if refill == "copy" else 1)   # copy: read + write
         self.step_bytes = L * self.k1_bytes_per_launch + self.refill_bytes
         self.launches_per_step = L
         self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}> (owned layout)"
         self.source = lambda l: self.pool[l & 1]
+        # write-only refill: the transient buffer receives a value, as an NVLink delivery would write it
+        self.fill = (lambda l, buf: buf.fill_(1e-4 * (1 + (l & 7)))) if refill == "fill" else None
         self.desc = (f"rank 0's resident shard of 80 LLaMA-70B-shaped layers ({len(w['tensors'])} tensors, "
                      f"855,654,400 params each), D={D}, S={S} per layer, {L * S} owned params "
                      f"({L * S * 14 / 1e9:.1f} GB of master+m+v+bf16); per step the 80 layers' owned bf16 "
                      f"contributions ({2 * D * S / 1e9:.2f} GB each) stream 79->0 through two transient buffers "
-                     f"(device-to-device refill on a copy stream) while the fused kernel runs")
+                     f"({'device-to-device copy from a pool' if refill == 'copy' else 'write-only fill'} "
+                     f"on a copy stream) while the fused kernel runs")
 
     def hp(self):
         a = self.synth.ADAMW
@@ -422,7 +429,7 @@ class ShardRunner:
                              weight_decay=a["weight_decay"], step=self.step_no)
 
     def step(self, k1_events=None):
-        self.streamer.step(self.source, self.hp(), k1_events)
+        self.streamer.step(self.source, self.hp(), k1_events, fill=self.fill)
 
     def step_in_place(self, k1_events=None):
         """The same 80 fused-kernel launches reading the pool in place: no refill traffic."""
@@ -471,7 +478,7 @@ def run_ours(args):
         raise SystemExit("--graph covers the block step without --unflatten-copy")
     seed = 1000 + rank  # every rank runs its own block
     if args.workload == "llama70b_shard":
-        R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev)
+        R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev, refill=args.refill)
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
                         stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph)

@@ -13,9 +13,9 @@
 //     so the block scheduler balances the SMs; streaming stores.
 //   - per-tensor copy: the host cuts every tensor into segments, one per rank
 //     partition it intersects, and numbers the 16-byte units of each
-//     segment's destination.  A thread takes one destination unit, finds its
-//     segment by binary search, and writes it with one 16-byte store when the
-//     unit is whole; the source run may start at any 2-byte position, so it is
+//     segment's destination.  A thread takes two destination units, finds
+//     their segments by binary search, and writes each with one 16-byte store
+//     when the unit is whole; the source run may start at any 2-byte position, so it is
 //     assembled from the two aligned 16-byte source vectors around it with
 //     funnel shifts.  Partial units at a segment's ends are written element
 //     by element.
@@ -105,27 +105,50 @@ __device__ __forceinline__ uint4 load8_unaligned(const uint16_t* s) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// The segment holding destination unit u: the last one whose unit_begin <= u.
+__device__ __forceinline__ int find_segment(const SegArgs& a, int64_t u) {
+    int lo = 0, hi = a.nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.seg[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// kSegUnits destination units per thread (consecutive threads on consecutive
+// units); the whole units' source vectors are all loaded before any store, so
+// a thread keeps several 16-byte loads in flight.
+constexpr int kSegUnits = 2;
+
 __global__ void __launch_bounds__(kThreads) k_gather_segments(const __grid_constant__ SegArgs a) {
-    const int64_t stride = int64_t(gridDim.x) * kThreads;
-    for (int64_t u = int64_t(blockIdx.x) * kThreads + threadIdx.x; u < a.units; u += stride) {
-        // segment holding unit u: the last one whose unit_begin <= u
-        int lo = 0, hi = a.nseg - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (a.seg[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+    const int64_t span = int64_t(kThreads) * kSegUnits;
+    for (int64_t u0 = int64_t(blockIdx.x) * span + threadIdx.x; u0 < a.units; u0 += int64_t(gridDim.x) * span) {
+        uint4 q[kSegUnits];
+        uintptr_t dst[kSegUnits];
+        bool whole[kSegUnits];
+#pragma unroll
+        for (int k = 0; k < kSegUnits; ++k) {
+            const int64_t u = u0 + int64_t(k) * kThreads;
+            whole[k] = false;
+            if (u >= a.units) continue;
+            const Seg& s = a.seg[find_segment(a, u)];
+            const uintptr_t d0 = reinterpret_cast<uintptr_t>(s.dst);
+            const uintptr_t unit_addr = (d0 & ~uintptr_t(15)) + uintptr_t(u - s.unit_begin) * 16u;
+            // elements of this unit inside the segment: [k0, k1) relative to s.dst
+            const int64_t k_first = (int64_t(unit_addr) - int64_t(d0)) / 2;  // may be negative
+            if (a.vec && k_first >= 0 && k_first + 8 <= s.len) {
+                q[k] = load8_unaligned(s.src + k_first);
+                dst[k] = unit_addr;
+                whole[k] = true;
+            } else {
+                const int64_t k0 = k_first < 0 ? 0 : k_first;
+                const int64_t k1 = k_first + 8 < s.len ? k_first + 8 : s.len;
+                for (int64_t e = k0; e < k1; ++e) s.dst[e] = s.src[e];
+            }
         }
-        const Seg& s = a.seg[lo];
-        const uintptr_t d0 = reinterpret_cast<uintptr_t>(s.dst);
-        const uintptr_t unit_addr = (d0 & ~uintptr_t(15)) + uintptr_t(u - s.unit_begin) * 16u;
-        // elements of this unit inside the segment: [k0, k1) relative to s.dst
-        const int64_t k_first = (int64_t(unit_addr) - int64_t(d0)) / 2;  // may be negative
-        const int64_t k0 = k_first < 0 ? 0 : k_first;
-        const int64_t k1 = k_first + 8 < s.len ? k_first + 8 : s.len;
-        if (a.vec && k_first >= 0 && k_first + 8 <= s.len) {
-            *reinterpret_cast<uint4*>(unit_addr) = load8_unaligned(s.src + k_first);
-        } else {
-            for (int64_t k = k0; k < k1; ++k) s.dst[k] = s.src[k];
-        }
+#pragma unroll
+        for (int k = 0; k < kSegUnits; ++k)
+            if (whole[k]) __stcs(reinterpret_cast<uint4*>(dst[k]), q[k]);
     }
 }
 
@@ -237,7 +260,7 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
                 a.seg[k] = s;
             }
             a.units = units;
-            int64_t blocks = (units + kThreads - 1) / kThreads;
+            int64_t blocks = (units + int64_t(kThreads) * kSegUnits - 1) / (int64_t(kThreads) * kSegUnits);
             blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, kMaxBlocks));
             k_gather_segments<<<dim3(unsigned(blocks)), dim3(kThreads), 0, stream>>>(a);
             if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;

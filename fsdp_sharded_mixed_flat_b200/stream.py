@@ -55,8 +55,9 @@ class LayerStreamer:
         S = self.plan.S
         return [self.buf[b][d * S:(d + 1) * S] for d in range(self.plan.D)]
 
-    def step(self, source: Callable[[int], torch.Tensor], hp: "z3.AdamW",
-             k1_events: Optional[Sequence] = None, copy_in: bool = True) -> None:
+    def step(self, source: Optional[Callable[[int], torch.Tensor]], hp: "z3.AdamW",
+             k1_events: Optional[Sequence] = None, copy_in: bool = True,
+             fill: Optional[Callable[[int, torch.Tensor], None]] = None) -> None:
         """One optimiser step over every block, last to first.
 
         source(layer) gives the tensor to copy in for that block: D * S bf16, the D
@@ -64,7 +65,9 @@ class LayerStreamer:
         k1_events, if given, is a list of L (start, end) CUDA event pairs recorded
         around each fused-kernel launch on the compute stream.  With copy_in=False
         the kernel reads each block's contributions where source(layer) holds them
-        (a device tensor that stays valid for the step) and nothing is copied."""
+        (a device tensor that stays valid for the step) and nothing is copied.
+        With fill given, fill(layer, buffer) writes the block's contributions into
+        the transient buffer on the copy stream instead of a copy from source."""
         caller = torch.cuda.current_stream(self.device)
         self.copy.wait_stream(caller)
         self.compute.wait_stream(caller)
@@ -85,10 +88,13 @@ class LayerStreamer:
                 continue
             with torch.cuda.stream(self.copy):
                 self.copy.wait_event(self.free[b])          # the kernel two blocks back is done with it
-                src = source(layer)
-                self.buf[b].copy_(src, non_blocking=True)
-                if src.is_cuda:
-                    src.record_stream(self.copy)
+                if fill is not None:
+                    fill(layer, self.buf[b])
+                else:
+                    src = source(layer)
+                    self.buf[b].copy_(src, non_blocking=True)
+                    if src.is_cuda:
+                        src.record_stream(self.copy)
                 self.filled[b].record(self.copy)
             self.compute.wait_event(self.filled[b])
             p, m, v, w = self.layer_views(layer)

@@ -58,6 +58,33 @@ def test_streamed_layers_match_oracle(z3, mode, copy_in):
     assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
 
 
+def test_streamed_layers_with_a_fill_refill(z3):
+    """The fill hook writes each block's contributions into the transient buffer."""
+    from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
+    L, D, rank = 5, 4, 1
+    plan = z3.zero3_plan([(4000,)], D, 8)
+    S = plan.S
+    n_real = max(0, min(S, plan.N - rank * S))
+    master = synth.master_weights(L * S, L * S, seed=6, device="cuda")
+    m, v = torch.zeros_like(master), torch.zeros_like(master)
+    w = torch.zeros(L * S, dtype=torch.bfloat16, device="cuda")
+    st = LayerStreamer(plan, L, rank, master, m, v, w)
+    src = {l: owned_contribs(D, S, n_real, 4, 1, l) for l in range(L)}
+    hp_, hm, hv, hw = f32_host(master).copy(), np.zeros(L * S, np.float32), np.zeros(L * S, np.float32), \
+        np.zeros(L * S, np.uint16)
+    st.step(None, z3.adamw(**hp_for(1)), fill=lambda l, buf: buf.copy_(src[l]))
+    for l in range(L):
+        host = synth.bf16_bits(src[l])
+        sl = slice(l * S, (l + 1) * S)
+        p_l, m_l, v_l, w_l = hp_[sl].copy(), hm[sl].copy(), hv[sl].copy(), hw[sl].copy()
+        oracle.reduce_adamw([host[d * S:(d + 1) * S] for d in range(D)], S, rank, p_l, m_l, v_l, w_l,
+                            oracle_hp(1), layout=oracle.LAYOUT_OWNED)
+        hp_[sl], hm[sl], hv[sl], hw[sl] = p_l, m_l, v_l, w_l
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(master), hp_, "master")
+    assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
+
+
 def test_llama70b_rank_shard_80_layers_sampled(z3):
     """The full resident shard of one rank (8.556B owned params, about 120 GB with
     the bf16 shard), one streamed step over all 80 layers; the oracle checks a
