@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
+    ap.add_argument("--offload", action="store_true",
+                    help="fp32 master / m / v in page-locked host memory, reached by the kernel over PCIe")
     ap.add_argument("--refill", choices=["copy", "fill"], default="copy",
                     help="70B shard: each layer's contributions arrive by a device-to-device copy from a "
                          "pool (read + write) or by a write-only fill of the transient buffer")
@@ -238,10 +240,11 @@ class BlockRunner:
     the replicated bf16 weights (the flat block), with no separate shard."""
 
     def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
-                 graph=False):
+                 graph=False, offload=False):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
+        self.device = dev
         self.shapes = [s for _, s in w["tensors"]]
         self.specs = z3.tensor_specs(self.shapes)       # the step's input: the block's tensor list
         plan = z3.zero3_plan(self.shapes, D, synth.ALIGN)
@@ -250,7 +253,16 @@ class BlockRunner:
                                             dist=w["dist"], zero_frac=w.get("zero_frac", 0.0), device=dev)
         self.master = synth.master_weights(self.N, self.N_pad, seed=seed, device=dev)
         self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
+        self.offload = offload
         self.work = torch.zeros(self.N_pad, dtype=torch.bfloat16, device=dev)
+        self.offloaded = None
+        if offload:
+            # the optimiser state leaves the GPU: page-locked host memory, streamed through the GPU
+            from fsdp_sharded_mixed_flat_b200.offload import OffloadedState
+            self.master, self.exp_avg, self.exp_avg_sq = (t.cpu().pin_memory() for t in
+                                                          (self.master, self.exp_avg, self.exp_avg_sq))
+            self.offloaded = OffloadedState(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
+                                            reduce_dtype=reduce_dtype)
         self.flat = torch.empty(self.N_pad, dtype=torch.bfloat16, device=dev)
         self.shards = [self.work[r * self.S:(r + 1) * self.S] for r in range(D)]
         self.stream = torch.cuda.current_stream(dev)
@@ -280,6 +292,13 @@ class BlockRunner:
             # events around the replay time every kernel of the graph
             self.k1_bytes_per_launch = self.step_bytes
             self.k1_name = "CUDA graph of the step (%s)" % ("fused kernel + gather" if stage == 3 else "fused kernel")
+        if offload:
+            what += ("; fp32 master/m/v in page-locked host memory, streamed partition by partition through "
+                     "device staging buffers (copy-in, kernel, copy-out on three streams)")
+            self.k1_name += " (rank-partition launches on staged state)"
+            self.k1_launches_per_step = D
+            self.k1_bytes_per_launch = (2 * D + 26) * self.S
+            self.launches_per_step = D + 1
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
                      f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
                      f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + {what}")
@@ -307,6 +326,10 @@ class BlockRunner:
             return self.views(pl, flat)
         if k1_events is not None:
             k1_events[0][0].record(self.stream)
+        if self.offloaded is not None:
+            self.offloaded.step(contribs, hp, k1_events)
+            z3.zero3_gather_block(pl, self.shards, flat, self.tensor_out, stream=self.stream)
+            return self.views(pl, flat)
         if self.stage != 3:
             # ZeRO-1/2: the kernel writes each new bf16 weight into the replicated block
             z3.zero3_reduce_adamw_gather(pl, -1, contribs, self.master, self.exp_avg, self.exp_avg_sq, None,
@@ -336,7 +359,7 @@ class BlockRunner:
         """Pinned host copies of the contributions and of the gathered block, and a
         second device set of both so that transfers of neighbouring steps overlap."""
         import torch
-        dev = self.master.device
+        dev = self.device
         self.host_c = [torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in range(self.D)]
         for h, c in zip(self.host_c, self.contribs):
             h.copy_(c)
@@ -476,12 +499,15 @@ def run_ours(args):
     mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
     if args.graph and (args.unflatten_copy or args.workload == "llama70b_shard"):
         raise SystemExit("--graph covers the block step without --unflatten-copy")
+    if args.offload and (args.graph or args.stage != 3 or args.workload == "llama70b_shard"):
+        raise SystemExit("--offload covers the ZeRO-3 block step without --graph")
     seed = 1000 + rank  # every rank runs its own block
     if args.workload == "llama70b_shard":
         R = ShardRunner(z3, synth, args.workload, args.D or 8, mode, seed, dev, refill=args.refill)
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
-                        stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph)
+                        stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph,
+                        offload=args.offload)
     stream = R.stream
 
     for _ in range(args.warmup):
@@ -579,6 +605,14 @@ def run_ours(args):
         "gpu_launches": R.launches_per_step * args.steps,
     }
     line.update(extra)
+    if getattr(R, "offload", False):
+        # 12 B of state read and 12 B written per element cross PCIe; HBM carries the rest
+        step_s = job_secs / args.steps
+        line["offload"] = {"pcie_gbs_per_direction": 12 * R.N_pad / step_s / 1e9,
+                           "note": "fp32 master/m/v (12 B per element) cross PCIe each way every step; the step "
+                                   "is bound by PCIe, not HBM, so the hbm roofline fields describe the kernels "
+                                   "on the staged device buffers only"}
+        line["roofline"]["traffic"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, secs_cpu, desc = oracle_sample(args.workload, args.cpu_sample, args.cpu_steps, D=R.D, reduce_dtype=mode)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,

@@ -199,11 +199,14 @@ def adamw(lr=3e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1, step=1) ->
     return AdamW(lr, beta1, beta2, eps, weight_decay, step)
 
 
-def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str) -> int:
+def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str, host_ok: bool = False) -> int:
+    """The address of a contiguous tensor the kernels may access: a CUDA tensor, or
+    with host_ok a page-locked host tensor (mapped into the device's address space,
+    so the kernel reaches it over PCIe)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
-        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.type != "cuda" and not (host_ok and t.device.type == "cpu" and t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor" + (" or a pinned host tensor" if host_ok else ""))
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
@@ -233,11 +236,11 @@ def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], m
     ptrs = (C.c_void_p * plan.D)()
     for d, c in enumerate(contrib):
         ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
-    mp = _dev_tensor(master, torch.float32, n, "master")
-    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
-    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
-    wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
-    dev = master.device
+    mp = _dev_tensor(master, torch.float32, n, "master", host_ok=True)
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
+    wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
+    dev = contrib[0].device
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                      reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
@@ -263,11 +266,11 @@ def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Ten
     gp = (C.c_void_p * len(gathered))()
     for k, g in enumerate(gathered):
         gp[k] = _dev_tensor(g, torch.bfloat16, plan.N_pad, f"gathered[{k}]")
-    mp = _dev_tensor(master, torch.float32, n, "master")
-    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
-    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
-    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
-    dev = master.device
+    mp = _dev_tensor(master, torch.float32, n, "master", host_ok=True)
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
+    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
+    dev = contrib[0].device
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw_gather(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp, gp,
                                             len(gathered), reduce_dtype, C.byref(hp),
@@ -308,11 +311,11 @@ def zero3_reduce_adamw_dev(plan: Plan, rank: int, contrib: Sequence[torch.Tensor
     for k, g in enumerate(gathered):
         gp[k] = _dev_tensor(g, torch.bfloat16, plan.N_pad, f"gathered[{k}]")
     sp = _dev_tensor(scalars, torch.float32, Z3_SCALARS, "scalars")
-    mp = _dev_tensor(master, torch.float32, n, "master")
-    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg")
-    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
-    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
-    dev = master.device
+    mp = _dev_tensor(master, torch.float32, n, "master", host_ok=True)
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
+    wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
+    dev = contrib[0].device
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw_dev(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                          gp if gathered else None, len(gathered), reduce_dtype, sp,

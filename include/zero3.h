@@ -177,9 +177,12 @@ Z3_API int zero3_transient_bytes(int64_t block_params, int32_t n_buffers, int64_
  *          launch (state arrays then hold all D partitions back to back).
  *   contrib host array of D device pointers, the ranks' bf16 gradient
  *          contributions in `contrib_layout` (Z3_CONTRIB_OWNED needs rank >= 0).
- *   master, exp_avg, exp_avg_sq  device fp32, S elements (N_pad if rank = -1),
- *          read and updated in place.
- *   work_bf16 device bf16 output, same extent as master.
+ *   master, exp_avg, exp_avg_sq  fp32, S elements (N_pad if rank = -1), read
+ *          and updated in place.  In device memory, or in page-locked host
+ *          memory mapped into the device's address space (the CPU-offload
+ *          placement of [P2] §8: the optimiser state leaves the GPU, which
+ *          then reads and writes it over PCIe; the arithmetic is unchanged).
+ *   work_bf16 bf16 output, same extent as master; device or mapped host memory.
  *   reduce_dtype  Z3_REDUCE_FP32 or Z3_REDUCE_BF16.
  *   hp     host struct; hp->step >= 1, all values finite.
  *   cuda_stream  stream to enqueue on.

@@ -212,6 +212,76 @@ def test_fused_gather_misaligned_scalar_path(z3):
     run_fused(z3, [3000, 17], 4, 8, 2, z3.Z3_CONTRIB_OWNED, 1, 1, with_work=False, skew=1)
 
 
+# ------------------------------------------------ offloaded optimiser state
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("numels,D,A,rank", [([300, 77, 1000], 4, 8, -1), ([123457], 8, 128, -1),
+                                             ([4097, 33], 32, 128, 7), ([999], 5, 1, 2)])
+def test_offloaded_state_matches_oracle(z3, numels, D, A, rank, mode):
+    """fp32 master / m / v in page-locked host memory, read and written by the kernel
+    over PCIe (the CPU-offload placement): same results as in HBM."""
+    plan = z3.zero3_plan([(k,) for k in numels], D, A)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    n = N_pad if rank < 0 else S
+    p_full, _, _ = state_init(N, N_pad, 8)
+    p0 = (p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]).cpu()
+    p, m, v = p0.clone().pin_memory(), torch.zeros(n).pin_memory(), torch.zeros(n).pin_memory()
+    w = torch.zeros(n, dtype=torch.bfloat16).pin_memory()
+    g = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    hp_, hm, hv, hw = p0.numpy().copy(), np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
+    for t in range(1, 4):
+        c = synth.contributions(D, N, N_pad, seed=8, step=t, sigma=1e-3, device="cuda")
+        if t == 3:
+            z3.zero3_reduce_adamw_gather(plan, rank, c, p, m, v, w, [g], z3.adamw(**hp_for(t)), reduce_dtype=mode)
+        else:
+            z3.zero3_reduce_adamw(plan, rank, c, p, m, v, w, z3.adamw(**hp_for(t)), reduce_dtype=mode)
+        oracle.reduce_adamw([synth.bf16_bits(x) for x in c], S, rank, hp_, hm, hv, hw, oracle_hp(t),
+                            reduce_dtype=mode)
+    torch.cuda.synchronize()
+    assert_f32_parity(p.numpy(), hp_, "master")
+    assert_f32_parity(m.numpy(), hm, "exp_avg")
+    assert_f32_parity(v.numpy(), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
+    lo = 0 if rank < 0 else rank * S
+    assert_bf16_parity(synth.bf16_bits(g)[lo:lo + n], hw, "gathered")
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+@pytest.mark.parametrize("numels,D,A,n_stage", [([300, 77, 1000], 4, 8, 3), ([123457], 8, 128, 2),
+                                                ([4097, 33], 32, 128, 3), ([999], 5, 1, 1)])
+def test_staged_offload_matches_oracle(z3, numels, D, A, n_stage, mode):
+    """The optimiser state in pinned host memory, streamed partition by partition
+    through device staging buffers: same results as the whole-block kernel."""
+    from fsdp_sharded_mixed_flat_b200.offload import OffloadedState
+    plan = z3.zero3_plan([(k,) for k in numels], D, A)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    p_full, _, _ = state_init(N, N_pad, 9)
+    p = p_full.cpu().pin_memory()
+    m, v = torch.zeros(N_pad).pin_memory(), torch.zeros(N_pad).pin_memory()
+    w = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    off = OffloadedState(plan, p, m, v, w, "cuda", n_stage=n_stage, reduce_dtype=mode)
+    hp_, hm, hv, hw = p_full.cpu().numpy().copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
+        np.zeros(N_pad, np.uint16)
+    for t in range(1, 5):
+        c = synth.contributions(D, N, N_pad, seed=9, step=t, sigma=1e-3, device="cuda")
+        off.step(c, z3.adamw(**hp_for(t)))
+        oracle.reduce_adamw([synth.bf16_bits(x) for x in c], S, -1, hp_, hm, hv, hw, oracle_hp(t),
+                            reduce_dtype=mode)
+    torch.cuda.synchronize()
+    assert_f32_parity(p.numpy(), hp_, "master")
+    assert_f32_parity(m.numpy(), hm, "exp_avg")
+    assert_f32_parity(v.numpy(), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
+
+
+def test_unpinned_host_state_is_refused(z3):
+    plan = z3.zero3_plan([(64,)], 2, 8)
+    c = [torch.zeros(plan.N_pad, dtype=torch.bfloat16, device="cuda")] * 2
+    host = torch.zeros(plan.N_pad)                   # pageable: the device cannot reach it
+    with pytest.raises(ValueError):
+        z3.zero3_reduce_adamw(plan, -1, c, host, host.clone(), host.clone(),
+                              torch.zeros(plan.N_pad, dtype=torch.bfloat16, device="cuda"), z3.adamw(step=1))
+
+
 # ------------------------------------------------------------- full sizes
 def sample_indices(n: int, S: int, D: int, k: int, seed: int) -> torch.Tensor:
     rng = np.random.default_rng(seed)
