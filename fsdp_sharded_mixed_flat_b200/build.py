@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libzero3.so")
 
-SOURCES = ["plan.cpp", "reduce_adamw.cu", "gather.cu"]
+SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "gather.cu"]
 EXPORTS = os.path.join(CSRC, "exports.map")
 HEADERS = [os.path.join(CSRC, "plan_impl.h"), os.path.join(INCLUDE, "zero3.h"), EXPORTS]
 

@@ -154,21 +154,6 @@ __global__ void __launch_bounds__(kThreads) k_gather_segments(const __grid_const
 
 }  // namespace
 
-namespace z3 {
-
-int sm_count() {
-    static int cached[Z3_D_MAX * 2] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-    if (dev >= 0 && dev < Z3_D_MAX * 2 && cached[dev] > 0) return cached[dev];
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    if (dev >= 0 && dev < Z3_D_MAX * 2) cached[dev] = n;
-    return n;
-}
-
-}  // namespace z3
-
 extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
                                          uint16_t* const* tensor_out, void* cuda_stream) {
     if (p == nullptr || shards == nullptr || (flat_out == nullptr && tensor_out == nullptr)) return Z3_EINVAL;
