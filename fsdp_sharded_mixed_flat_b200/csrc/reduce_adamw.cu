@@ -22,16 +22,18 @@
 // leaves the SMs that finish first idle, while the block scheduler keeps
 // every SM fed until the end.  Stores carry the streaming cache hint: every
 // byte is written exactly once.  Asking for three resident blocks per SM caps
-// the registers at 85 (left alone the compiler takes up to 128 at D >= 16 and
-// spills at D = 4 and 8 in bf16 mode); measured on B200 this never loses and
-// gains up to 12 % (bf16 reduce at D = 16).
+// the registers at 80 (65,536 / (3 x 256), rounded down to the allocation
+// granularity; left alone the compiler takes up to 128 at D >= 16); measured
+// on B200 this never loses and gains up to 12 % (bf16 reduce at D = 16).
+//
+// Every arithmetic step is an explicitly rounded fp32 intrinsic, so nothing is
+// contracted into an FMA and the results are fixed by the stated operation
+// order.
 //
 // Measured ceilings of HBM on the B200s used here, for a full-grid kernel with
 // two or more independent 16-byte vectors per thread: read-only 7.54 TB/s,
 // write-only 7.56 TB/s, copy 6.94 TB/s, two reads per write 7.16 TB/s.  This
-// pass reads 28 B and writes 14 B per element at D = 8, the two-to-one mix.  Every arithmetic step is an explicitly
-// rounded fp32 intrinsic so that nothing is contracted into an FMA and the
-// results are fixed by the stated operation order.
+// pass reads 28 B and writes 14 B per element at D = 8, the two-to-one mix.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -88,7 +90,7 @@ AdamScalars step_scalars(const z3_adamw* hp) {
 }
 
 constexpr int kThreads = 256;
-constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: caps registers at 85 per thread
+constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: at most 80 registers per thread
 constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
 
