@@ -381,3 +381,42 @@ def test_tiny_gpt_full_ten_steps_then_gather(z3):
     for o, r, view in zip(outs, ref_t, plan.views(flat)):
         assert np.array_equal(synth.bf16_bits(o).ravel(), r)
         assert np.array_equal(synth.bf16_bits(view).ravel(), r)
+
+
+def test_single_launch_beyond_2_31_elements(z3):
+    """One launch over more than 2^31 elements (no 32-bit index anywhere): the fused
+    kernel and the flat gather, sampled around 2^31 and at the end."""
+    D = 2
+    N = 2 ** 31 + 777
+    torch.cuda.empty_cache()
+    free, _ = torch.cuda.mem_get_info()
+    if free < 48e9:
+        pytest.skip("needs about 45 GB of free device memory")
+    plan = z3.zero3_plan([(N,)], D, synth.ALIGN)
+    N_pad, S = plan.N_pad, plan.S
+    p = synth.master_weights(N, N_pad, seed=21, device="cuda")
+    m, v = torch.zeros_like(p), torch.zeros_like(p)
+    w = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    c = synth.contributions(D, N, N_pad, seed=21, step=1, sigma=1e-3, device="cuda")
+    rng = np.random.default_rng(21)
+    idx = np.unique(np.concatenate([rng.choice(N_pad, 50_000, replace=False),
+                                    np.arange(2 ** 31 - 64, 2 ** 31 + 64), np.arange(S - 64, S + 64),
+                                    np.arange(N - 64, N_pad)]))
+    ti = torch.from_numpy(idx).cuda()
+    hp_ = f32_host(p[ti]).copy()
+    hm, hv, hw = np.zeros(idx.size, np.float32), np.zeros(idx.size, np.float32), np.zeros(idx.size, np.uint16)
+    z3.zero3_reduce_adamw(plan, -1, c, p, m, v, w, z3.adamw(**hp_for(1)))
+    oracle.reduce_adamw([synth.bf16_bits(x[ti]) for x in c], idx.size, 0, hp_, hm, hv, hw, oracle_hp(1),
+                        layout=oracle.LAYOUT_OWNED)
+    del c
+    flat = torch.empty(N_pad, dtype=torch.bfloat16, device="cuda")
+    z3.zero3_gather_block(plan, [w[r * S:(r + 1) * S] for r in range(D)], flat)
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(p[ti]), hp_, "master")
+    assert_f32_parity(f32_host(m[ti]), hm, "exp_avg")
+    assert_f32_parity(f32_host(v[ti]), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(w[ti]), hw, "work_bf16")
+    assert np.array_equal(synth.bf16_bits(flat[ti]), hw)
+    assert not p[N:].any() and not w[N:].view(torch.int16).any()
+    del p, m, v, w, flat
+    torch.cuda.empty_cache()
