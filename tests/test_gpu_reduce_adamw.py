@@ -347,6 +347,34 @@ def test_llama7b_policy_sweep_bf16_reduce(z3, D):
     run_sampled(z3, "llama7b_policy", D, -1, z3.Z3_CONTRIB_FULL, 1, steps=3, k=100_000)
 
 
+@pytest.mark.parametrize("D", [2, 4, 8, 16])
+def test_policy_sweep_hundred_steps_every_element(z3, D):
+    """The policy sweep's 100 steps (Student-t nu=3 gradients, 1% exact zeros, fresh
+    every step) on a 2^20-element slice of the 7B block, both reduce dtypes, every
+    element compared after the last step."""
+    w = synth.WORKLOADS["llama7b_policy"]
+    n_real = 1 << 20
+    plan = z3.zero3_plan([(n_real,)], D, synth.ALIGN)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    for mode in (0, 1):
+        p, m, v = state_init(N, N_pad, 31)
+        wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+        hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
+            np.zeros(N_pad, np.uint16)
+        for t in range(1, w["steps"] + 1):
+            c = synth.contributions(D, N, N_pad, seed=31, step=t, sigma=w["sigma"], dist=w["dist"],
+                                    zero_frac=w["zero_frac"], device="cuda")
+            z3.zero3_reduce_adamw(plan, -1, c, p, m, v, wk, z3.adamw(**hp_for(t)), reduce_dtype=mode)
+            oracle.reduce_adamw([synth.bf16_bits(x) for x in c], S, -1, hp_, hm, hv, hw, oracle_hp(t),
+                                reduce_dtype=mode)
+        torch.cuda.synchronize()
+        what = f"100 steps D={D} mode={mode}"
+        assert_f32_parity(f32_host(p), hp_, "master " + what)
+        assert_f32_parity(f32_host(m), hm, "exp_avg " + what)
+        assert_f32_parity(f32_host(v), hv, "exp_avg_sq " + what)
+        assert_bf16_parity(synth.bf16_bits(wk), hw, "work_bf16 " + what)
+
+
 def test_llama70b_layer_owned_rank(z3):
     """One 70B layer's owned shard of rank 3 at D = 8, contributions in the owned layout."""
     run_sampled(z3, "llama70b_layer", 8, 3, z3.Z3_CONTRIB_OWNED, 0, steps=2, k=100_000)
