@@ -32,38 +32,56 @@ def lib():
     """Load (building first if needed) the oracle's shared library."""
     global _lib
     if _lib is None:
-        path = _build.build()
-        L = C.CDLL(path)
-        p = C.c_void_p
-        i64, i32 = C.c_int64, C.c_int32
-        L.ref_bf16_from_f32.argtypes = [C.c_float]
-        L.ref_bf16_from_f32.restype = C.c_uint16
-        L.ref_f32_from_bf16.argtypes = [C.c_uint16]
-        L.ref_f32_from_bf16.restype = C.c_float
-        L.ref_bf16_from_f32_array.argtypes = [p, i64, p]
-        L.ref_bf16_from_f32_array.restype = None
-        L.ref_plan.argtypes = [i32, p, i32, i32, p, p, p, p]
-        L.ref_plan.restype = C.c_int
-        L.ref_rank_range.argtypes = [i64, i64, i32, p, p]
-        L.ref_rank_range.restype = None
-        L.ref_memory_bytes.argtypes = [C.c_double, C.c_double, i32]
-        L.ref_memory_bytes.restype = C.c_double
-        L.ref_transient_bytes.argtypes = [C.c_double, i32]
-        L.ref_transient_bytes.restype = C.c_double
-        L.ref_reduce_scatter.argtypes = [i32, i64, i32, p, i32, i32, p]
-        L.ref_reduce_scatter.restype = C.c_int
-        L.ref_adamw_consts_of.argtypes = [C.POINTER(AdamWHP), p]
-        L.ref_adamw_consts_of.restype = None
-        L.ref_adamw.argtypes = [i64, p, p, p, p, C.POINTER(AdamWHP)]
-        L.ref_adamw.restype = C.c_int
-        L.ref_reduce_adamw.argtypes = [i32, i64, i32, p, i32, p, p, p, p, i32, C.POINTER(AdamWHP)]
-        L.ref_reduce_adamw.restype = C.c_int
-        L.ref_all_gather.argtypes = [i32, i64, p, p]
-        L.ref_all_gather.restype = None
-        L.ref_unflatten.argtypes = [p, i32, p, p, p]
-        L.ref_unflatten.restype = None
-        _lib = L
+        _lib = _bind(C.CDLL(_build.build()))
     return _lib
+
+
+def use_library(path):
+    """Swap in another build of the oracle's C source (the mutation tests plant a
+    mistake in a copy of the source, build it, and check that the pins fail).
+    Returns the library that was in use, for restoring."""
+    global _lib
+    previous = _lib
+    _lib = None if path is None else _bind(C.CDLL(path))
+    return previous
+
+
+def restore_library(previous):
+    global _lib
+    _lib = previous
+
+
+def _bind(L):
+    """Declare the C signatures on a loaded oracle library."""
+    p = C.c_void_p
+    i64, i32 = C.c_int64, C.c_int32
+    L.ref_bf16_from_f32.argtypes = [C.c_float]
+    L.ref_bf16_from_f32.restype = C.c_uint16
+    L.ref_f32_from_bf16.argtypes = [C.c_uint16]
+    L.ref_f32_from_bf16.restype = C.c_float
+    L.ref_bf16_from_f32_array.argtypes = [p, i64, p]
+    L.ref_bf16_from_f32_array.restype = None
+    L.ref_plan.argtypes = [i32, p, i32, i32, p, p, p, p]
+    L.ref_plan.restype = C.c_int
+    L.ref_rank_range.argtypes = [i64, i64, i32, p, p]
+    L.ref_rank_range.restype = None
+    L.ref_memory_bytes.argtypes = [C.c_double, C.c_double, i32]
+    L.ref_memory_bytes.restype = C.c_double
+    L.ref_transient_bytes.argtypes = [C.c_double, i32]
+    L.ref_transient_bytes.restype = C.c_double
+    L.ref_reduce_scatter.argtypes = [i32, i64, i32, p, i32, i32, p]
+    L.ref_reduce_scatter.restype = C.c_int
+    L.ref_adamw_consts_of.argtypes = [C.POINTER(AdamWHP), p]
+    L.ref_adamw_consts_of.restype = None
+    L.ref_adamw.argtypes = [i64, p, p, p, p, C.POINTER(AdamWHP)]
+    L.ref_adamw.restype = C.c_int
+    L.ref_reduce_adamw.argtypes = [i32, i64, i32, p, i32, p, p, p, p, i32, C.POINTER(AdamWHP)]
+    L.ref_reduce_adamw.restype = C.c_int
+    L.ref_all_gather.argtypes = [i32, i64, p, p]
+    L.ref_all_gather.restype = None
+    L.ref_unflatten.argtypes = [p, i32, p, p, p]
+    L.ref_unflatten.restype = None
+    return L
 
 
 def _ptr(a: np.ndarray):
