@@ -51,7 +51,7 @@ class GraphedStep:
                 z3.zero3_reduce_adamw_dev(plan, -1, contribs, master, exp_avg, exp_avg_sq, work_bf16, [flat],
                                           self.scalars, reduce_dtype=reduce_dtype, stream=stream)
 
-        self._warm_up(plan, stage, reduce_dtype, contribs[0].data_ptr() % 16 == 0)
+        self._warm_up(plan, stage, reduce_dtype)
         side = torch.cuda.Stream(dev)
         side.wait_stream(torch.cuda.current_stream(dev))
         self.graph = torch.cuda.CUDAGraph()
@@ -59,24 +59,28 @@ class GraphedStep:
             launches(side)
         torch.cuda.current_stream(dev).wait_stream(side)
 
-    def _warm_up(self, plan, stage, reduce_dtype, aligned):
-        """Run the same kernels once on a small scratch block so that every kernel the
-        graph captures is loaded before capture; the real state is not touched."""
+    def _warm_up(self, plan, stage, reduce_dtype):
+        """Run the same kernels once on a small scratch block, through both the
+        16-byte vector path and the scalar path (buffers one element off), so that
+        whichever kernel the graph captures is loaded before capture; the real
+        state is not touched."""
         dev = self.device
         D = plan.D
         tiny = z3.zero3_plan([(D * plan.align_elems,)], D, plan.align_elems)
         n = tiny.N_pad
-        c = [torch.zeros(n, dtype=torch.bfloat16, device=dev) for _ in range(D)]
-        p, m, v = (torch.zeros(n, dtype=torch.float32, device=dev) for _ in range(3))
-        w = torch.zeros(n, dtype=torch.bfloat16, device=dev)
-        f = torch.zeros(n, dtype=torch.bfloat16, device=dev)
         sc = torch.zeros(z3.Z3_SCALARS, dtype=torch.float32, device=dev)
         sc.copy_(torch.tensor(z3.zero3_step_scalars(z3.adamw(step=1)), dtype=torch.float32))
-        if stage == 3:
-            z3.zero3_reduce_adamw_dev(tiny, -1, c, p, m, v, w, [], sc, reduce_dtype=reduce_dtype)
-            z3.zero3_gather_block(tiny, [w[r * tiny.S:(r + 1) * tiny.S] for r in range(D)], f, None)
-        else:
-            z3.zero3_reduce_adamw_dev(tiny, -1, c, p, m, v, None, [f], sc, reduce_dtype=reduce_dtype)
+        for skew in (0, 1):
+            def buf(dtype):
+                return torch.zeros(n + skew, dtype=dtype, device=dev)[skew:]
+            c = [buf(torch.bfloat16) for _ in range(D)]
+            p, m, v = buf(torch.float32), buf(torch.float32), buf(torch.float32)
+            w, f = buf(torch.bfloat16), buf(torch.bfloat16)
+            if stage == 3:
+                z3.zero3_reduce_adamw_dev(tiny, -1, c, p, m, v, w, [], sc, reduce_dtype=reduce_dtype)
+                z3.zero3_gather_block(tiny, [w[r * tiny.S:(r + 1) * tiny.S] for r in range(D)], f, None)
+            else:
+                z3.zero3_reduce_adamw_dev(tiny, -1, c, p, m, v, None, [f], sc, reduce_dtype=reduce_dtype)
         torch.cuda.synchronize(dev)
 
     def step(self, hp: "z3.AdamW") -> None:
