@@ -216,6 +216,16 @@ def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str, host_
     return t.data_ptr()
 
 
+def _launch_device(*candidates):
+    """The device the kernels launch on: that of the first local CUDA tensor given
+    (the state and outputs come first; contributions and shards may be mapped
+    from peer GPUs)."""
+    for t in candidates:
+        if isinstance(t, torch.Tensor) and t.device.type == "cuda":
+            return t.device
+    raise ValueError("no CUDA tensor among the arguments")
+
+
 def _stream_handle(stream, device) -> int:
     if stream is None:
         return torch.cuda.current_stream(device).cuda_stream
@@ -240,7 +250,7 @@ def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], m
     ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
-    dev = contrib[0].device
+    dev = _launch_device(work_bf16, master, *contrib)
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                      reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
@@ -270,7 +280,7 @@ def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Ten
     ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
-    dev = contrib[0].device
+    dev = _launch_device(work_bf16, master, *contrib)
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw_gather(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp, gp,
                                             len(gathered), reduce_dtype, C.byref(hp),
@@ -315,7 +325,7 @@ def zero3_reduce_adamw_dev(plan: Plan, rank: int, contrib: Sequence[torch.Tensor
     ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
-    dev = contrib[0].device
+    dev = _launch_device(scalars, work_bf16, master, *contrib)
     with torch.cuda.device(dev):
         rc = _lib.zero3_reduce_adamw_dev(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                          gp if gathered else None, len(gathered), reduce_dtype, sp,
@@ -339,7 +349,7 @@ def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Opt
         tp = (C.c_void_p * max(1, plan.n_tensors))()
         for i, t in enumerate(tensor_out):
             tp[i] = None if t is None else _dev_tensor(t, torch.bfloat16, plan.numels[i], f"tensor_out[{i}]")
-    dev = shards[0].device
+    dev = _launch_device(flat_out, *(tensor_out or []), *shards)
     with torch.cuda.device(dev):
         rc = _lib.zero3_gather_block(plan.handle, sp, fp, tp, _stream_handle(stream, dev))
     _check(rc, "zero3_gather_block")
