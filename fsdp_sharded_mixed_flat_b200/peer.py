@@ -57,6 +57,8 @@ class PeerGroup:
     def share(self, t: torch.Tensor) -> List[torch.Tensor]:
         """Every rank's tensor `t`, in rank order: this rank's own, the others
         opened through their IPC handles (mapped into this process)."""
+        if self.size == 1:
+            return [t]                              # nobody to share with
         handles = [None] * self.size
         dist.all_gather_object(handles, self._share(t), group=self.group)
         return [t if k == self.rank else self._open(h) for k, h in enumerate(handles)]

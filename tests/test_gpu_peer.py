@@ -1,5 +1,5 @@
-"""The D-GPU step's code path on one GPU: a one-rank group (D = 1), real CUDA IPC
-export of the buffers and the real kernels, compared with the oracle.  (Groups
+"""The D-GPU step's code path on one GPU: a one-rank group (D = 1), its fences and
+the real kernels, compared with the oracle.  (Groups
 of several GPUs cannot run here: every run has one GPU; their host-side logic is
 tested with gloo ranks in test_peer_host.py.)"""
 import os
