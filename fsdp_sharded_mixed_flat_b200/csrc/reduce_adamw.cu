@@ -411,6 +411,9 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
             if (z3::overlaps(outs[x], out_bytes[x], outs[y], out_bytes[y])) return Z3_EINVAL;
         for (int32_t d = 0; d < D; ++d)
             if (z3::overlaps(outs[x], out_bytes[x], contrib[d] + c_off, hb)) return Z3_EINVAL;
+        if (dev_scalars != nullptr &&
+            z3::overlaps(outs[x], out_bytes[x], dev_scalars, Z3_SCALARS * int64_t(sizeof(float))))
+            return Z3_EINVAL;
     }
     if (n == 0) return Z3_OK;
 

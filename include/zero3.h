@@ -248,8 +248,8 @@ Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint1
  * only the scalars rewritten (stream-ordered) before each replay.  The
  * arithmetic and results are those of zero3_reduce_adamw.  work_bf16 may be
  * NULL only when n_gathered >= 1.
- * Errors: those of zero3_reduce_adamw_gather, Z3_EINVAL (scalars NULL),
- * Z3_EALIGN (scalars not 16-byte aligned). */
+ * Errors: those of zero3_reduce_adamw_gather, Z3_EINVAL (scalars NULL, or
+ * overlapping an output), Z3_EALIGN (scalars not 16-byte aligned). */
 Z3_API int zero3_step_scalars(const z3_adamw* hp, float* out);
 Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
                                   int32_t contrib_layout, float* master, float* exp_avg, float* exp_avg_sq,

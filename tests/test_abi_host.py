@@ -249,6 +249,7 @@ def test_reduce_adamw_dev_argument_errors():
     assert call(P16 * 9000, work=None) == z3.Z3_EINVAL          # no shard and no gathered block
     assert call(P16 * 9000, gathered=[P16 * 5000] * 9) == z3.Z3_EINVAL
     assert call(P16 * 9000, rank=7) == z3.Z3_EINVAL
+    assert call(P16 * 2 + 16) == z3.Z3_EINVAL                   # the scalars inside exp_avg
     e = z3.zero3_plan([], 4, 8)
     assert L.zero3_reduce_adamw_dev(e.handle, -1, arr, 0, C.c_void_p(P16), C.c_void_p(P16 * 2),
                                     C.c_void_p(P16 * 3), C.c_void_p(P16 * 4), None, 0, 0,
