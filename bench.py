@@ -5,7 +5,8 @@ the flat block (with zero-copy per-tensor views) and the host-side plan and
 memory ledger.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--e2e-steps E]
+                    [--workload NAME] [--D D] [--reduce-dtype fp32|bf16] [--stage 1|2|3]
+                    [--graph] [--offload] [--unflatten-copy] [--refill copy|fill] [--drift]
 
 One process per GPU (torchrun for N > 1).  Each rank runs its own block
 (independent replicas: the path needs no inter-GPU exchange), so the work per
@@ -154,6 +155,7 @@ class ClockSampler:
         loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
         return {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "slowdown_seen": any(r in SLOW_REASONS for r in reasons),
                 "samples": len(sm), "samples_under_load": len(loaded),
                 "power_w_max": max(power) if power else None}
 
@@ -183,7 +185,6 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
     workload's owned elements (all D contributions, AdamW, cast).  Returns
     (owned params/s, seconds, description)."""
     import numpy as np
-    import torch
 
     import oracle
     import synth
@@ -203,7 +204,6 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
         oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED,
                             reduce_dtype=reduce_dtype)
     dt = time.perf_counter() - t0
-    del torch
     desc = (f"{workload}: first {n} owned elements x {steps} steps, D={D}, "
             f"{'bf16' if reduce_dtype else 'fp32'} reduce, one thread "
             f"(oracle/zero3_ref.c, single-threaded C)")

@@ -56,6 +56,7 @@ def test_clock_sampler_parses_reasons():
     r = c.stop()
     assert r["sm_mhz"] == pytest.approx(1882.5) and r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"] and r["samples"] == 3 and r["samples_under_load"] == 2
+    assert r["slowdown_seen"] is False
 
 
 def test_reference_arm_prints_one_contract_line():
