@@ -16,9 +16,10 @@
 // no contraction, so no tensor-core work.  Each thread owns 8 consecutive
 // elements: one 16-byte load per rank, two per state array, all issued before
 // the arithmetic so that (D + 6) x 16 bytes per thread are in flight; the
-// ranks are folded in order 0..D-1 in chunks of 8 to bound registers at large
-// D.  The grid covers the whole range rather than looping over a resident
-// grid: HBM bandwidth does not divide evenly over the SMs, and a resident grid
+// ranks are folded in order 0..D-1 in chunks (8 ranks, 16 for the bf16 fold at
+// D = 32) to bound registers at large D.  The grid covers the whole range
+// rather than looping over a resident grid: HBM bandwidth does not divide
+// evenly over the SMs, and a resident grid
 // leaves the SMs that finish first idle, while the block scheduler keeps
 // every SM fed until the end.  Stores carry the streaming cache hint: every
 // byte is written exactly once.  Asking for three resident blocks per SM caps
