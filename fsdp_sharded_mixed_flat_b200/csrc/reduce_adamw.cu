@@ -19,9 +19,8 @@
 // ranks are folded in order 0..D-1 in chunks (8 ranks, 16 for the bf16 fold at
 // D = 32) to bound registers at large D.  The grid covers the whole range
 // rather than looping over a resident grid: HBM bandwidth does not divide
-// evenly over the SMs, and a resident grid
-// leaves the SMs that finish first idle, while the block scheduler keeps
-// every SM fed until the end.  Stores carry the streaming cache hint: every
+// evenly over the SMs, and a resident grid leaves the SMs that finish first
+// idle, while the block scheduler keeps every SM fed until the end.  Stores carry the streaming cache hint: every
 // byte is written exactly once.  Asking for three resident blocks per SM caps
 // the registers at 80 (65,536 / (3 x 256), rounded down to the allocation
 // granularity; left alone the compiler takes up to 128 at D >= 16); measured
