@@ -26,7 +26,7 @@ memory: only libzero3.so's own kernels touch the mappings.
 """
 from __future__ import annotations
 
-from typing import Callable, List, Optional, Sequence
+from typing import Callable, List, Optional
 
 import torch
 import torch.distributed as dist

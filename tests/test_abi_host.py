@@ -4,7 +4,6 @@ agree with the oracle, and every argument error is reported before any device
 work.  No call here reaches a CUDA API: each one either fails validation or
 has nothing to do (an empty plan)."""
 import ctypes as C
-import math
 import os
 import random
 import re

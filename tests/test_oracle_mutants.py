@@ -11,7 +11,6 @@ import os
 import subprocess
 import tempfile
 
-import pytest
 
 import oracle
 import test_oracle as pins
