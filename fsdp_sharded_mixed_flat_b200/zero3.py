@@ -338,14 +338,14 @@ def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Opt
     """All-gather of the D bf16 shards into the flat block and/or per-tensor buffers."""
     if len(shards) != plan.D:
         raise ValueError(f"need {plan.D} shards, got {len(shards)}")
+    if tensor_out is not None and len(tensor_out) != plan.n_tensors:
+        raise ValueError(f"need {plan.n_tensors} tensor outputs, got {len(tensor_out)}")
     sp = (C.c_void_p * plan.D)()
     for r, s in enumerate(shards):
         sp[r] = _dev_tensor(s, torch.bfloat16, plan.S, f"shards[{r}]")
     fp = None if flat_out is None else _dev_tensor(flat_out, torch.bfloat16, plan.N_pad, "flat_out")
     tp = None
     if tensor_out is not None:
-        if len(tensor_out) != plan.n_tensors:
-            raise ValueError(f"need {plan.n_tensors} tensor outputs, got {len(tensor_out)}")
         tp = (C.c_void_p * max(1, plan.n_tensors))()
         for i, t in enumerate(tensor_out):
             tp[i] = None if t is None else _dev_tensor(t, torch.bfloat16, plan.numels[i], f"tensor_out[{i}]")
