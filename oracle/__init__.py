@@ -1,7 +1,7 @@
 """The oracle: a plain, slow, single-threaded CPU restatement of the per-rank
 ZeRO-3 / FSDP step (plan, memory ledger, reduce-scatter, AdamW, bf16 cast,
-all-gather, unflatten), written in C (oracle/zero3_ref.c) and driven here
-through ctypes on numpy arrays.
+all-gather, unflatten, and the HYBRID_SHARD form of the reduction), written in
+C (oracle/zero3_ref.c) and driven here through ctypes on numpy arrays.
 
 TEST INFRASTRUCTURE ONLY.  Only tests/, the package's smoke check and the
 benchmark's CPU-baseline leg may import this module.  It shares no code with
@@ -77,6 +77,10 @@ def _bind(L):
     L.ref_adamw.restype = C.c_int
     L.ref_reduce_adamw.argtypes = [i32, i64, i32, p, i32, p, p, p, p, i32, C.POINTER(AdamWHP)]
     L.ref_reduce_adamw.restype = C.c_int
+    L.ref_reduce_scatter_hybrid.argtypes = [i32, i32, i64, i32, p, i32, i32, p]
+    L.ref_reduce_scatter_hybrid.restype = C.c_int
+    L.ref_reduce_adamw_hybrid.argtypes = [i32, i32, i64, i32, p, i32, p, p, p, p, i32, C.POINTER(AdamWHP)]
+    L.ref_reduce_adamw_hybrid.restype = C.c_int
     L.ref_all_gather.argtypes = [i32, i64, p, p]
     L.ref_all_gather.restype = None
     L.ref_unflatten.argtypes = [p, i32, p, p, p]
@@ -189,6 +193,41 @@ def reduce_adamw(contribs, S: int, rank: int, master, exp_avg, exp_avg_sq, work_
                                 C.byref(h))
     if rc != 0:
         raise ValueError("invalid reduce_adamw arguments")
+
+
+# ------------------------------------------------------------- HYBRID_SHARD
+def _replica_split(contribs, R: int) -> int:
+    if R < 1 or len(contribs) % R:
+        raise ValueError(f"{len(contribs)} contributions do not split into {R} nodes")
+    return len(contribs) // R
+
+
+def reduce_scatter_hybrid(contribs, R: int, S: int, rank: int, layout: int = LAYOUT_FULL,
+                          reduce_dtype: int = REDUCE_FP32) -> np.ndarray:
+    """The averaged gradient for R nodes of D = len(contribs) / R ranks; the
+    contribution of local rank d on node k is contribs[k * D + d]."""
+    contribs = [_u16(c) for c in contribs]
+    D = _replica_split(contribs, R)
+    out = np.empty(D * S if rank < 0 else S, dtype=np.float32)
+    rc = lib().ref_reduce_scatter_hybrid(R, D, S, rank, _ptr_array(contribs), layout, reduce_dtype, _ptr(out))
+    if rc != 0:
+        raise ValueError("invalid reduce_scatter_hybrid arguments")
+    return out
+
+
+def reduce_adamw_hybrid(contribs, R: int, S: int, rank: int, master, exp_avg, exp_avg_sq, work_bf16,
+                        h: AdamWHP, layout: int = LAYOUT_FULL, reduce_dtype: int = REDUCE_FP32) -> None:
+    """The HYBRID_SHARD step, in place on master / exp_avg / exp_avg_sq; writes work_bf16."""
+    contribs = [_u16(c) for c in contribs]
+    D = _replica_split(contribs, R)
+    for a in (master, exp_avg, exp_avg_sq):
+        assert a.flags.c_contiguous and a.dtype == np.float32
+    assert work_bf16.flags.c_contiguous and work_bf16.dtype == np.uint16
+    rc = lib().ref_reduce_adamw_hybrid(R, D, S, rank, _ptr_array(contribs), layout, _ptr(master),
+                                       _ptr(exp_avg), _ptr(exp_avg_sq), _ptr(work_bf16), reduce_dtype,
+                                       C.byref(h))
+    if rc != 0:
+        raise ValueError("invalid reduce_adamw_hybrid arguments")
 
 
 # ------------------------------------------------------- gather and unflatten

@@ -30,8 +30,9 @@
  *         memory in three buckets, §3 ZeRO-1, §4 ZeRO-2, §5.1 Forward and
  *         backward pass under FSDP, §5.2 Memory accounting.
  *   [P3] "Building GPT from Scratch — Part 8: FSDP — When the Model Won't
- *         Fit", sections "AllGather vs AllReduce" and "Mixed Precision:
- *         Cutting Memory in Half".
+ *         Fit", sections "AllGather vs AllReduce", "Mixed Precision:
+ *         Cutting Memory in Half", "HYBRID_SHARD: The Multi-Node Strategy"
+ *         and "Key Takeaways".
  *
  * Readings where the pages are silent:
  *   - flat layout: tensors packed row-major in list order, no padding between
@@ -39,6 +40,8 @@
  *   - the reduction sums ranks 0..D-1 left to right, starting from rank 0's
  *     value, then multiplies by the binary32 constant 1/D;
  *   - bf16 reduce: every partial sum is rounded to bf16 (round-nearest-even);
+ *   - HYBRID_SHARD: node sums first, then the node sums in node order, then
+ *     1/(R*D) (reduce_hybrid_one() below);
  *   - AdamW: decoupled weight decay applied to every element, bias-corrected
  *     moments, 1-based step count, the operation order of adamw_one() below;
  *   - every fp32 -> bf16 conversion rounds to nearest-even.
@@ -318,6 +321,98 @@ int ref_reduce_adamw(int32_t D, int64_t S, int32_t rank, const uint16_t* const* 
         for (int64_t j = 0; j < S; ++j) {
             int64_t s = rank < 0 ? (int64_t)r * S + j : j;
             float g = reduce_one(D, contrib, contrib_index(layout, S, r, j), reduce_dtype, inv_D);
+            adamw_one(&c, g, &master[s], &exp_avg[s], &exp_avg_sq[s]);
+            work_bf16[s] = ref_bf16_from_f32(master[s]);
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* HYBRID_SHARD.  [P3] "HYBRID_SHARD: The Multi-Node Strategy": R nodes of D */
+/* GPUs; the model is sharded D ways inside each node and replicated across  */
+/* the nodes, and the gradient crosses nodes in one all-reduce.  [P3] "Key   */
+/* Takeaways": the result is the same gradient as on one GPU, so the sum is  */
+/* scaled by 1/(R*D), the average over every data-parallel rank.             */
+/* Reading: global rank k*D + d is local rank d of node k, and its           */
+/* contribution is contrib[k*D + d].  Inside node k the ranks are folded     */
+/* 0..D-1 left to right (the node's reduce-scatter); the R node sums are     */
+/* then folded in node order 0..R-1 (the cross-node all-reduce, which leaves */
+/* the same sum on every node, so the replicas stay identical); the total is */
+/* multiplied by the binary32 constant 1/(R*D).  In bf16 mode every partial  */
+/* sum, inside a node and across nodes, is rounded to bf16.  R = 1 is the    */
+/* plain reduction above.                                                    */
+/* ------------------------------------------------------------------------ */
+static float reduce_hybrid_one(int32_t R, int32_t D, const uint16_t* const* contrib, int64_t idx,
+                               int32_t reduce_dtype, float inv_RD)
+{
+    if (reduce_dtype == 0) {
+        float total = 0.0f;
+        for (int32_t k = 0; k < R; ++k) {
+            const uint16_t* const* node = contrib + (int64_t)k * D;
+            float node_sum = ref_f32_from_bf16(node[0][idx]);
+            for (int32_t d = 1; d < D; ++d)
+                node_sum = node_sum + ref_f32_from_bf16(node[d][idx]);
+            total = (k == 0) ? node_sum : total + node_sum;
+        }
+        return total * inv_RD;
+    } else {
+        uint16_t total = 0;
+        for (int32_t k = 0; k < R; ++k) {
+            const uint16_t* const* node = contrib + (int64_t)k * D;
+            uint16_t node_sum = node[0][idx];
+            for (int32_t d = 1; d < D; ++d)
+                node_sum = ref_bf16_from_f32(ref_f32_from_bf16(node_sum) + ref_f32_from_bf16(node[d][idx]));
+            total = (k == 0) ? node_sum
+                             : ref_bf16_from_f32(ref_f32_from_bf16(total) + ref_f32_from_bf16(node_sum));
+        }
+        return ref_f32_from_bf16(ref_bf16_from_f32(ref_f32_from_bf16(total) * inv_RD));
+    }
+}
+
+static int hybrid_args_invalid(int32_t R, int32_t D, int64_t S, int32_t rank, int32_t layout,
+                               int32_t reduce_dtype)
+{
+    return R < 1 || D < 1 || S < 0 || rank < -1 || rank >= D || (layout != 0 && layout != 1) ||
+           (reduce_dtype != 0 && reduce_dtype != 1) || (rank == -1 && layout == 1);
+}
+
+/* The averaged gradient of the HYBRID_SHARD step for local rank `rank`'s
+ * partition (S elements), or for every local rank in order (rank = -1: the
+ * node's N_pad elements).  contrib holds R*D buffers; layouts as for
+ * ref_reduce_scatter.  Returns 0, or -1 on an invalid argument. */
+int ref_reduce_scatter_hybrid(int32_t R, int32_t D, int64_t S, int32_t rank, const uint16_t* const* contrib,
+                              int32_t layout, int32_t reduce_dtype, float* g_out)
+{
+    if (hybrid_args_invalid(R, D, S, rank, layout, reduce_dtype))
+        return -1;
+    float inv_RD = inverse_of(R * D);
+    int32_t r0 = rank < 0 ? 0 : rank;
+    int32_t r1 = rank < 0 ? D : rank + 1;
+    for (int32_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < S; ++j) {
+            int64_t out = rank < 0 ? (int64_t)r * S + j : j;
+            g_out[out] = reduce_hybrid_one(R, D, contrib, contrib_index(layout, S, r, j), reduce_dtype, inv_RD);
+        }
+    return 0;
+}
+
+/* The whole HYBRID_SHARD step of local rank `rank` (or of every local rank):
+ * the two-level reduction above, AdamW on the owned state, the bf16 cast.
+ * Every node's replica of the rank computes exactly this. */
+int ref_reduce_adamw_hybrid(int32_t R, int32_t D, int64_t S, int32_t rank, const uint16_t* const* contrib,
+                            int32_t layout, float* master, float* exp_avg, float* exp_avg_sq,
+                            uint16_t* work_bf16, int32_t reduce_dtype, const ref_adamw_hp* hp)
+{
+    if (hybrid_args_invalid(R, D, S, rank, layout, reduce_dtype) || hp->step < 1)
+        return -1;
+    ref_adamw_consts c = adamw_consts(hp);
+    float inv_RD = inverse_of(R * D);
+    int32_t r0 = rank < 0 ? 0 : rank;
+    int32_t r1 = rank < 0 ? D : rank + 1;
+    for (int32_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < S; ++j) {
+            int64_t s = rank < 0 ? (int64_t)r * S + j : j;
+            float g = reduce_hybrid_one(R, D, contrib, contrib_index(layout, S, r, j), reduce_dtype, inv_RD);
             adamw_one(&c, g, &master[s], &exp_avg[s], &exp_avg_sq[s]);
             work_bf16[s] = ref_bf16_from_f32(master[s]);
         }

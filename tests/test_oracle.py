@@ -382,6 +382,117 @@ def test_reduce_adamw_composes_reduce_then_adamw():
         assert np.array_equal(a[3], bf16_torch_bits(b[0]))
 
 
+# -------------------------------------------------------------- HYBRID_SHARD
+def test_hybrid_worked_examples(golden):
+    """Pin: hand-derived HYBRID_SHARD reductions (R nodes of D ranks) in which
+    the node-then-cross-node order, the rank-to-node map, the node order, the
+    bf16 rounding of every partial sum and the 1/(R*D) scale each change the
+    result."""
+    g = golden("hybrid_worked_examples.json")
+    for case in g["cases"]:
+        R, D = case["R"], case["D"]
+        contribs = [bf16_torch_bits(np.array([x], dtype=np.float32)) for x in case["contributions"]]
+        assert [float(oracle.f32_from_bf16(c)[0]) for c in contribs] == case["contributions"]
+        got = oracle.reduce_scatter_hybrid(contribs, R, 1, 0, oracle.LAYOUT_OWNED, case["reduce_dtype"])
+        assert float(got[0]) == case["expected"], case["name"]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("D", [1, 2, 3, 8])
+def test_hybrid_one_node_is_the_plain_reduction(D, mode):
+    """Pin: with one node, HYBRID_SHARD is FULL_SHARD: bit-identical to the
+    plain reduce-scatter, for every rank and layout."""
+    rng = np.random.default_rng(300 + D)
+    S = 29
+    contribs = [rand_bf16(rng, D * S) for _ in range(D)]
+    every = oracle.reduce_scatter_hybrid(contribs, 1, S, -1, oracle.LAYOUT_FULL, mode)
+    plain = oracle.reduce_scatter(contribs, S, -1, reduce_dtype=mode)
+    assert np.array_equal(every.view(np.uint32), plain.view(np.uint32))
+    for r in range(D):
+        owned = [c[r * S:(r + 1) * S].copy() for c in contribs]
+        got = oracle.reduce_scatter_hybrid(owned, 1, S, r, oracle.LAYOUT_OWNED, mode)
+        assert np.array_equal(got.view(np.uint32), every[r * S:(r + 1) * S].view(np.uint32))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("R", [2, 3, 4, 8])
+def test_hybrid_one_rank_per_node_is_the_plain_fold_over_nodes(R, mode):
+    """Pin: with one rank per node, the node sums are the contributions and the
+    result is the plain left fold over R ranks times 1/R."""
+    rng = np.random.default_rng(400 + R)
+    S = 31
+    contribs = [rand_bf16(rng, S) for _ in range(R)]
+    got = oracle.reduce_scatter_hybrid(contribs, R, S, -1, oracle.LAYOUT_FULL, mode)
+    ref = oracle.reduce_scatter(contribs, S, 0, oracle.LAYOUT_OWNED, mode)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("R,D", [(2, 2), (4, 8), (2, 16), (8, 4)])
+def test_hybrid_integers_are_the_exact_mean(R, D):
+    """Pin: with small-integer contributions every partial sum is exact, so
+    both reduce dtypes give exactly sum / (R*D) for power-of-two R*D."""
+    S = 16
+    contribs = [synth.bf16_bits(synth.contribution(D * S, D * S, seed=5, step=1, rank=i, sigma=0,
+                                                   dist="integers")) for i in range(R * D)]
+    exact = np.sum([oracle.f32_from_bf16(c).astype(np.float64) for c in contribs], axis=0) / (R * D)
+    for mode in (oracle.REDUCE_FP32, oracle.REDUCE_BF16):
+        got = oracle.reduce_scatter_hybrid(contribs, R, S, -1, oracle.LAYOUT_FULL, mode)
+        assert np.array_equal(got.astype(np.float64), exact)
+
+
+@pytest.mark.parametrize("R,D", [(2, 3), (4, 8), (3, 5)])
+def test_hybrid_matches_torch_two_level_fold(R, D):
+    """Pin: torch's own fp32 and bf16 tensor additions, node by node and then
+    across nodes, scaled by fp32(1/(R*D)) (rounded to bf16 in bf16 mode)."""
+    rng = np.random.default_rng(500 + R * D)
+    S = 19
+    contribs = [rand_bf16(rng, D * S) for _ in range(R * D)]
+    t = [torch.from_numpy(c.view(np.int16)).view(torch.bfloat16) for c in contribs]
+    inv = torch.tensor(1.0 / (R * D), dtype=torch.float32)
+    for mode, cast in ((oracle.REDUCE_FP32, lambda x: x.float()), (oracle.REDUCE_BF16, lambda x: x)):
+        nodes = []
+        for k in range(R):
+            acc = cast(t[k * D]).clone()
+            for d in range(1, D):
+                acc = acc + cast(t[k * D + d])
+            nodes.append(acc)
+        total = nodes[0]
+        for k in range(1, R):
+            total = total + nodes[k]
+        ref = total.float() * inv
+        if mode == oracle.REDUCE_BF16:
+            ref = ref.to(torch.bfloat16).float()
+        got = oracle.reduce_scatter_hybrid(contribs, R, S, -1, oracle.LAYOUT_FULL, mode)
+        assert np.array_equal(got.view(np.uint32), ref.numpy().view(np.uint32))
+
+
+def test_hybrid_step_composes_reduce_then_adamw():
+    """The fused HYBRID_SHARD step is its reduction followed by AdamW and the cast."""
+    rng = np.random.default_rng(22)
+    R, D, S = 3, 4, 40
+    contribs = [rand_bf16(rng, D * S) for _ in range(R * D)]
+    p0 = (rng.standard_normal(D * S) * 0.02).astype(np.float32)
+    for mode in (oracle.REDUCE_FP32, oracle.REDUCE_BF16):
+        a = [p0.copy(), np.zeros(D * S, np.float32), np.zeros(D * S, np.float32), np.zeros(D * S, np.uint16)]
+        oracle.reduce_adamw_hybrid(contribs, R, S, -1, *a, oracle.hp(step=2), reduce_dtype=mode)
+        g = oracle.reduce_scatter_hybrid(contribs, R, S, -1, reduce_dtype=mode)
+        b = [p0.copy(), np.zeros(D * S, np.float32), np.zeros(D * S, np.float32)]
+        oracle.adamw(g, *b, oracle.hp(step=2))
+        for x, y in zip(a[:3], b):
+            assert np.array_equal(x, y)
+        assert np.array_equal(a[3], bf16_torch_bits(b[0]))
+
+
+def test_hybrid_rejects_bad_arguments():
+    c = [np.zeros(8, dtype=np.uint16)] * 4
+    with pytest.raises(ValueError):
+        oracle.reduce_scatter_hybrid(c, 3, 4, -1)          # 4 contributions do not split into 3 nodes
+    with pytest.raises(ValueError):
+        oracle.reduce_scatter_hybrid(c, 2, 4, 2)           # local rank out of range (D = 2)
+    with pytest.raises(ValueError):
+        oracle.reduce_scatter_hybrid(c, 2, 4, -1, oracle.LAYOUT_OWNED)
+
+
 # --------------------------------------------------------- gather, unflatten
 def test_allgather_worked_example(golden):
     """Pin: page 3's 4-GPU all-gather: every GPU ends with [A, B, C, D]."""

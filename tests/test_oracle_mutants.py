@@ -46,6 +46,46 @@ MUTANTS = [
      "case 1: return optim * N / D + weights * N;"),
     ("the unflatten starts one element late", "out[t][k] = flat[offset[t] + k];",
      "out[t][k] = flat[offset[t] + k + (k + 1 < numel[t] ? 1 : 0)];"),
+    ("HYBRID_SHARD folds all ranks flat, ignoring the nodes",
+     "float node_sum = ref_f32_from_bf16(node[0][idx]);",
+     "float node_sum = k == 0 ? ref_f32_from_bf16(node[0][idx]) : total + ref_f32_from_bf16(node[0][idx]);"
+     " total = 0.0f;"),
+    ("HYBRID_SHARD scales by 1/D instead of 1/(R*D)", "return total * inv_RD;",
+     "return total * (inv_RD * (float)R);"),
+    ("HYBRID_SHARD sums the nodes in reverse order",
+     "const uint16_t* const* node = contrib + (int64_t)k * D;\n            float node_sum",
+     "const uint16_t* const* node = contrib + (int64_t)(R - 1 - k) * D;\n            float node_sum"),
+    ("HYBRID_SHARD maps rank k*D+d to node d",
+     "node_sum = node_sum + ref_f32_from_bf16(node[d][idx]);",
+     "node_sum = node_sum + ref_f32_from_bf16(contrib[(int64_t)d * R + k][idx]);"),
+    ("HYBRID_SHARD rounds each bf16 node sum once, at the node's end",
+     "uint16_t node_sum = node[0][idx];\n"
+     "            for (int32_t d = 1; d < D; ++d)\n"
+     "                node_sum = ref_bf16_from_f32(ref_f32_from_bf16(node_sum) + ref_f32_from_bf16(node[d][idx]));",
+     "float node_f = ref_f32_from_bf16(node[0][idx]);\n"
+     "            for (int32_t d = 1; d < D; ++d)\n"
+     "                node_f = node_f + ref_f32_from_bf16(node[d][idx]);\n"
+     "            uint16_t node_sum = ref_bf16_from_f32(node_f);"),
+    ("HYBRID_SHARD bf16 cross-node sums are kept in fp32",
+     "        uint16_t total = 0;\n"
+     "        for (int32_t k = 0; k < R; ++k) {\n"
+     "            const uint16_t* const* node = contrib + (int64_t)k * D;\n"
+     "            uint16_t node_sum = node[0][idx];\n"
+     "            for (int32_t d = 1; d < D; ++d)\n"
+     "                node_sum = ref_bf16_from_f32(ref_f32_from_bf16(node_sum) + ref_f32_from_bf16(node[d][idx]));\n"
+     "            total = (k == 0) ? node_sum\n"
+     "                             : ref_bf16_from_f32(ref_f32_from_bf16(total) + ref_f32_from_bf16(node_sum));\n"
+     "        }\n"
+     "        return ref_f32_from_bf16(ref_bf16_from_f32(ref_f32_from_bf16(total) * inv_RD));",
+     "        float total = 0.0f;\n"
+     "        for (int32_t k = 0; k < R; ++k) {\n"
+     "            const uint16_t* const* node = contrib + (int64_t)k * D;\n"
+     "            uint16_t node_sum = node[0][idx];\n"
+     "            for (int32_t d = 1; d < D; ++d)\n"
+     "                node_sum = ref_bf16_from_f32(ref_f32_from_bf16(node_sum) + ref_f32_from_bf16(node[d][idx]));\n"
+     "            total = (k == 0) ? ref_f32_from_bf16(node_sum) : total + ref_f32_from_bf16(node_sum);\n"
+     "        }\n"
+     "        return ref_f32_from_bf16(ref_bf16_from_f32(total * inv_RD));"),
 ]
 
 
@@ -73,6 +113,13 @@ PINS = [
     lambda: pins.test_adamw_ten_steps_matches_torch_adamw_float64(),
     lambda: pins.test_reduce_adamw_composes_reduce_then_adamw(),
     lambda: pins.test_sharded_steps_equal_one_unsharded_step(4, 1, [5, 7, 1]),
+    lambda: pins.test_hybrid_worked_examples(golden),
+    lambda: pins.test_hybrid_integers_are_the_exact_mean(4, 8),
+    lambda: pins.test_hybrid_one_node_is_the_plain_reduction(3, 0),
+    lambda: pins.test_hybrid_one_node_is_the_plain_reduction(3, 1),
+    lambda: pins.test_hybrid_one_rank_per_node_is_the_plain_fold_over_nodes(3, 0),
+    lambda: pins.test_hybrid_one_rank_per_node_is_the_plain_fold_over_nodes(3, 1),
+    lambda: pins.test_hybrid_matches_torch_two_level_fold(2, 3),
 ]
 
 
