@@ -39,7 +39,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "owned params/s for fused reduce+AdamW+cast; achieved HBM GB/s vs ~8 TB/s"
 UNIT = "owned params/s"
-PROFILE_K1 = os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md")
+# committed ncu summaries of the fused kernel, by workload (fp32 reduce), with its DRAM traffic
+PROFILE_K1 = {"llama7b_d8": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md"),
+              "llama7b_hybrid": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_hybrid_llama7b_4x8.md")}
 K1_SOURCE = os.path.join(ROOT, "fsdp_sharded_mixed_flat_b200", "csrc", "reduce_adamw.cu")
 SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
@@ -84,12 +86,13 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per launch from the committed ncu summary of the fused kernel,
-    if that summary was taken on the current kernel source; else None."""
-    if not os.path.exists(PROFILE_K1):
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary of the fused kernel on
+    this workload, if that summary was taken on the current kernel source; else None."""
+    path = PROFILE_K1.get(workload)
+    if path is None or not os.path.exists(path):
         return None
-    text = open(PROFILE_K1).read()
+    text = open(path).read()
     sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     tb = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not sha or not tb:
@@ -192,19 +195,25 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
         workload = "llama70b_layer"
     w = synth.WORKLOADS[workload]
     D = D or w["D"]
+    nodes = w.get("nodes", 1)
     n = min(sample, synth.block_numel(w["tensors"]))
     contribs = [synth.bf16_bits(synth.contribution(n, n, seed=seed, step=1, rank=d, sigma=w["sigma"],
                                                    dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
-                                                   device="cpu")) for d in range(D)]
+                                                   device="cpu")) for d in range(nodes * D)]
     p = synth.master_weights(n, n, seed=seed).numpy().copy()
     m, v, wk = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
     oracle.lib()
     t0 = time.perf_counter()
     for t in range(1, steps + 1):
-        oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED,
-                            reduce_dtype=reduce_dtype)
+        if nodes > 1:
+            oracle.reduce_adamw_hybrid(contribs, nodes, n, 0, p, m, v, wk, oracle.hp(step=t),
+                                       layout=oracle.LAYOUT_OWNED, reduce_dtype=reduce_dtype)
+        else:
+            oracle.reduce_adamw(contribs, n, 0, p, m, v, wk, oracle.hp(step=t), layout=oracle.LAYOUT_OWNED,
+                                reduce_dtype=reduce_dtype)
     dt = time.perf_counter() - t0
-    desc = (f"{workload}: first {n} owned elements x {steps} steps, D={D}, "
+    shape = f"{nodes} nodes x D={D}" if nodes > 1 else f"D={D}"
+    desc = (f"{workload}: first {n} owned elements x {steps} steps, {shape}, "
             f"{'bf16' if reduce_dtype else 'fp32'} reduce, one thread "
             f"(oracle/zero3_ref.c, single-threaded C)")
     return n * steps / dt, dt, desc
@@ -249,8 +258,13 @@ class BlockRunner:
         self.specs = z3.tensor_specs(self.shapes)       # the step's input: the block's tensor list
         plan = z3.zero3_plan(self.shapes, D, synth.ALIGN)
         self.N, self.N_pad, self.S = plan.N, plan.N_pad, plan.S
-        self.contribs = synth.contributions(D, self.N, self.N_pad, seed=seed, step=1, sigma=w["sigma"],
-                                            dist=w["dist"], zero_frac=w.get("zero_frac", 0.0), device=dev)
+        # HYBRID_SHARD: `nodes` nodes of D ranks, contribution k*D + d from rank d of node k
+        self.nodes = w.get("nodes", 1)
+        if self.nodes > 1 and (stage != 3 or graph or offload):
+            raise SystemExit("the HYBRID_SHARD workload runs the plain ZeRO-3 block step")
+        self.contribs = synth.contributions(self.nodes * D, self.N, self.N_pad, seed=seed, step=1,
+                                            sigma=w["sigma"], dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
+                                            device=dev)
         self.master = synth.master_weights(self.N, self.N_pad, seed=seed, device=dev)
         self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
         self.offload = offload
@@ -272,14 +286,19 @@ class BlockRunner:
                            if unflatten_copy and stage == 3 else None)
         self.units_per_step = self.N_pad                       # owned params, all ranks
         self.k1_launches_per_step = 1
-        self.k1_bytes_per_launch = (2 * D + 26) * self.N_pad   # stage 1/2: the bf16 goes to the block instead
+        # stage 1/2: the bf16 goes to the block instead of the shard; same bytes
+        self.k1_bytes_per_launch = (2 * self.nodes * D + 26) * self.N_pad
         self.step_bytes = self.k1_bytes_per_launch + (4 * self.N_pad if stage == 3 else 0) + \
             (4 * self.N if self.tensor_out is not None else 0)
         self.launches_per_step = (2 + (1 if self.tensor_out is not None else 0)) if stage == 3 else 1
-        self.k1_name = (f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}"
+        ranks = f"{self.nodes} nodes x D={D}" if self.nodes > 1 else f"D={D}"
+        self.k1_name = (f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, {ranks}"
                         f"{', gather' if stage != 3 else ''}>")
-        what = ("fused reduce/AdamW/cast over all %d partitions + gather into the flat block%s" %
-                (D, " and into one buffer per tensor" if self.tensor_out is not None else "") if stage == 3
+        hybrid = (" (HYBRID_SHARD: each node's rank fold, then the node sums across %d nodes, then 1/%d)"
+                  % (self.nodes, self.nodes * D) if self.nodes > 1 else "")
+        what = ("fused reduce/AdamW/cast over all %d partitions%s + gather into the flat block%s" %
+                (D, hybrid, " and into one buffer per tensor" if self.tensor_out is not None else "")
+                if stage == 3
                 else "one kernel: reduce/AdamW/cast over all %d partitions writing the replicated bf16 "
                      "weights in place of the gather (ZeRO-%d)" % (D, stage))
         self.graphed = None
@@ -338,8 +357,12 @@ class BlockRunner:
                 k1_events[0][1].record(self.stream)
             return self.views(pl, flat)
         # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
-        z3.zero3_reduce_adamw(pl, -1, contribs, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
-                              reduce_dtype=self.mode, stream=self.stream)
+        if self.nodes > 1:
+            z3.zero3_reduce_adamw_hybrid(pl, -1, self.nodes, contribs, self.master, self.exp_avg,
+                                         self.exp_avg_sq, self.work, hp, reduce_dtype=self.mode, stream=self.stream)
+        else:
+            z3.zero3_reduce_adamw(pl, -1, contribs, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
+                                  reduce_dtype=self.mode, stream=self.stream)
         if k1_events is not None:
             k1_events[0][1].record(self.stream)
         # a5 + a6: all-gather of the D bf16 shards into the flat block; views are zero-copy
@@ -360,7 +383,7 @@ class BlockRunner:
         second device set of both so that transfers of neighbouring steps overlap."""
         import torch
         dev = self.device
-        self.host_c = [torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in range(self.D)]
+        self.host_c = [torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True) for _ in self.contribs]
         for h, c in zip(self.host_c, self.contribs):
             h.copy_(c)
         self.host_flat = torch.empty(self.N_pad, dtype=torch.bfloat16, pin_memory=True)
@@ -584,7 +607,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D, "stage": getattr(R, "stage", 3),
+        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D, "nodes": getattr(R, "nodes", 1),
+                   "stage": getattr(R, "stage", 3),
                    "reduce_dtype": "bf16" if mode == z3.Z3_REDUCE_BF16 else "fp32",
                    "owned_params_per_step": R.units_per_step,
                    "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (R.step_bytes / 1e9),
@@ -598,7 +622,8 @@ def run_ours(args):
                      "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
                      "frac_of_nominal_8000": k1_gbs / 8000.0, "kernel": R.k1_name,
                      "algorithmic_bytes_per_launch": R.k1_bytes_per_launch,
-                     "traffic": profiled_traffic() if args.workload == "llama7b_d8" and mode == 0 else None},
+                     "traffic": (profiled_traffic(args.workload)
+                                 if mode == 0 and args.stage == 3 and not args.graph else None)},
         "clocks": clk,
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},

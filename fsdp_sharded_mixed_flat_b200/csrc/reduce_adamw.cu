@@ -8,7 +8,10 @@
 // every rank's gradient) and "Mixed Precision: Cutting Memory in Half" (fp32
 // master, bf16 params); "7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)",
 // §3 (rank r updates only P_r from its fp32 master, m, v and gradient slice)
-// and §4 (reduce-scatter replaces the all-reduce).
+// and §4 (reduce-scatter replaces the all-reduce).  The HYBRID_SHARD form
+// ("Building GPT from Scratch — Part 8", "HYBRID_SHARD: The Multi-Node
+// Strategy") reduces R nodes of D ranks in two levels: each node's ranks in
+// rank order, then the node sums in node order.
 //
 // The pass is bound by HBM bandwidth: per owned element it reads 2*D bytes of
 // contributions and 12 bytes of state, and writes 12 bytes of state and 2
@@ -56,7 +59,7 @@ struct AdamScalars {
 };
 
 struct K1Args {
-    const uint16_t* c[Z3_D_MAX];  // contributions, each at the launch's first element
+    const uint16_t* c[Z3_D_MAX];  // contributions c[k*D + d] (node k, rank d), each at the launch's first element
     float* p;                     // master
     float* m;                     // exp_avg
     float* v;                     // exp_avg_sq
@@ -64,10 +67,11 @@ struct K1Args {
     uint16_t* g[Z3_GATHER_MAX];   // gathered blocks, each at the launch's first element
     int32_t ng;                   // number of gathered blocks
     int64_t n;                    // elements in this launch
-    int32_t D;
-    float inv_D;                  // fp32 nearest to 1/D
+    int32_t D;                    // ranks per node
+    float inv_n;                  // fp32 nearest to 1/(R*D)
     AdamScalars s;                // this step's scalars (unless s_dev is used)
     const AdamScalars* s_dev;     // device copy of the scalars (the DEVS kernels)
+    int32_t R;                    // nodes (HYBRID_SHARD; 1 otherwise)
 };
 
 static_assert(sizeof(AdamScalars) == Z3_SCALARS * sizeof(float), "scalar layout");
@@ -162,14 +166,13 @@ __device__ __forceinline__ void fold8_bf16(uint32_t (&acc)[4], const uint4& q, b
     for (int k = 0; k < 4; ++k) acc[k] = first ? w[k] : add_bf16x2(acc[k], w[k]);
 }
 
-// Reduce ranks 0..D-1 for the 8 elements starting at e, left to right, in
-// chunks of ranks (the chunk's loads are all issued before its folds), and
-// return the averaged gradient g = sum * (1/D) in the reduce dtype.
+// Fold ranks base..base+D-1 for the 8 elements starting at e into the fp32 or
+// packed-bf16 accumulators, left to right, in chunks of ranks (the chunk's
+// loads are all issued before its folds).
 template <int MODE, int DT>
-__device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8]) {
+__device__ __forceinline__ void fold_ranks(const K1Args& a, int base, int64_t e, float (&acc)[8],
+                                           uint32_t (&accw)[4]) {
     const int D = DT > 0 ? DT : a.D;
-    float acc[8];
-    uint32_t accw[4];
     // ranks per chunk: 8, or 16 for the bf16 fold at D = 32 (measured 1.3 % faster there,
     // slower at D = 16; the fp32 fold did not change)
     constexpr int CH = (MODE != Z3_REDUCE_FP32 && DT >= 32) ? 16 : 8;
@@ -179,7 +182,7 @@ __device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8
         uint4 q[CH];
 #pragma unroll
         for (int k = 0; k < CH; ++k)
-            if (d0 + k < D) q[k] = ld16(reinterpret_cast<const uint4*>(a.c[d0 + k] + e));
+            if (d0 + k < D) q[k] = ld16(reinterpret_cast<const uint4*>(a.c[base + d0 + k] + e));
 #pragma unroll
         for (int k = 0; k < CH; ++k) {
             if (d0 + k >= D) continue;
@@ -189,33 +192,72 @@ __device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8
                 fold8_bf16(accw, q[k], d0 + k == 0);
         }
     }
+}
+
+// The averaged gradient g of the 8 elements starting at e, in the reduce dtype.
+// RT = 1: ranks 0..D-1 folded in order, times 1/D.  RT != 1 (HYBRID_SHARD; 0
+// means R from the arguments): each node's D ranks folded in order, the node
+// sums folded in node order, times 1/(R*D).
+template <int MODE, int DT, int RT>
+__device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8]) {
+    float acc[8];
+    uint32_t accw[4];
+    if constexpr (RT == 1) {
+        fold_ranks<MODE, DT>(a, 0, e, acc, accw);
+    } else {
+        const int D = DT > 0 ? DT : a.D;
+        const int R = RT > 0 ? RT : a.R;
+        float node[8];
+        uint32_t nodew[4];
+#pragma unroll(RT > 0 ? RT : 1)
+        for (int k = 0; k < R; ++k) {
+            fold_ranks<MODE, DT>(a, k * D, e, node, nodew);
+            if constexpr (MODE == Z3_REDUCE_FP32) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = k == 0 ? node[i] : __fadd_rn(acc[i], node[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) accw[i] = k == 0 ? nodew[i] : add_bf16x2(accw[i], nodew[i]);
+            }
+        }
+    }
     if constexpr (MODE == Z3_REDUCE_FP32) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) g[k] = __fmul_rn(acc[k], a.inv_D);
+        for (int k = 0; k < 8; ++k) g[k] = __fmul_rn(acc[k], a.inv_n);
     } else {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            g[2 * k] = round_to_bf16(__fmul_rn(lo_bf16(accw[k]), a.inv_D));
-            g[2 * k + 1] = round_to_bf16(__fmul_rn(hi_bf16(accw[k]), a.inv_D));
+            g[2 * k] = round_to_bf16(__fmul_rn(lo_bf16(accw[k]), a.inv_n));
+            g[2 * k + 1] = round_to_bf16(__fmul_rn(hi_bf16(accw[k]), a.inv_n));
         }
     }
 }
 
+// One partial sum in the reduce dtype: the fp32 sum, rounded to bf16 in bf16 mode.
 template <int MODE>
-__device__ __forceinline__ float finish(float acc, float inv_D) {
-    const float g = __fmul_rn(acc, inv_D);
-    return MODE == Z3_REDUCE_FP32 ? g : round_to_bf16(g);
+__device__ __forceinline__ float add_in(float x, float y) {
+    const float s = __fadd_rn(x, y);
+    return MODE == Z3_REDUCE_FP32 ? s : round_to_bf16(s);
 }
 
-// One element on the scalar path (tails and misaligned buffers).
-template <int MODE, bool GATHER>
+// One element on the scalar path (tails and misaligned buffers).  RT = 1: the
+// rank fold; otherwise the nodes' rank folds, then the fold of the node sums.
+template <int MODE, int RT, bool GATHER>
 __device__ __forceinline__ void scalar_elem(const K1Args& a, const AdamScalars& sc, int64_t i) {
-    float acc = bf16_of(a.c[0][i]);
-    for (int d = 1; d < a.D; ++d) {
-        const float x = bf16_of(a.c[d][i]);
-        acc = MODE == Z3_REDUCE_FP32 ? __fadd_rn(acc, x) : round_to_bf16(__fadd_rn(acc, x));
+    float total;
+    if constexpr (RT == 1) {
+        total = bf16_of(a.c[0][i]);
+        for (int d = 1; d < a.D; ++d) total = add_in<MODE>(total, bf16_of(a.c[d][i]));
+    } else {
+        const int R = RT > 0 ? RT : a.R;
+        for (int k = 0; k < R; ++k) {
+            float node = bf16_of(a.c[k * a.D][i]);
+            for (int d = 1; d < a.D; ++d) node = add_in<MODE>(node, bf16_of(a.c[k * a.D + d][i]));
+            total = k == 0 ? node : add_in<MODE>(total, node);
+        }
     }
-    const float g = finish<MODE>(acc, a.inv_D);
+    const float g0 = __fmul_rn(total, a.inv_n);
+    const float g = MODE == Z3_REDUCE_FP32 ? g0 : round_to_bf16(g0);
     float p = a.p[i], m = a.m[i], v = a.v[i];
     adamw_elem(sc, g, p, m, v);
     a.p[i] = p;
@@ -230,7 +272,7 @@ __device__ __forceinline__ void scalar_elem(const K1Args& a, const AdamScalars& 
 // The 8 elements starting at e: state loads, the rank fold, AdamW, stores.
 // GATHER: the bf16 result also goes to every gathered block (the all-gather's
 // data movement done by the producer of the data).
-template <int MODE, int DT, bool GATHER>
+template <int MODE, int DT, int RT, bool GATHER>
 __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc, int64_t e) {
     const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
     const float4 p1 = ld16(reinterpret_cast<const float4*>(a.p + e + 4));
@@ -239,7 +281,7 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
     const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
     const float4 v1 = ld16(reinterpret_cast<const float4*>(a.v + e + 4));
     float g[8];
-    reduce8<MODE, DT>(a, e, g);
+    reduce8<MODE, DT, RT>(a, e, g);
     float p[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
     float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
     float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
@@ -276,7 +318,7 @@ __device__ __forceinline__ AdamScalars load_scalars(const AdamScalars* p) {
 // free and every SM keeps streaming to the end; the outer loop only runs more
 // than once when the range exceeds the largest grid.  The last n % 8 elements
 // go through the scalar path.
-template <int MODE, int DT, bool GATHER>
+template <int MODE, int DT, int RT, bool GATHER>
 __device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc) {
     const int64_t n8 = a.n >> 3;
     const int64_t span = int64_t(kThreads) * kChunks;
@@ -285,38 +327,38 @@ __device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc)
 #pragma unroll
         for (int k = 0; k < kChunks; ++k) {
             const int64_t q = first + int64_t(k) * kThreads;
-            if (q < n8) process8<MODE, DT, GATHER>(a, sc, q << 3);
+            if (q < n8) process8<MODE, DT, RT, GATHER>(a, sc, q << 3);
         }
     }
     const int64_t tail = (n8 << 3) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
-    if (tail < a.n) scalar_elem<MODE, GATHER>(a, sc, tail);
+    if (tail < a.n) scalar_elem<MODE, RT, GATHER>(a, sc, tail);
 }
 
-template <int MODE, int DT, bool GATHER, bool DEVS>
+template <int MODE, int DT, int RT, bool GATHER, bool DEVS>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
     if constexpr (DEVS) {
         const AdamScalars sc = load_scalars(a.s_dev);
-        vec_body<MODE, DT, GATHER>(a, sc);
+        vec_body<MODE, DT, RT, GATHER>(a, sc);
     } else {
-        vec_body<MODE, DT, GATHER>(a, a.s);   // the scalars stay in the parameter block
+        vec_body<MODE, DT, RT, GATHER>(a, a.s);   // the scalars stay in the parameter block
     }
 }
 
 // Scalar kernel: any element-aligned pointers.
-template <int MODE, bool GATHER>
+template <int MODE, int RT, bool GATHER>
 __device__ __forceinline__ void scalar_body(const K1Args& a, const AdamScalars& sc) {
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t i = int64_t(blockIdx.x) * kThreads + threadIdx.x; i < a.n; i += stride)
-        scalar_elem<MODE, GATHER>(a, sc, i);
+        scalar_elem<MODE, RT, GATHER>(a, sc, i);
 }
 
-template <int MODE, bool GATHER, bool DEVS>
+template <int MODE, int RT, bool GATHER, bool DEVS>
 __global__ void __launch_bounds__(kThreads) k_reduce_adamw_scalar(const __grid_constant__ K1Args a) {
     if constexpr (DEVS) {
         const AdamScalars sc = load_scalars(a.s_dev);
-        scalar_body<MODE, GATHER>(a, sc);
+        scalar_body<MODE, RT, GATHER>(a, sc);
     } else {
-        scalar_body<MODE, GATHER>(a, a.s);
+        scalar_body<MODE, RT, GATHER>(a, a.s);
     }
 }
 
@@ -325,13 +367,13 @@ using KernelFn = void (*)(K1Args);
 template <int MODE, bool GATHER, bool DEVS>
 KernelFn pick_vec(int D) {
     switch (D) {
-    case 1: return k_reduce_adamw_vec<MODE, 1, GATHER, DEVS>;
-    case 2: return k_reduce_adamw_vec<MODE, 2, GATHER, DEVS>;
-    case 4: return k_reduce_adamw_vec<MODE, 4, GATHER, DEVS>;
-    case 8: return k_reduce_adamw_vec<MODE, 8, GATHER, DEVS>;
-    case 16: return k_reduce_adamw_vec<MODE, 16, GATHER, DEVS>;
-    case 32: return k_reduce_adamw_vec<MODE, 32, GATHER, DEVS>;
-    default: return k_reduce_adamw_vec<MODE, 0, GATHER, DEVS>;
+    case 1: return k_reduce_adamw_vec<MODE, 1, 1, GATHER, DEVS>;
+    case 2: return k_reduce_adamw_vec<MODE, 2, 1, GATHER, DEVS>;
+    case 4: return k_reduce_adamw_vec<MODE, 4, 1, GATHER, DEVS>;
+    case 8: return k_reduce_adamw_vec<MODE, 8, 1, GATHER, DEVS>;
+    case 16: return k_reduce_adamw_vec<MODE, 16, 1, GATHER, DEVS>;
+    case 32: return k_reduce_adamw_vec<MODE, 32, 1, GATHER, DEVS>;
+    default: return k_reduce_adamw_vec<MODE, 0, 1, GATHER, DEVS>;
     }
 }
 
@@ -340,11 +382,26 @@ KernelFn pick(bool vec, int32_t reduce_dtype, int D) {
     if (vec)
         return reduce_dtype == Z3_REDUCE_FP32 ? pick_vec<Z3_REDUCE_FP32, GATHER, DEVS>(D)
                                               : pick_vec<Z3_REDUCE_BF16, GATHER, DEVS>(D);
-    return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, GATHER, DEVS>
-                                          : k_reduce_adamw_scalar<Z3_REDUCE_BF16, GATHER, DEVS>;
+    return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, 1, GATHER, DEVS>
+                                          : k_reduce_adamw_scalar<Z3_REDUCE_BF16, 1, GATHER, DEVS>;
 }
 
-KernelFn pick_any(bool gather, bool devs, bool vec, int32_t reduce_dtype, int D) {
+// HYBRID_SHARD kernels (no fused gather, scalars by value): a specialised
+// vector kernel for 4 nodes of 8 ranks, and one for any other shape.
+template <int MODE>
+KernelFn pick_hybrid_vec(int R, int D) {
+    if (R == 4 && D == 8) return k_reduce_adamw_vec<MODE, 8, 4, false, false>;
+    return k_reduce_adamw_vec<MODE, 0, 0, false, false>;
+}
+
+KernelFn pick_any(bool gather, bool devs, bool vec, int32_t reduce_dtype, int D, int R) {
+    if (R > 1) {
+        if (vec)
+            return reduce_dtype == Z3_REDUCE_FP32 ? pick_hybrid_vec<Z3_REDUCE_FP32>(R, D)
+                                                  : pick_hybrid_vec<Z3_REDUCE_BF16>(R, D);
+        return reduce_dtype == Z3_REDUCE_FP32 ? k_reduce_adamw_scalar<Z3_REDUCE_FP32, 0, false, false>
+                                              : k_reduce_adamw_scalar<Z3_REDUCE_BF16, 0, false, false>;
+    }
     if (gather)
         return devs ? pick<true, true>(vec, reduce_dtype, D) : pick<true, false>(vec, reduce_dtype, D);
     return devs ? pick<false, true>(vec, reduce_dtype, D) : pick<false, false>(vec, reduce_dtype, D);
@@ -360,18 +417,22 @@ bool hp_valid(const z3_adamw* hp) {
            hp->beta1 < 1.0 && hp->beta2 >= 0.0 && hp->beta2 < 1.0;
 }
 
-// Validation and launch shared by both entry points.  `gathered` holds
+// Validation and launch shared by every entry point.  `gathered` holds
 // n_gathered whole padded blocks (0 for the plain entry point); `work_bf16`
 // may be null only when n_gathered > 0.
 // Exactly one of hp (scalars computed here, passed by value) and dev_scalars
 // (read by the kernel from device memory) is non-null.
-int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, int32_t contrib_layout,
+// R: nodes of D ranks each (HYBRID_SHARD, contrib holds R*D pointers; only
+// with n_gathered = 0 and hp), 1 otherwise.
+int launch_k1(const z3_plan* p, int32_t rank, int32_t R, const uint16_t* const* contrib, int32_t contrib_layout,
               float* master, float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
               uint16_t* const* gathered, int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
               const float* dev_scalars, void* cuda_stream) {
     // ---- arguments
     if (p == nullptr || contrib == nullptr || (hp == nullptr) == (dev_scalars == nullptr)) return Z3_EINVAL;
     const int32_t D = p->D;
+    if (R < 1 || R > Z3_D_MAX / D || (R > 1 && (n_gathered != 0 || hp == nullptr))) return Z3_EINVAL;
+    const int32_t n_contrib = R * D;
     if (rank < -1 || rank >= D) return Z3_EINVAL;
     if (contrib_layout != Z3_CONTRIB_FULL && contrib_layout != Z3_CONTRIB_OWNED) return Z3_EINVAL;
     if (contrib_layout == Z3_CONTRIB_OWNED && rank < 0) return Z3_EINVAL;
@@ -381,7 +442,7 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
     if (master == nullptr || exp_avg == nullptr || exp_avg_sq == nullptr ||
         (work_bf16 == nullptr && n_gathered == 0))
         return Z3_EINVAL;
-    for (int32_t d = 0; d < D; ++d)
+    for (int32_t d = 0; d < n_contrib; ++d)
         if (contrib[d] == nullptr) return Z3_EINVAL;
     for (int32_t k = 0; k < n_gathered; ++k)
         if (gathered[k] == nullptr) return Z3_EINVAL;
@@ -390,7 +451,7 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
     if (!z3::aligned(master, 4) || !z3::aligned(exp_avg, 4) || !z3::aligned(exp_avg_sq, 4) ||
         !z3::aligned(work_bf16, 2))
         return Z3_EALIGN;
-    for (int32_t d = 0; d < D; ++d)
+    for (int32_t d = 0; d < n_contrib; ++d)
         if (!z3::aligned(contrib[d], 2)) return Z3_EALIGN;
     for (int32_t k = 0; k < n_gathered; ++k)
         if (!z3::aligned(gathered[k], 2)) return Z3_EALIGN;
@@ -412,7 +473,7 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
     for (int x = 0; x < n_out; ++x) {
         for (int y = x + 1; y < n_out; ++y)
             if (z3::overlaps(outs[x], out_bytes[x], outs[y], out_bytes[y])) return Z3_EINVAL;
-        for (int32_t d = 0; d < D; ++d)
+        for (int32_t d = 0; d < n_contrib; ++d)
             if (z3::overlaps(outs[x], out_bytes[x], contrib[d] + c_off, hb)) return Z3_EINVAL;
         if (dev_scalars != nullptr &&
             z3::overlaps(outs[x], out_bytes[x], dev_scalars, Z3_SCALARS * int64_t(sizeof(float))))
@@ -424,8 +485,9 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
     K1Args a;
     a.s = hp != nullptr ? step_scalars(hp) : AdamScalars{};
     a.s_dev = reinterpret_cast<const AdamScalars*>(dev_scalars);
-    a.inv_D = float(1.0 / double(D));
+    a.inv_n = float(1.0 / double(n_contrib));
     a.D = D;
+    a.R = R;
     a.n = n;
     a.p = master;
     a.m = exp_avg;
@@ -435,8 +497,8 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
     bool vec = z3::aligned(master, 16) && z3::aligned(exp_avg, 16) && z3::aligned(exp_avg_sq, 16) &&
                z3::aligned(work_bf16, 16);
     for (int32_t d = 0; d < Z3_D_MAX; ++d) {
-        a.c[d] = d < D ? contrib[d] + c_off : nullptr;
-        if (d < D && !z3::aligned(a.c[d], 16)) vec = false;
+        a.c[d] = d < n_contrib ? contrib[d] + c_off : nullptr;
+        if (d < n_contrib && !z3::aligned(a.c[d], 16)) vec = false;
     }
     for (int32_t k = 0; k < Z3_GATHER_MAX; ++k) {
         a.g[k] = k < n_gathered ? gathered[k] + g_off : nullptr;
@@ -445,7 +507,7 @@ int launch_k1(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, in
 
     // ---- launch: the vector kernel's grid covers the range; the scalar kernel
     // runs a whole number of resident waves with a grid-stride loop
-    const KernelFn fn = pick_any(n_gathered > 0, dev_scalars != nullptr, vec, reduce_dtype, D);
+    const KernelFn fn = pick_any(n_gathered > 0, dev_scalars != nullptr, vec, reduce_dtype, D, R);
     int64_t blocks;
     if (vec) {
         const int64_t span = int64_t(kThreads) * kChunks;
@@ -474,8 +536,18 @@ extern "C" Z3_API int zero3_reduce_adamw(const z3_plan* p, int32_t rank, const u
                                          float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
                                          const z3_adamw* hp, void* cuda_stream) {
     if (hp == nullptr) return Z3_EINVAL;
-    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, nullptr, 0,
+    return launch_k1(p, rank, 1, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, nullptr, 0,
                      reduce_dtype, hp, nullptr, cuda_stream);
+}
+
+extern "C" Z3_API int zero3_reduce_adamw_hybrid(const z3_plan* p, int32_t rank, int32_t n_nodes,
+                                                const uint16_t* const* contrib, int32_t contrib_layout,
+                                                float* master, float* exp_avg, float* exp_avg_sq,
+                                                uint16_t* work_bf16, int32_t reduce_dtype, const z3_adamw* hp,
+                                                void* cuda_stream) {
+    if (hp == nullptr || n_nodes < 1) return Z3_EINVAL;
+    return launch_k1(p, rank, n_nodes, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, nullptr,
+                     0, reduce_dtype, hp, nullptr, cuda_stream);
 }
 
 extern "C" Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
@@ -484,7 +556,7 @@ extern "C" Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, 
                                                 uint16_t* const* gathered, int32_t n_gathered,
                                                 int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream) {
     if (n_gathered < 1 || hp == nullptr) return Z3_EINVAL;
-    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
+    return launch_k1(p, rank, 1, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
                      n_gathered, reduce_dtype, hp, nullptr, cuda_stream);
 }
 
@@ -501,6 +573,6 @@ extern "C" Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, con
                                              int32_t n_gathered, int32_t reduce_dtype, const float* scalars,
                                              void* cuda_stream) {
     if (scalars == nullptr) return Z3_EINVAL;
-    return launch_k1(p, rank, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
+    return launch_k1(p, rank, 1, contrib, contrib_layout, master, exp_avg, exp_avg_sq, work_bf16, gathered,
                      n_gathered, reduce_dtype, nullptr, scalars, cuda_stream);
 }

@@ -66,6 +66,8 @@ def _load() -> C.CDLL:
     L.zero3_transient_bytes.restype = C.c_int
     L.zero3_reduce_adamw.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw.restype = C.c_int
+    L.zero3_reduce_adamw_hybrid.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
+    L.zero3_reduce_adamw_hybrid.restype = C.c_int
     L.zero3_reduce_adamw_gather.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
                                             C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw_gather.restype = C.c_int
@@ -255,6 +257,33 @@ def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], m
         rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
                                      reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw")
+
+
+def zero3_reduce_adamw_hybrid(plan: Plan, rank: int, n_nodes: int, contrib: Sequence[torch.Tensor],
+                              master: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
+                              work_bf16: torch.Tensor, hp: AdamW, contrib_layout: int = Z3_CONTRIB_FULL,
+                              reduce_dtype: int = Z3_REDUCE_FP32, stream=None) -> None:
+    """The HYBRID_SHARD step: n_nodes nodes of plan.D ranks, contrib[k * D + d] from
+    local rank d of node k; node sums, then the node sums across nodes, then
+    1/(n_nodes * D), AdamW and the bf16 cast (see include/zero3.h)."""
+    if n_nodes < 1 or n_nodes * plan.D > Z3_D_MAX:
+        raise ValueError(f"n_nodes * D must be in [1, {Z3_D_MAX}], got {n_nodes} * {plan.D}")
+    if len(contrib) != n_nodes * plan.D:
+        raise ValueError(f"need {n_nodes * plan.D} contributions, got {len(contrib)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * len(contrib))()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    mp = _dev_tensor(master, torch.float32, n, "master", host_ok=True)
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
+    wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
+    dev = _launch_device(work_bf16, master, *contrib)
+    with torch.cuda.device(dev):
+        rc = _lib.zero3_reduce_adamw_hybrid(plan.handle, rank, n_nodes, ptrs, contrib_layout, mp, ap, vp, wp,
+                                            reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
+    _check(rc, "zero3_reduce_adamw_hybrid")
 
 
 def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], master: torch.Tensor,

@@ -55,7 +55,8 @@ enum {
     Z3_EOVERFLOW = -5  /* a size does not fit in int64_t */
 };
 
-/* Largest number of simulated ranks D one call accepts. */
+/* Largest number of simulated ranks D one call accepts (with HYBRID_SHARD,
+ * the largest n_nodes * D). */
 #define Z3_D_MAX 64
 
 /* Largest number of gathered blocks zero3_reduce_adamw_gather writes in one call. */
@@ -228,6 +229,35 @@ Z3_API int zero3_reduce_adamw_gather(const z3_plan* p, int32_t rank, const uint1
                                      float* exp_avg_sq, uint16_t* work_bf16, uint16_t* const* gathered,
                                      int32_t n_gathered, int32_t reduce_dtype, const z3_adamw* hp,
                                      void* cuda_stream);
+
+/* ------------------------------------- HYBRID_SHARD: reduce + AdamW + cast
+ * zero3_reduce_adamw_hybrid: the per-rank step of HYBRID_SHARD ([P3]
+ * "HYBRID_SHARD: The Multi-Node Strategy": n_nodes nodes of D GPUs; the block
+ * is sharded D ways inside each node, as the plan describes, and replicated
+ * across the nodes; the gradient crosses nodes in one all-reduce).  The
+ * reduction has two levels:
+ *   node k's sum   n_k = c_{k,0} + c_{k,1} + ... + c_{k,D-1}  (its reduce-scatter)
+ *   total          (n_0 + n_1) + ... + n_{n_nodes-1}          (the cross-node all-reduce)
+ *   g              total * (1/(n_nodes*D))
+ * each sum left to right in the reduce dtype (every partial sum rounded to
+ * fp32 or to bf16), the factor being the fp32 constant nearest 1/(n_nodes*D):
+ * the average over every data-parallel rank, the same gradient as on one GPU
+ * ([P3] "Key Takeaways").  Steps 2 and 3 are those of zero3_reduce_adamw.  The
+ * all-reduce leaves the same sum on every node, so every node's replica of a
+ * local rank computes exactly this update; one call stands for all of them.
+ *   n_nodes  number of nodes, >= 1, with n_nodes * D <= Z3_D_MAX.  n_nodes = 1
+ *            is zero3_reduce_adamw.
+ *   contrib  host array of n_nodes * D device pointers: contrib[k*D + d] is the
+ *            bf16 contribution of local rank d on node k (global rank k*D + d),
+ *            each in `contrib_layout` as for zero3_reduce_adamw.
+ * Every other argument, the alignment rules and the state placement are those
+ * of zero3_reduce_adamw.
+ * Errors: those of zero3_reduce_adamw, plus Z3_EINVAL for n_nodes < 1 or
+ * n_nodes * D > Z3_D_MAX. */
+Z3_API int zero3_reduce_adamw_hybrid(const z3_plan* p, int32_t rank, int32_t n_nodes,
+                                     const uint16_t* const* contrib, int32_t contrib_layout, float* master,
+                                     float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
+                                     int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream);
 
 /* ------------------------------------- scalars in device memory (graphs)
  * zero3_step_scalars: the Z3_SCALARS fp32 scalars of one AdamW step, formed in

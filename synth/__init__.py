@@ -73,10 +73,16 @@ WORKLOADS = {
                            dist="student_t", zero_frac=0.01, steps=100),
     "llama70b_layer": dict(tensors=_llama70b_layer(), D=8, sigma=1e-4, dist="normal",
                            steps=10, layers=80),
+    # HYBRID_SHARD over 4 nodes of 8 GPUs on the 7B block: sharded 8 ways inside a
+    # node, replicated over the 4 nodes; 32 contributions per element
+    "llama7b_hybrid": dict(tensors=_llama7b_block(), D=8, nodes=4, sigma=1e-4, dist="normal", steps=10),
     # a 33.5M-element slice of the 7B block (two 4096 x 4096 projections) at D = 8:
     # about 1.4 GB of traffic per step, larger than L2, small enough for profiler replays
     "profile_d8": dict(tensors=[("q", (4096, 4096)), ("k", (4096, 4096))], D=8, sigma=1e-4,
                        dist="normal", steps=10),
+    # the same slice as 4 nodes of 8 ranks (HYBRID_SHARD): about 3 GB of traffic per step
+    "profile_hybrid": dict(tensors=[("q", (4096, 4096)), ("k", (4096, 4096))], D=8, nodes=4, sigma=1e-4,
+                           dist="normal", steps=10),
 }
 
 

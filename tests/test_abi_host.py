@@ -32,7 +32,8 @@ def test_library_exports_every_declared_symbol():
     names = declared_symbols()
     assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
                             "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
-                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_reduce_adamw_gather",
+                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_reduce_adamw_hybrid",
+                            "zero3_reduce_adamw_gather",
                             "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
@@ -187,6 +188,35 @@ def test_reduce_adamw_argument_errors():
     S = p.S
     base = P16 * 1000
     assert call_reduce(p, rank=1, contrib=[base] * 4, ptrs=[base + 2 * S, P16 * 20, P16 * 30, P16 * 40]) == E
+
+
+def call_hybrid(plan, n_nodes, contrib=None, rank=-1, ptrs=None, count=None):
+    n = plan.D * n_nodes if count is None else count
+    if contrib is None:
+        contrib = [P16 * (100 + d) for d in range(n)]
+    arr = (C.c_void_p * max(1, len(contrib)))(*contrib)
+    ptrs = ptrs or [P16 * 1, P16 * 2, P16 * 3, P16 * 4]
+    hp = z3.adamw(step=1)
+    return z3.lib().zero3_reduce_adamw_hybrid(plan.handle, rank, n_nodes, arr, 0, *[C.c_void_p(x) for x in ptrs],
+                                              0, C.byref(hp), None)
+
+
+def test_reduce_adamw_hybrid_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)
+    E = z3.Z3_EINVAL
+    assert call_hybrid(p, 0, contrib=[P16 * 100] * 4) == E            # at least one node
+    assert call_hybrid(p, -1, contrib=[P16 * 100] * 4) == E
+    assert call_hybrid(p, 17) == E                                    # 17 * 4 ranks > Z3_D_MAX
+    assert call_hybrid(p, 2, rank=4) == E
+    c = [P16 * (100 + d) for d in range(8)]
+    assert call_hybrid(p, 2, contrib=c[:5] + [0] + c[6:]) == E        # a NULL contribution on node 1
+    assert call_hybrid(p, 2, contrib=c[:7] + [c[7] + 1]) == z3.Z3_EALIGN
+    assert call_hybrid(p, 2, contrib=c[:6] + [P16 * 3] + c[7:]) == E  # exp_avg_sq over a node-1 contribution
+    assert z3.lib().zero3_reduce_adamw_hybrid(p.handle, -1, 2, None, 0, None, None, None, None, 0, None,
+                                              None) == E
+    e = z3.zero3_plan([], 4, 8)
+    assert call_hybrid(e, 16) == z3.Z3_OK                             # 64 contributions, empty plan
+    assert call_hybrid(e, 1) == z3.Z3_OK
 
 
 def call_fused(plan, gathered, work=P16 * 4, rank=-1, n=None):

@@ -38,6 +38,19 @@ def test_host_tensors_are_refused_where_device_memory_is_needed(plan):
                               state(128, torch.bfloat16), z3.adamw())
 
 
+def test_hybrid_node_and_contribution_counts(plan):
+    c = [state(128, torch.bfloat16)] * 4
+    args = (state(128), state(128), state(128), state(128, torch.bfloat16), z3.adamw())
+    with pytest.raises(ValueError, match="n_nodes"):
+        z3.zero3_reduce_adamw_hybrid(plan, -1, 0, c, *args)
+    with pytest.raises(ValueError, match="n_nodes"):
+        z3.zero3_reduce_adamw_hybrid(plan, -1, 33, c * 17, *args)
+    with pytest.raises(ValueError, match="need 4 contributions"):
+        z3.zero3_reduce_adamw_hybrid(plan, -1, 2, c[:3], *args)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        z3.zero3_reduce_adamw_hybrid(plan, -1, 2, c, *args)
+
+
 def test_gathered_block_count_is_bounded(plan):
     c = [state(128, torch.bfloat16)] * 2
     with pytest.raises(ValueError, match="gathered blocks"):
