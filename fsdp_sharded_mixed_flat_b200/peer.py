@@ -21,8 +21,9 @@ kernels can address the peers' memory with plain loads and stores:
 
 Every wait is a host-side stream synchronisation followed by a group barrier,
 so no kernel ever waits on another rank; the barriers take the process group's
-timeout.  No TMA, no multicast, and no library kernel is ever handed a peer's
-memory: only libzero3.so's own kernels touch the mappings.
+timeout.  The kernels reach the peers' memory with plain loads and stores only (no
+TMA), and no library kernel is ever handed a peer's memory: only libzero3.so's
+own kernels touch the mappings.
 """
 from __future__ import annotations
 
