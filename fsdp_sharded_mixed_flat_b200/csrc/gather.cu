@@ -13,12 +13,16 @@
 //     so the block scheduler balances the SMs; streaming stores.
 //   - per-tensor copy: the host cuts every tensor into segments, one per rank
 //     partition it intersects, and numbers the 16-byte units of each
-//     segment's destination.  A thread takes two destination units, finds
-//     their segments by binary search, and writes each with one 16-byte store
-//     when the unit is whole; the source run may start at any 2-byte position, so it is
-//     assembled from the two aligned 16-byte source vectors around it with
-//     funnel shifts.  Partial units at a segment's ends are written element
-//     by element.
+//     segment's destination.  A block takes a run of consecutive units; one
+//     thread finds the run's first segment by binary search and shares it
+//     through shared memory, and each thread steps forward from there to the
+//     segment of each of its two units (segments are long, so this is
+//     rarely more than one step).  A whole unit is written with one 16-byte
+//     store.  When the segment's source run is 16-byte aligned, the unit is
+//     one aligned 16-byte load; otherwise the source run may start at any
+//     2-byte position, and the unit is assembled from the two aligned 16-byte
+//     source vectors around it with funnel shifts.  Partial units at a
+//     segment's ends are written element by element.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -33,7 +37,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 2;                 // 16-byte vectors per thread in the flat copy
 constexpr int64_t kMaxBlocks = 1 << 30;   // grid.x cap; beyond it the kernels loop
-constexpr int kSegMax = 112;  // segments per launch; keeps the parameter block under 4 KB
+constexpr int kSegMax = 100;  // segments per launch; keeps the parameter block under 4 KB
 
 struct FlatArgs {
     const uint16_t* shard[Z3_D_MAX];
@@ -46,6 +50,7 @@ struct Seg {
     uint16_t* dst;        // first destination element
     int64_t len;          // elements
     int64_t unit_begin;   // index of the segment's first destination unit in this launch
+    int32_t src_aligned;  // 1: src and dst both 16-byte aligned (whole units load one aligned vector)
 };
 
 struct SegArgs {
@@ -54,6 +59,7 @@ struct SegArgs {
     int32_t vec;          // 1: sources may be read as aligned 16-byte vectors
     int64_t units;        // destination units in this launch
 };
+static_assert(sizeof(SegArgs) <= 4096, "segment table must fit the 4 KB parameter block");
 
 __global__ void __launch_bounds__(kThreads) k_gather_flat_vec(const __grid_constant__ FlatArgs a) {
     const int r = blockIdx.y;
@@ -121,23 +127,31 @@ __device__ __forceinline__ int find_segment(const SegArgs& a, int64_t u) {
 constexpr int kSegUnits = 2;
 
 __global__ void __launch_bounds__(kThreads) k_gather_segments(const __grid_constant__ SegArgs a) {
+    __shared__ int first_seg;
     const int64_t span = int64_t(kThreads) * kSegUnits;
-    for (int64_t u0 = int64_t(blockIdx.x) * span + threadIdx.x; u0 < a.units; u0 += int64_t(gridDim.x) * span) {
+    // the loop bounds are the same for every thread of the block, so the barriers are uniform
+    for (int64_t ub = int64_t(blockIdx.x) * span; ub < a.units; ub += int64_t(gridDim.x) * span) {
+        if (threadIdx.x == 0) first_seg = find_segment(a, ub);
+        __syncthreads();
+        int si = first_seg;
+        __syncthreads();  // first_seg is rewritten in the next iteration
         uint4 q[kSegUnits];
         uintptr_t dst[kSegUnits];
         bool whole[kSegUnits];
 #pragma unroll
         for (int k = 0; k < kSegUnits; ++k) {
-            const int64_t u = u0 + int64_t(k) * kThreads;
+            const int64_t u = ub + threadIdx.x + int64_t(k) * kThreads;
             whole[k] = false;
             if (u >= a.units) continue;
-            const Seg& s = a.seg[find_segment(a, u)];
+            while (si + 1 < a.nseg && a.seg[si + 1].unit_begin <= u) ++si;
+            const Seg& s = a.seg[si];
             const uintptr_t d0 = reinterpret_cast<uintptr_t>(s.dst);
             const uintptr_t unit_addr = (d0 & ~uintptr_t(15)) + uintptr_t(u - s.unit_begin) * 16u;
             // elements of this unit inside the segment: [k0, k1) relative to s.dst
             const int64_t k_first = (int64_t(unit_addr) - int64_t(d0)) / 2;  // may be negative
             if (a.vec && k_first >= 0 && k_first + 8 <= s.len) {
-                q[k] = load8_unaligned(s.src + k_first);
+                q[k] = s.src_aligned ? *reinterpret_cast<const uint4*>(s.src + k_first)
+                                     : load8_unaligned(s.src + k_first);
                 dst[k] = unit_addr;
                 whole[k] = true;
             } else {
@@ -228,7 +242,9 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
             for (int64_t r = b / S; r < D && r * S < e; ++r) {
                 const int64_t lo = std::max(b, r * S), hi = std::min(e, (r + 1) * S);
                 if (hi <= lo) continue;
-                segs.push_back(Seg{shards[r] + (lo - r * S), tensor_out[i] + (lo - b), hi - lo, 0});
+                Seg g{shards[r] + (lo - r * S), tensor_out[i] + (lo - b), hi - lo, 0, 0};
+                g.src_aligned = z3::aligned(g.src, 16) && z3::aligned(g.dst, 16) ? 1 : 0;
+                segs.push_back(g);
             }
         }
         for (size_t first = 0; first < segs.size(); first += kSegMax) {
