@@ -126,6 +126,7 @@ class Plan:
         h = C.c_void_p()
         _check(_lib.zero3_plan(specs, n, D, align_elems, C.byref(h)), "zero3_plan")
         self._h = h
+        self._free = _lib.zero3_plan_free   # held here: module globals may be gone when __del__ runs at exit
         d, nt, a = C.c_int32(), C.c_int32(), C.c_int32()
         N, N_pad, S = C.c_int64(), C.c_int64(), C.c_int64()
         _check(_lib.zero3_plan_info(h, C.byref(d), C.byref(nt), C.byref(a), C.byref(N),
@@ -162,9 +163,9 @@ class Plan:
         return [flat[o:o + k].view(s) for o, k, s in zip(self.offsets, self.numels, self.shapes)]
 
     def __del__(self):
-        h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            _lib.zero3_plan_free(h)
+        h, free = getattr(self, "_h", None), getattr(self, "_free", None)
+        if h is not None and h.value and free is not None:
+            free(h)
             self._h = None
 
 

@@ -80,3 +80,17 @@ def test_plan_views_and_lazy_offsets(plan):
     assert (again.N, again.N_pad, again.S, again.offsets) == (plan.N, plan.N_pad, plan.S, plan.offsets)
     with pytest.raises(ValueError):
         z3.tensor_specs([(1, 2, 3, 4, 5)])
+
+
+def test_plan_alive_at_interpreter_exit_is_freed_quietly():
+    """A plan still referenced when the interpreter exits is freed without errors
+    (module globals may already be cleared when its finaliser runs)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys; sys.path.insert(0, %r)\n"
+            "from fsdp_sharded_mixed_flat_b200 import zero3 as z3\n"
+            "keep = z3.zero3_plan([(10,), (3, 4)], 2, 8)\n") % root
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "Error" not in r.stderr and "Exception" not in r.stderr, r.stderr
