@@ -87,8 +87,9 @@ def test_streamed_layers_with_a_fill_refill(z3):
 
 def test_llama70b_rank_shard_80_layers_sampled(z3):
     """The full resident shard of one rank (8.556B owned params, about 120 GB with
-    the bf16 shard), one streamed step over all 80 layers; the oracle checks a
-    sample of every layer and the whole of layers 79 and 0."""
+    the bf16 shard), one streamed step over all 80 layers; the oracle checks
+    every element of layers 79, 40 and 0 and a seeded 2^20-element subset of
+    every other layer (master, moments and bf16 weights)."""
     from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
     w_ = synth.WORKLOADS["llama70b_layer"]
     L, D, rank = w_["layers"], w_["D"], 5
@@ -107,9 +108,10 @@ def test_llama70b_rank_shard_80_layers_sampled(z3):
     pool = [owned_contribs(D, S, S, 77, 1, k, sigma=1e-4) for k in range(2)]
     st = LayerStreamer(plan, L, rank, master, m, v, w)
     rng = np.random.default_rng(0)
-    idx = torch.from_numpy(np.unique(rng.choice(S, 20_000, replace=False))).cuda()
-    before = {l: f32_host(master[l * S:(l + 1) * S][idx]) for l in range(L)}
-    full_before = {l: f32_host(master[l * S:(l + 1) * S]) for l in (0, L - 1)}
+    idx = torch.from_numpy(np.unique(rng.choice(S, 1 << 20, replace=False))).cuda()
+    full_layers = (0, L // 2, L - 1)
+    before = {l: f32_host(master[l * S:(l + 1) * S][idx]) for l in range(L) if l not in full_layers}
+    full_before = {l: f32_host(master[l * S:(l + 1) * S]) for l in full_layers}
     st.step(lambda l: pool[l % 2], z3.adamw(**hp_for(1)))
     torch.cuda.synchronize()
     hosts = [synth.bf16_bits(p) for p in pool]
@@ -125,11 +127,14 @@ def test_llama70b_rank_shard_80_layers_sampled(z3):
             p_l = before[l].copy()
             got = master[l * S:(l + 1) * S][idx]
             got_w = w[l * S:(l + 1) * S][idx]
+            got_m = m[l * S:(l + 1) * S][idx]
+            got_v = v[l * S:(l + 1) * S][idx]
         m_l, v_l, w_l = np.zeros(sel.size, np.float32), np.zeros(sel.size, np.float32), np.zeros(sel.size, np.uint16)
         oracle.reduce_adamw([np.ascontiguousarray(c[d * S:(d + 1) * S][sel]) for d in range(D)], sel.size, 0,
                             p_l, m_l, v_l, w_l, oracle_hp(1), layout=oracle.LAYOUT_OWNED)
         assert_f32_parity(f32_host(got), p_l, f"master layer {l}")
         assert_bf16_parity(synth.bf16_bits(got_w), w_l, f"work layer {l}")
         if l in full_before:
-            assert_f32_parity(f32_host(m[l * S:(l + 1) * S]), m_l, f"exp_avg layer {l}")
-            assert_f32_parity(f32_host(v[l * S:(l + 1) * S]), v_l, f"exp_avg_sq layer {l}")
+            got_m, got_v = m[l * S:(l + 1) * S], v[l * S:(l + 1) * S]
+        assert_f32_parity(f32_host(got_m), m_l, f"exp_avg layer {l}")
+        assert_f32_parity(f32_host(got_v), v_l, f"exp_avg_sq layer {l}")
