@@ -91,6 +91,15 @@ def host_info() -> dict:
     return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
+def ledger(z3, N: int, N_pad: int, D: int, block_params: int) -> dict:
+    """The memory ledger (bytes per device, per stage) for N real and N_pad padded
+    parameters over D ranks, and the transient bytes of two gathered blocks."""
+    stages = {"ddp": 0, "zero1": 1, "zero2": 2, "zero3": 3}
+    return {"N": {k: z3.zero3_memory_bytes(N, D, v) for k, v in stages.items()},
+            "N_pad": {k: z3.zero3_memory_bytes(N_pad, D, v) for k, v in stages.items()},
+            "transient_2_blocks": z3.zero3_transient_bytes(block_params, 2)}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -300,6 +309,7 @@ class BlockRunner:
         self.tensor_out = ([torch.empty(shape, dtype=torch.bfloat16, device=dev) for shape in self.shapes]
                            if unflatten_copy and stage == 3 else None)
         self.units_per_step = self.N_pad                       # owned params, all ranks
+        self.ledger_args = (self.N, self.N_pad, D, self.N_pad)
         self.k1_launches_per_step = 1
         # stage 1/2: the bf16 goes to the block instead of the shard; same bytes
         self.k1_bytes_per_launch = (2 * self.nodes * D + 26) * self.N_pad
@@ -466,6 +476,7 @@ class ShardRunner:
         self.stream = torch.cuda.current_stream(dev)
         self.step_no = 0
         self.units_per_step = L * S                            # owned params of this rank
+        self.ledger_args = (L * plan.N, L * plan.N_pad, D, plan.N_pad)
         self.k1_launches_per_step = L
         self.k1_bytes_per_launch = (2 * D + 26) * S
         self.refill = refill
@@ -643,6 +654,7 @@ def run_ours(args):
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": R.launches_per_step * args.steps,
+        "ledger_bytes_per_device": ledger(z3, *R.ledger_args),
     }
     line.update(extra)
     if getattr(R, "offload", False):
