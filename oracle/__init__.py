@@ -69,6 +69,8 @@ def _bind(L):
     L.ref_memory_bytes.restype = C.c_double
     L.ref_transient_bytes.argtypes = [C.c_double, i32]
     L.ref_transient_bytes.restype = C.c_double
+    L.ref_allgather_bytes.argtypes = [C.c_double, i32, i32]
+    L.ref_allgather_bytes.restype = C.c_double
     L.ref_reduce_scatter.argtypes = [i32, i64, i32, p, i32, i32, p]
     L.ref_reduce_scatter.restype = C.c_int
     L.ref_adamw_consts_of.argtypes = [C.POINTER(AdamWHP), p]
@@ -153,6 +155,10 @@ def memory_bytes(N: float, D: float, stage: int) -> float:
 
 def transient_bytes(block_params: float, n_buffers: int = 1) -> float:
     return lib().ref_transient_bytes(float(block_params), n_buffers)
+
+
+def allgather_bytes(block_bytes: float, n_blocks: int, D: int) -> float:
+    return lib().ref_allgather_bytes(float(block_bytes), n_blocks, D)
 
 
 # ----------------------------------------------------------- reduce and AdamW

@@ -28,7 +28,8 @@
  *         Production Python Snippet (the MixedPrecision policy).
  *   [P2] "7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)", §2 Recap: DP
  *         memory in three buckets, §3 ZeRO-1, §4 ZeRO-2, §5.1 Forward and
- *         backward pass under FSDP, §5.2 Memory accounting.
+ *         backward pass under FSDP, §5.2 Memory accounting, §5.3 Extra
+ *         communication.
  *   [P3] "Building GPT from Scratch — Part 8: FSDP — When the Model Won't
  *         Fit", sections "AllGather vs AllReduce", "Mixed Precision:
  *         Cutting Memory in Half", "HYBRID_SHARD: The Multi-Node Strategy"
@@ -154,6 +155,14 @@ double ref_memory_bytes(double N, double D, int32_t stage)
 double ref_transient_bytes(double block_params, int32_t n_buffers)
 {
     return (double)n_buffers * block_params * 2.0;
+}
+
+/* [P2] §5.3: every pass gathers each block once; a device already holds its
+ * own 1/D of the block and receives the other (D-1)/D.  Bytes received per
+ * device for n_blocks blocks of block_bytes each. */
+double ref_allgather_bytes(double block_bytes, int32_t n_blocks, int32_t D)
+{
+    return (double)n_blocks * block_bytes * (double)(D - 1) / (double)D;
 }
 
 /* ------------------------------------------------------------------------ */

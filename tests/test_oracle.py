@@ -148,6 +148,20 @@ def test_transient_and_steady_state_golden(golden):
     assert got == pytest.approx(s["GB"], rel=s["rel_tol"])
 
 
+def test_allgather_volume_golden(golden):
+    """Pin: page 2 §5.3's forward and backward all-gather volume per device
+    (each block gathered once per pass; a device receives the (D-1)/D it does
+    not own), and the cases the formula fixes exactly."""
+    a = golden("memory_figures.json")["allgather"]
+    got = oracle.allgather_bytes(a["block_MB"] * 1e6, a["L"], a["D"]) / 1e9
+    assert got == pytest.approx(a["forward_GB"], rel=a["rel_tol"])
+    assert got == pytest.approx(a["backward_GB"], rel=a["rel_tol"])
+    assert oracle.allgather_bytes(123456.0, 7, 1) == 0.0            # one rank holds everything
+    for block, L, D in [(1000, 3, 2), (4096, 5, 8), (999, 1, 3)]:
+        exact = Fraction(L) * block * (D - 1) / D
+        assert oracle.allgather_bytes(block, L, D) == pytest.approx(float(exact), rel=1e-15)
+
+
 # ----------------------------------------------------------------- reduction
 def test_reduce_scatter_worked_example(golden):
     """Pin: page 3's 4-GPU reduce-scatter: GPU x gets the sum of slice x."""

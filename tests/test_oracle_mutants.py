@@ -46,6 +46,9 @@ MUTANTS = [
      "case 1: return optim * N / D + weights * N;"),
     ("the unflatten starts one element late", "out[t][k] = flat[offset[t] + k];",
      "out[t][k] = flat[offset[t] + k + (k + 1 < numel[t] ? 1 : 0)];"),
+    ("the all-gather counts the device's own shard as received",
+     "return (double)n_blocks * block_bytes * (double)(D - 1) / (double)D;",
+     "return (double)n_blocks * block_bytes * (double)(D) / (double)D;"),
     ("HYBRID_SHARD folds all ranks flat, ignoring the nodes",
      "float node_sum = ref_f32_from_bf16(node[0][idx]);",
      "float node_sum = k == 0 ? ref_f32_from_bf16(node[0][idx]) : total + ref_f32_from_bf16(node[0][idx]);"
@@ -102,6 +105,7 @@ PINS = [
     lambda: pins.test_plan_workloads_golden(golden),
     lambda: pins.test_memory_figures_golden(golden),
     lambda: pins.test_transient_and_steady_state_golden(golden),
+    lambda: pins.test_allgather_volume_golden(golden),
     lambda: pins.test_adamw_step1_closed_form(),
     lambda: pins.test_adamw_zero_gradient_keeps_zero_pad(),
     lambda: pins.test_reduce_fp32_matches_torch_left_fold(8),
