@@ -93,11 +93,14 @@ def host_info() -> dict:
 
 def ledger(z3, N: int, N_pad: int, D: int, block_params: int) -> dict:
     """The memory ledger (bytes per device, per stage) for N real and N_pad padded
-    parameters over D ranks, and the transient bytes of two gathered blocks."""
+    parameters over D ranks, the transient bytes of two gathered blocks, and the
+    bytes one device receives in the all-gathers of one pass over the blocks."""
     stages = {"ddp": 0, "zero1": 1, "zero2": 2, "zero3": 3}
+    n_blocks = N_pad // block_params if block_params else 0
     return {"N": {k: z3.zero3_memory_bytes(N, D, v) for k, v in stages.items()},
             "N_pad": {k: z3.zero3_memory_bytes(N_pad, D, v) for k, v in stages.items()},
-            "transient_2_blocks": z3.zero3_transient_bytes(block_params, 2)}
+            "transient_2_blocks": z3.zero3_transient_bytes(block_params, 2),
+            "allgather_per_pass": z3.zero3_allgather_bytes(block_params, n_blocks, D)}
 
 
 def measured_peaks():

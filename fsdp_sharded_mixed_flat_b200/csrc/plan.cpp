@@ -150,4 +150,14 @@ Z3_API int zero3_transient_bytes(int64_t block_params, int32_t n_buffers, int64_
     return Z3_OK;
 }
 
+Z3_API int zero3_allgather_bytes(int64_t block_params, int32_t n_blocks, int32_t D, int64_t* bytes) {
+    if (bytes == nullptr || block_params < 0 || n_blocks < 0 || D < 1) return Z3_EINVAL;
+    const int64_t one = mul_checked(2, block_params);            // one block in bf16
+    const int64_t all = one < 0 ? -1 : mul_checked(one, n_blocks);
+    if (all < 0) return Z3_EOVERFLOW;
+    // all * (D - 1) / D rounded up, which is exactly all - floor(all / D)
+    *bytes = all - all / D;
+    return Z3_OK;
+}
+
 }  // extern "C"

@@ -64,6 +64,8 @@ def _load() -> C.CDLL:
     L.zero3_memory_bytes.restype = C.c_int
     L.zero3_transient_bytes.argtypes = [i64, i32, C.POINTER(i64)]
     L.zero3_transient_bytes.restype = C.c_int
+    L.zero3_allgather_bytes.argtypes = [i64, i32, i32, C.POINTER(i64)]
+    L.zero3_allgather_bytes.restype = C.c_int
     L.zero3_reduce_adamw.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw.restype = C.c_int
     L.zero3_reduce_adamw_hybrid.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
@@ -194,6 +196,12 @@ def zero3_memory_bytes(N: int, D: int, stage: int) -> int:
 def zero3_transient_bytes(block_params: int, n_buffers: int = 1) -> int:
     out = C.c_int64()
     _check(_lib.zero3_transient_bytes(block_params, n_buffers, C.byref(out)), "zero3_transient_bytes")
+    return out.value
+
+
+def zero3_allgather_bytes(block_params: int, n_blocks: int, D: int) -> int:
+    out = C.c_int64()
+    _check(_lib.zero3_allgather_bytes(block_params, n_blocks, D, C.byref(out)), "zero3_allgather_bytes")
     return out.value
 
 

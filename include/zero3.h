@@ -157,6 +157,14 @@ Z3_API int zero3_memory_bytes(int64_t N, int32_t D, int32_t stage, int64_t* byte
  * Errors: Z3_EINVAL (negative argument, bytes NULL), Z3_EOVERFLOW. */
 Z3_API int zero3_transient_bytes(int64_t block_params, int32_t n_buffers, int64_t* bytes);
 
+/* All-gather volume ([P2] §5.3): each pass (forward, and again backward)
+ * gathers every block once; a device already holds its own 1/D of a block
+ * and receives the other (D-1)/D.  *bytes = the bf16 bytes one device
+ * receives for n_blocks blocks of block_params parameters each,
+ * ceil(n_blocks * 2 * block_params * (D-1) / D).  D = 1 gives 0.
+ * Errors: Z3_EINVAL (negative argument, D < 1, bytes NULL), Z3_EOVERFLOW. */
+Z3_API int zero3_allgather_bytes(int64_t block_params, int32_t n_blocks, int32_t D, int64_t* bytes);
+
 /* ------------------------------------------- reduce-scatter + AdamW + cast
  * zero3_reduce_adamw: one fused pass over the owned partition(s):
  *   1. reduce-scatter's reduction ([P3] "AllGather vs AllReduce": rank r

@@ -124,6 +124,11 @@ static void check_ledger(void)
     CHECK(zero3_memory_bytes(N, 32, 4, &bytes) == Z3_EINVAL);
     CHECK(zero3_memory_bytes(-1, 32, 3, &bytes) == Z3_EINVAL);
     CHECK(zero3_memory_bytes(N, 32, 3, NULL) == Z3_EINVAL);
+    /* all-gather volume: 32 blocks of 100M bf16 parameters (200 MB) at D = 32 receive 31/32 of each */
+    CHECK(zero3_allgather_bytes(100000000LL, 32, 32, &bytes) == Z3_OK && bytes == 6200000000LL);
+    CHECK(zero3_allgather_bytes(7, 1, 3, &bytes) == Z3_OK && bytes == 10);   /* ceil(14 * 2 / 3) */
+    CHECK(zero3_allgather_bytes(7, 1, 1, &bytes) == Z3_OK && bytes == 0);
+    CHECK(zero3_allgather_bytes(7, 1, 0, &bytes) == Z3_EINVAL);
     /* one 12 x 4096^2 block in bf16, two buffers live (next block's gather overlapping) */
     CHECK(zero3_transient_bytes(12LL * 4096 * 4096, 2, &bytes) == Z3_OK && bytes == 4LL * 12 * 4096 * 4096);
 }

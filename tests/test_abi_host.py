@@ -32,7 +32,8 @@ def test_library_exports_every_declared_symbol():
     names = declared_symbols()
     assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
                             "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
-                            "zero3_transient_bytes", "zero3_reduce_adamw", "zero3_reduce_adamw_hybrid",
+                            "zero3_transient_bytes", "zero3_allgather_bytes", "zero3_reduce_adamw",
+                            "zero3_reduce_adamw_hybrid",
                             "zero3_reduce_adamw_gather",
                             "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
@@ -144,6 +145,26 @@ def test_transient_bytes_matches_oracle():
     for block in (0, 1, 12 * 4096 * 4096, 855_654_400):
         for nb in (0, 1, 2):
             assert z3.zero3_transient_bytes(block, nb) == oracle.transient_bytes(block, nb)
+
+
+def test_allgather_bytes_matches_oracle():
+    """The ABI's integer all-gather volume is the oracle's, rounded up to a byte."""
+    for block in (0, 1, 3, 12 * 4096 * 4096, 855_654_400, 100_000_000):
+        for nb in (0, 1, 32, 80):
+            for D in (1, 2, 3, 8, 32, 64):
+                ref = oracle.allgather_bytes(2.0 * block, nb, D)
+                got = z3.zero3_allgather_bytes(block, nb, D)
+                exact_num = nb * 2 * block * (D - 1)          # the exact value is exact_num / D
+                assert got == -(-exact_num // D), (block, nb, D)
+                assert abs(got - ref) <= 1.0 + 1e-12 * ref
+    # the page's figure: 32 blocks of 200 MB (100M bf16 parameters) at D = 32
+    assert z3.zero3_allgather_bytes(100_000_000, 32, 32) == 6_200_000_000
+    with pytest.raises(z3.Zero3Error) as e:
+        z3.zero3_allgather_bytes(1, 1, 0)
+    assert e.value.status == z3.Z3_EINVAL
+    with pytest.raises(z3.Zero3Error) as e:
+        z3.zero3_allgather_bytes(2 ** 62, 2, 2)
+    assert e.value.status == z3.Z3_EOVERFLOW
 
 
 # ------------------------------------------- argument errors, no device work
