@@ -216,7 +216,7 @@ def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str, host_
     so the kernel reaches it over PCIe)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda" and not (host_ok and t.device.type == "cpu" and t.is_pinned()):
+    if not t.is_cuda and not (host_ok and t.device.type == "cpu" and t.is_pinned()):
         raise ValueError(f"{name} must be a CUDA tensor" + (" or a pinned host tensor" if host_ok else ""))
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
@@ -227,14 +227,23 @@ def _dev_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str, host_
     return t.data_ptr()
 
 
-def _launch_device(*candidates):
+def _launch_device(*candidates) -> int:
     """The device the kernels launch on: that of the first local CUDA tensor given
     (the state and outputs come first; contributions and shards may be mapped
     from peer GPUs)."""
     for t in candidates:
-        if isinstance(t, torch.Tensor) and t.device.type == "cuda":
-            return t.device
+        if isinstance(t, torch.Tensor) and t.is_cuda:
+            return t.get_device()
     raise ValueError("no CUDA tensor among the arguments")
+
+
+def _call_on(dev: int, fn, *args) -> int:
+    """fn(*args) with `dev` as the current CUDA device (the library launches on the
+    current device); the device switch is skipped when it is current already."""
+    if torch.cuda.current_device() == dev:
+        return fn(*args)
+    with torch.cuda.device(dev):
+        return fn(*args)
 
 
 def _stream_handle(stream, device) -> int:
@@ -262,9 +271,8 @@ def zero3_reduce_adamw(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], m
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
     dev = _launch_device(work_bf16, master, *contrib)
-    with torch.cuda.device(dev):
-        rc = _lib.zero3_reduce_adamw(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
-                                     reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
+    rc = _call_on(dev, _lib.zero3_reduce_adamw, plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
+                  reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw")
 
 
@@ -289,9 +297,8 @@ def zero3_reduce_adamw_hybrid(plan: Plan, rank: int, n_nodes: int, contrib: Sequ
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
     dev = _launch_device(work_bf16, master, *contrib)
-    with torch.cuda.device(dev):
-        rc = _lib.zero3_reduce_adamw_hybrid(plan.handle, rank, n_nodes, ptrs, contrib_layout, mp, ap, vp, wp,
-                                            reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
+    rc = _call_on(dev, _lib.zero3_reduce_adamw_hybrid, plan.handle, rank, n_nodes, ptrs, contrib_layout, mp, ap,
+                  vp, wp, reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw_hybrid")
 
 
@@ -319,10 +326,8 @@ def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Ten
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
     dev = _launch_device(work_bf16, master, *contrib)
-    with torch.cuda.device(dev):
-        rc = _lib.zero3_reduce_adamw_gather(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp, gp,
-                                            len(gathered), reduce_dtype, C.byref(hp),
-                                            _stream_handle(stream, dev))
+    rc = _call_on(dev, _lib.zero3_reduce_adamw_gather, plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
+                  gp, len(gathered), reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw_gather")
 
 
@@ -364,10 +369,8 @@ def zero3_reduce_adamw_dev(plan: Plan, rank: int, contrib: Sequence[torch.Tensor
     vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
     wp = None if work_bf16 is None else _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
     dev = _launch_device(scalars, work_bf16, master, *contrib)
-    with torch.cuda.device(dev):
-        rc = _lib.zero3_reduce_adamw_dev(plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
-                                         gp if gathered else None, len(gathered), reduce_dtype, sp,
-                                         _stream_handle(stream, dev))
+    rc = _call_on(dev, _lib.zero3_reduce_adamw_dev, plan.handle, rank, ptrs, contrib_layout, mp, ap, vp, wp,
+                  gp if gathered else None, len(gathered), reduce_dtype, sp, _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw_dev")
 
 
@@ -388,6 +391,5 @@ def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Opt
         for i, t in enumerate(tensor_out):
             tp[i] = None if t is None else _dev_tensor(t, torch.bfloat16, plan.numels[i], f"tensor_out[{i}]")
     dev = _launch_device(flat_out, *(tensor_out or []), *shards)
-    with torch.cuda.device(dev):
-        rc = _lib.zero3_gather_block(plan.handle, sp, fp, tp, _stream_handle(stream, dev))
+    rc = _call_on(dev, _lib.zero3_gather_block, plan.handle, sp, fp, tp, _stream_handle(stream, dev))
     _check(rc, "zero3_gather_block")
