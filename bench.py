@@ -55,7 +55,8 @@ def parse_args():
     ap.add_argument("--workload", default="llama7b_d8")
     ap.add_argument("--e2e-steps", type=int, default=12)
     ap.add_argument("--cpu-sample", type=int, default=1 << 24, help="elements of the oracle's sample")
-    ap.add_argument("--cpu-steps", type=int, default=20)
+    ap.add_argument("--cpu-steps", type=int, default=20,
+                    help="most oracle steps in the CPU baseline; fewer when a step takes long (about 10 s in all)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
@@ -209,16 +210,22 @@ def aggregate(local_seconds: float, local_units: float, world: int, device=None)
 
 
 # --------------------------------------------------------------- the oracle
-def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int = 0, reduce_dtype: int = 0):
+def oracle_workload(workload: str) -> str:
+    """The workload whose elements the oracle samples (the 70B shard's are its layers')."""
+    return "llama70b_layer" if workload == "llama70b_shard" else workload
+
+
+def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int = 0, reduce_dtype: int = 0,
+                  keep: bool = False):
     """Time the oracle over `steps` passes of a `sample`-element slice of the
     workload's owned elements (all D contributions, AdamW, cast).  Returns
-    (owned params/s, seconds, description)."""
+    (owned params/s, seconds, description, kept), where kept holds the sample's
+    inputs and the oracle's final state when `keep` is set (else None)."""
     import numpy as np
 
     import oracle
     import synth
-    if workload == "llama70b_shard":
-        workload = "llama70b_layer"
+    workload = oracle_workload(workload)
     w = synth.WORKLOADS[workload]
     D = D or w["D"]
     nodes = w.get("nodes", 1)
@@ -227,6 +234,7 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
                                                    dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
                                                    device="cpu")) for d in range(nodes * D)]
     p = synth.master_weights(n, n, seed=seed).numpy().copy()
+    p0 = p.copy() if keep else None
     m, v, wk = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
     oracle.lib()
     t0 = time.perf_counter()
@@ -242,7 +250,52 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
     desc = (f"{workload}: first {n} owned elements x {steps} steps, {shape}, "
             f"{'bf16' if reduce_dtype else 'fp32'} reduce, one thread "
             f"(oracle/zero3_ref.c, single-threaded C)")
-    return n * steps / dt, dt, desc
+    kept = dict(contribs=contribs, p0=p0, p=p, m=m, v=v, wk=wk, n=n, D=D, nodes=nodes, steps=steps) if keep else None
+    return n * steps / dt, dt, desc, kept
+
+
+def sample_parity(z3, dev, kept: dict, reduce_dtype: int) -> dict:
+    """Our path, through the public API on the GPU, over the CPU baseline's own
+    sample (the same contributions, master and steps, as rank 0's owned slice),
+    compared element by element with the oracle's results."""
+    import numpy as np
+    import torch
+
+    import synth
+    n, D, nodes, steps = kept["n"], kept["D"], kept["nodes"], kept["steps"]
+    plan = z3.zero3_plan([(n * D,)], D, 1)                     # S = n
+    c = [synth.bits_to_bf16(x, dev) for x in kept["contribs"]]
+    p = torch.from_numpy(kept["p0"]).to(dev)
+    m, v = torch.zeros_like(p), torch.zeros_like(p)
+    w = torch.zeros(n, dtype=torch.bfloat16, device=dev)
+    for t in range(1, steps + 1):
+        hp = z3.adamw(step=t)
+        if nodes > 1:
+            z3.zero3_reduce_adamw_hybrid(plan, 0, nodes, c, p, m, v, w, hp, contrib_layout=z3.Z3_CONTRIB_OWNED,
+                                         reduce_dtype=reduce_dtype)
+        else:
+            z3.zero3_reduce_adamw(plan, 0, c, p, m, v, w, hp, contrib_layout=z3.Z3_CONTRIB_OWNED,
+                                  reduce_dtype=reduce_dtype)
+    torch.cuda.synchronize(dev)
+
+    def rel(got, ref):
+        return float(np.max(np.abs(got.astype(np.float64) - ref) /
+                            np.maximum(np.abs(ref.astype(np.float64)), np.finfo(np.float32).tiny)))
+
+    def ulps(a, b):
+        def ordered(x):
+            x = x.astype(np.int32)
+            return np.where(x & 0x8000, 0x8000 - (x & 0x7FFF), 0x8000 + (x & 0x7FFF))
+        return int(np.max(np.abs(ordered(a) - ordered(b))))
+
+    got = [t.cpu().numpy() for t in (p, m, v)]
+    refs = [kept["p"], kept["m"], kept["v"]]
+    gw = synth.bf16_bits(w)
+    exact = all(np.array_equal(g.view(np.uint32), r.view(np.uint32)) for g, r in zip(got, refs)) and \
+        np.array_equal(gw, kept["wk"])
+    return {"elements": n, "steps": steps, "master_max_rel": rel(got[0], refs[0]),
+            "exp_avg_max_rel": rel(got[1], refs[1]), "exp_avg_sq_max_rel": rel(got[2], refs[2]),
+            "work_bf16_max_ulp": ulps(gw, kept["wk"]), "bit_exact": bool(exact)}
 
 
 def run_reference(args):
@@ -255,7 +308,7 @@ def run_reference(args):
     mode = 1 if args.reduce_dtype == "bf16" else 0
     if args.warmup > 0:
         oracle_sample(args.workload, min(sample, 1 << 16), 1, D=args.D, reduce_dtype=mode)
-    value, secs, desc = oracle_sample(args.workload, sample, steps, D=args.D, reduce_dtype=mode)
+    value, secs, desc, _ = oracle_sample(args.workload, sample, steps, D=args.D, reduce_dtype=mode)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
@@ -669,10 +722,16 @@ def run_ours(args):
                                    "on the staged device buffers only"}
         line["roofline"]["traffic"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, secs_cpu, desc = oracle_sample(args.workload, args.cpu_sample, args.cpu_steps, D=R.D, reduce_dtype=mode)
+        # calibrate on a small slice, then size the step count for about 10 s of oracle work
+        rate, _, _, _ = oracle_sample(args.workload, 1 << 16, 1, D=R.D, reduce_dtype=mode)
+        n_cpu = min(args.cpu_sample, synth.block_numel(synth.WORKLOADS[oracle_workload(args.workload)]["tensors"]))
+        cpu_steps = max(1, min(args.cpu_steps, round(10.0 * rate / max(1, n_cpu))))
+        v, secs_cpu, desc, kept = oracle_sample(args.workload, args.cpu_sample, cpu_steps, D=R.D,
+                                                reduce_dtype=mode, keep=True)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                 "host": host_info(),
-                                "seconds": secs_cpu}
+                                "seconds": secs_cpu,
+                                "parity_vs_oracle": sample_parity(z3, dev, kept, mode)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
