@@ -18,6 +18,17 @@ stream, max over ranks.  Each step streams about 9.3 GB through HBM, far more
 than the 126 MB L2, so no flush is needed between steps.  The fused kernel is
 also timed launch by launch with its own events for the roofline figure.
 
+Workloads (--workload): llama7b_d8 (default), llama7b_d32, llama7b_policy (with
+--D), llama7b_hybrid (HYBRID_SHARD, 4 nodes of 8), llama70b_shard (one rank's
+80-layer shard, streamed), tiny_gpt, and the small profiling slices
+profile_d8 and profile_hybrid.
+
+Besides the throughput, the line carries the roofline of the fused kernel, the
+SM clocks seen during the timed region, an end-to-end figure through the public
+API from pinned host buffers, the memory ledger, and (N = 1, rank 0) the CPU
+baseline: the oracle timed on one host core on a bounded sample, with our path
+checked against it on that same sample (parity_vs_oracle).
+
 --impl reference times the oracle (plain single-threaded C) on the host on a
 bounded sample of the same workload; it is a deliberately slow baseline.
 """
