@@ -311,6 +311,41 @@ def test_adamw_ten_steps_matches_torch_adamw_float64():
     np.testing.assert_allclose(p, rp, rtol=1e-6, atol=1e-6 * np.abs(rp).max())
 
 
+@pytest.mark.parametrize("lr,b1,b2,eps,wd,t0", [
+    (1e-3, 0.0, 0.999, 1e-8, 0.0, 1),       # no momentum, no decay
+    (1e-2, 0.95, 0.99, 1e-3, 0.3, 1),      # a large eps: its place in the denominator shows
+    (5e-5, 0.5, 0.5, 1e-6, 0.01, 1),
+    (3e-4, 0.9, 0.95, 1e-8, 0.1, 990),     # late steps: the bias corrections are nearly 1
+])
+def test_adamw_hyperparameters_match_torch_adamw_float64(lr, b1, b2, eps, wd, t0):
+    """Pin: with t0 = 1, ten fp32 steps track torch.optim.AdamW run in float64
+    across the hyper-parameters.  torch always counts steps from 1, so a late
+    step (t0 > 1) is checked instead as one step from zero moments against the
+    closed form in float64, where the bias corrections are nearly 1."""
+    rng = np.random.default_rng(int(lr * 1e6) + t0)
+    n = 3000
+    p0 = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    grads = [(rng.standard_normal(n) * 1e-3).astype(np.float32) for _ in range(10)]
+    if t0 == 1:
+        p, m, v = p0.copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+        for t, g in enumerate(grads, 1):
+            oracle.adamw(g, p, m, v, oracle.hp(lr, b1, b2, eps, wd, t))
+        rp, rm, rv = torch_adamw64(p0, grads, lr, b1, b2, eps, wd)
+        np.testing.assert_allclose(m, rm, rtol=2e-6, atol=1e-6 * np.abs(rm).max())
+        np.testing.assert_allclose(v, rv, rtol=2e-6, atol=1e-6 * np.abs(rv).max())
+        np.testing.assert_allclose(p, rp, rtol=1e-6, atol=1e-6 * np.abs(rp).max())
+    else:
+        # one step at t0 from zero moments, against the closed form in float64
+        g = grads[0].astype(np.float64)
+        p, m, v = p0.copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+        oracle.adamw(grads[0], p, m, v, oracle.hp(lr, b1, b2, eps, wd, t0))
+        m64, v64 = (1 - b1) * g, (1 - b2) * g * g
+        step = lr / (1 - b1 ** t0)
+        denom = np.sqrt(v64) / np.sqrt(1 - b2 ** t0) + eps
+        p64 = p0.astype(np.float64) * (1 - lr * wd) - step * m64 / denom
+        np.testing.assert_allclose(p, p64, rtol=1e-6, atol=1e-6 * np.abs(p64).max())
+
+
 def test_adamw_detects_coupled_decay_and_missing_bias_correction():
     """The torch pin separates the plausible wrong variants of AdamW."""
     rng = np.random.default_rng(12)
