@@ -448,3 +448,34 @@ def test_single_launch_beyond_2_31_elements(z3):
     assert not p[N:].any() and not w[N:].view(torch.int16).any()
     del p, m, v, w, flat
     torch.cuda.empty_cache()
+
+
+def test_random_hyperparameters_match_oracle(z3):
+    """Bit-exact parity across AdamW hyper-parameters (momentum off, large eps,
+    large learning rate, no decay, late steps) and both reduce dtypes."""
+    import random
+    rnd = random.Random(99)
+    plan = z3.zero3_plan([(30000,), (4097,)], 4, 8)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    for case in range(12):
+        a = dict(lr=10 ** rnd.uniform(-5, -1.5), beta1=rnd.choice([0.0, 0.5, 0.9, 0.99]),
+                 beta2=rnd.choice([0.5, 0.95, 0.999]), eps=10 ** rnd.uniform(-10, -2),
+                 weight_decay=rnd.choice([0.0, 0.01, 0.1, 0.5]))
+        t0 = rnd.choice([1, 1, 7, 1000, 123456])
+        mode = case % 2
+        p, m, v = state_init(N, N_pad, case)
+        w = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+        hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
+            np.zeros(N_pad, np.uint16)
+        for t in range(t0, t0 + 3):
+            c = synth.contributions(4, N, N_pad, seed=case, step=t, sigma=1e-3, device="cuda")
+            z3.zero3_reduce_adamw(plan, -1, c, p, m, v, w, z3.adamw(step=t, **a), reduce_dtype=mode)
+            oracle.reduce_adamw([synth.bf16_bits(x) for x in c], S, -1, hp_, hm, hv, hw,
+                                oracle.hp(a["lr"], a["beta1"], a["beta2"], a["eps"], a["weight_decay"], t),
+                                reduce_dtype=mode)
+        torch.cuda.synchronize()
+        what = f"case {case} {a} t0={t0} mode={mode}"
+        assert_f32_parity(f32_host(p), hp_, "master " + what)
+        assert_f32_parity(f32_host(m), hm, "exp_avg " + what)
+        assert_f32_parity(f32_host(v), hv, "exp_avg_sq " + what)
+        assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16 " + what)
