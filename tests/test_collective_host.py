@@ -1,0 +1,111 @@
+"""The collective D-rank step (fsdp_sharded_mixed_flat_b200/collective.py) on
+CPU: gloo groups of 2 and 4 ranks move the real bytes (the all-to-all of the
+gradients, the all-gather of the shards), and the oracle stands in for the
+fused kernel on each rank.  Every rank's state and gathered block must equal a
+single-process oracle run over all ranks, bit for bit."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+import synth
+
+SHAPES = [(3000,), (77, 5), (4097,)]
+SEED = 5
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """A host bf16 tensor's storage as uint16 bit patterns (shared, not copied)."""
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+class OracleKernels:
+    """The fused kernel's entry point, computed by the oracle on host tensors."""
+    Z3_CONTRIB_OWNED = oracle.LAYOUT_OWNED
+
+    def zero3_reduce_adamw(self, plan, rank, contrib, master, exp_avg, exp_avg_sq, work, hp, contrib_layout,
+                           reduce_dtype):
+        assert contrib_layout == oracle.LAYOUT_OWNED
+        oracle.reduce_adamw([_bits(c) for c in contrib], plan.S, rank, master.numpy(), exp_avg.numpy(),
+                            exp_avg_sq.numpy(), _bits(work),
+                            oracle.hp(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, hp.step),
+                            layout=oracle.LAYOUT_OWNED, reduce_dtype=reduce_dtype)
+
+
+def _worker(rank, world, port, mode, steps, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
+    plan = z3.zero3_plan(SHAPES, world, 8)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    p_full = synth.master_weights(N, N_pad, seed=SEED)
+    grad = torch.zeros(N_pad, dtype=torch.bfloat16)
+    master = p_full[rank * S:(rank + 1) * S].clone()
+    m, v = torch.zeros(S), torch.zeros(S)
+    work = torch.zeros(S, dtype=torch.bfloat16)
+    flat = torch.zeros(N_pad, dtype=torch.bfloat16)
+    step = CollectiveZero3Step(plan, grad, master, m, v, work, flat, reduce_dtype=mode, kernels=OracleKernels())
+    for t in range(1, steps + 1):
+        grad.copy_(synth.contribution(N, N_pad, seed=SEED, step=t, rank=rank, sigma=1e-3))
+        step.step(z3.adamw(step=t))
+    out[rank] = (master.numpy().copy(), m.numpy().copy(), v.numpy().copy(), _bits(work).copy(), _bits(flat).copy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,mode", [(2, 0), (4, 0), (4, 1)])
+def test_collective_step_equals_one_oracle_run_over_all_ranks(world, mode):
+    steps = 3
+    with mp.Manager() as manager:
+        out = manager.dict()
+        mp.spawn(_worker, args=(world, _free_port(), mode, steps, out), nprocs=world, join=True)
+        results = dict(out)
+    offs, N, N_pad, S = oracle.plan([int(np.prod(s)) for s in SHAPES], world, 8)
+    p = synth.master_weights(N, N_pad, seed=SEED).numpy().copy()
+    m, v, w = np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.uint16)
+    for t in range(1, steps + 1):
+        c = [synth.bf16_bits(synth.contribution(N, N_pad, seed=SEED, step=t, rank=d, sigma=1e-3))
+             for d in range(world)]
+        oracle.reduce_adamw(c, S, -1, p, m, v, w, oracle.hp(step=t), reduce_dtype=mode)
+    for r in range(world):
+        rp, rm, rv, rw, rflat = results[r]
+        sl = slice(r * S, (r + 1) * S)
+        assert np.array_equal(rp.view(np.uint32), p[sl].view(np.uint32)), f"master rank {r}"
+        assert np.array_equal(rm.view(np.uint32), m[sl].view(np.uint32)), f"exp_avg rank {r}"
+        assert np.array_equal(rv.view(np.uint32), v[sl].view(np.uint32)), f"exp_avg_sq rank {r}"
+        assert np.array_equal(rw, w[sl]), f"work rank {r}"
+        assert np.array_equal(rflat, w), f"gathered block rank {r}"
+
+
+def test_collective_step_rejects_a_plan_for_another_group_size():
+    port = _free_port()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1)
+    try:
+        from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+        from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
+        plan = z3.zero3_plan(SHAPES, 2, 8)
+        bf = lambda n: torch.zeros(n, dtype=torch.bfloat16)   # noqa: E731
+        with pytest.raises(ValueError, match="group has 1"):
+            CollectiveZero3Step(plan, bf(plan.N_pad), torch.zeros(plan.S), torch.zeros(plan.S),
+                                torch.zeros(plan.S), bf(plan.S), bf(plan.N_pad))
+        plan1 = z3.zero3_plan(SHAPES, 1, 8)
+        with pytest.raises(ValueError, match="flat"):
+            CollectiveZero3Step(plan1, bf(plan1.N_pad), torch.zeros(plan1.S), torch.zeros(plan1.S),
+                                torch.zeros(plan1.S), bf(plan1.S), bf(plan1.N_pad - 1))
+    finally:
+        dist.destroy_process_group()

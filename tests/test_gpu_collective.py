@@ -1,0 +1,66 @@
+"""The collective D-rank step on one GPU: a one-rank NCCL group (the all-to-all
+and all-gather reduce to copies), with the real fused kernel, against the
+oracle.  Groups of several GPUs cannot run here (one GPU per run); the same
+step's data movement with 2 and 4 ranks is tested on CPU with gloo in
+test_collective_host.py."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+import oracle
+import synth
+from parity_util import assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def z3():
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    from fsdp_sharded_mixed_flat_b200 import build
+    build.build()
+    from fsdp_sharded_mixed_flat_b200 import zero3
+    return zero3
+
+
+@pytest.fixture()
+def nccl_one_rank():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    from datetime import timedelta
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=timedelta(seconds=60), device_id=dev)
+    yield
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+def test_one_rank_nccl_group_matches_oracle(z3, nccl_one_rank, mode):
+    from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
+    plan = z3.zero3_plan([(50000,), (77, 3), (4097,)], 1, 128)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    grad = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    p = synth.master_weights(N, N_pad, seed=31, device="cuda")
+    m, v = torch.zeros_like(p), torch.zeros_like(p)
+    w = torch.zeros(S, dtype=torch.bfloat16, device="cuda")
+    flat = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    step = CollectiveZero3Step(plan, grad, p, m, v, w, flat, reduce_dtype=mode)
+    hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(S, np.float32), np.zeros(S, np.float32), np.zeros(S, np.uint16)
+    for t in range(1, 4):
+        grad.copy_(synth.contribution(N, N_pad, seed=31, step=t, rank=0, sigma=1e-3, device="cuda"))
+        step.step(z3.adamw(**hp_for(t)))
+        oracle.reduce_adamw([synth.bf16_bits(grad)], S, 0, hp_, hm, hv, hw, oracle_hp(t), reduce_dtype=mode)
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(p), hp_, "master")
+    assert_f32_parity(f32_host(m), hm, "exp_avg")
+    assert_f32_parity(f32_host(v), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
+    assert np.array_equal(synth.bf16_bits(flat), hw)
