@@ -83,6 +83,10 @@ def _bind(L):
     L.ref_reduce_scatter_hybrid.restype = C.c_int
     L.ref_reduce_adamw_hybrid.argtypes = [i32, i32, i64, i32, p, i32, p, p, p, p, i32, C.POINTER(AdamWHP)]
     L.ref_reduce_adamw_hybrid.restype = C.c_int
+    L.ref_node_sum.argtypes = [i32, i64, i32, p, i32, i32, p]
+    L.ref_node_sum.restype = C.c_int
+    L.ref_fold_adamw.argtypes = [i32, i32, i64, p, p, p, p, p, i32, C.POINTER(AdamWHP)]
+    L.ref_fold_adamw.restype = C.c_int
     L.ref_all_gather.argtypes = [i32, i64, p, p]
     L.ref_all_gather.restype = None
     L.ref_unflatten.argtypes = [p, i32, p, p, p]
@@ -234,6 +238,32 @@ def reduce_adamw_hybrid(contribs, R: int, S: int, rank: int, master, exp_avg, ex
                                        C.byref(h))
     if rc != 0:
         raise ValueError("invalid reduce_adamw_hybrid arguments")
+
+
+def node_sum(contribs, S: int, rank: int, layout: int = LAYOUT_FULL, reduce_dtype: int = REDUCE_FP32) -> np.ndarray:
+    """HYBRID_SHARD across nodes, part 1: the node's unscaled rank-ordered sum of
+    its D contributions (D = len(contribs)) for one partition or all of them."""
+    contribs = [_u16(c) for c in contribs]
+    D = len(contribs)
+    out = np.empty(D * S if rank < 0 else S, dtype=np.float32)
+    rc = lib().ref_node_sum(D, S, rank, _ptr_array(contribs), layout, reduce_dtype, _ptr(out))
+    if rc != 0:
+        raise ValueError("invalid node_sum arguments")
+    return out
+
+
+def fold_adamw(node_sums, D: int, master, exp_avg, exp_avg_sq, work_bf16, h: AdamWHP,
+               reduce_dtype: int = REDUCE_FP32) -> None:
+    """HYBRID_SHARD across nodes, part 2: the R = len(node_sums) node sums folded
+    in node order, 1/(R*D), AdamW and the cast; in place, writes work_bf16."""
+    sums = [_f32(x) for x in node_sums]
+    for a in (master, exp_avg, exp_avg_sq):
+        assert a.flags.c_contiguous and a.dtype == np.float32
+    assert work_bf16.flags.c_contiguous and work_bf16.dtype == np.uint16
+    rc = lib().ref_fold_adamw(len(sums), D, master.size, _ptr_array(sums), _ptr(master), _ptr(exp_avg),
+                              _ptr(exp_avg_sq), _ptr(work_bf16), reduce_dtype, C.byref(h))
+    if rc != 0:
+        raise ValueError("invalid fold_adamw arguments")
 
 
 # ------------------------------------------------------- gather and unflatten

@@ -429,6 +429,74 @@ int ref_reduce_adamw_hybrid(int32_t R, int32_t D, int64_t S, int32_t rank, const
 }
 
 /* ------------------------------------------------------------------------ */
+/* HYBRID_SHARD across nodes, in two parts.  Between nodes the node sums have */
+/* to exist in memory: each rank computes its node's sum for its partition,  */
+/* the sums cross the nodes (one exchange per step), and every node folds    */
+/* them in node order.  Composed, the two parts are reduce_hybrid_one above. */
+/* ------------------------------------------------------------------------ */
+
+/* Part 1: the node's sum for local rank `rank`'s partition (S elements), or for
+ * every partition (rank = -1, D*S elements): its D contributions folded left
+ * to right in rank order, not scaled.  reduce_dtype 1 rounds every partial sum
+ * to bf16, so every result is a bf16 value (held here in binary32).
+ * Returns 0, or -1 on an invalid argument. */
+int ref_node_sum(int32_t D, int64_t S, int32_t rank, const uint16_t* const* contrib, int32_t layout,
+                 int32_t reduce_dtype, float* out)
+{
+    if (hybrid_args_invalid(1, D, S, rank, layout, reduce_dtype))
+        return -1;
+    int32_t r0 = rank < 0 ? 0 : rank;
+    int32_t r1 = rank < 0 ? D : rank + 1;
+    for (int32_t r = r0; r < r1; ++r)
+        for (int64_t j = 0; j < S; ++j) {
+            int64_t idx = contrib_index(layout, S, r, j);
+            int64_t o = rank < 0 ? (int64_t)r * S + j : j;
+            if (reduce_dtype == 0) {
+                float acc = ref_f32_from_bf16(contrib[0][idx]);
+                for (int32_t d = 1; d < D; ++d)
+                    acc = acc + ref_f32_from_bf16(contrib[d][idx]);
+                out[o] = acc;
+            } else {
+                uint16_t acc = contrib[0][idx];
+                for (int32_t d = 1; d < D; ++d)
+                    acc = ref_bf16_from_f32(ref_f32_from_bf16(acc) + ref_f32_from_bf16(contrib[d][idx]));
+                out[o] = ref_f32_from_bf16(acc);
+            }
+        }
+    return 0;
+}
+
+/* Part 2: for n owned elements, the R node sums (node_sums[k][i], node k's sum,
+ * as part 1 wrote it) folded in node order 0..R-1, multiplied by the binary32
+ * constant 1/(R*D), then AdamW on master / exp_avg / exp_avg_sq and the cast
+ * of the new master to work_bf16.  In bf16 mode every partial sum across nodes
+ * and the scaled result are rounded to bf16.  Returns 0, or -1 on an invalid
+ * argument. */
+int ref_fold_adamw(int32_t R, int32_t D, int64_t n, const float* const* node_sums, float* master,
+                   float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16, int32_t reduce_dtype,
+                   const ref_adamw_hp* hp)
+{
+    if (R < 1 || D < 1 || n < 0 || (reduce_dtype != 0 && reduce_dtype != 1) || hp->step < 1)
+        return -1;
+    ref_adamw_consts c = adamw_consts(hp);
+    float inv_RD = inverse_of(R * D);
+    for (int64_t i = 0; i < n; ++i) {
+        float total = node_sums[0][i];
+        for (int32_t k = 1; k < R; ++k) {
+            total = total + node_sums[k][i];
+            if (reduce_dtype == 1)
+                total = ref_f32_from_bf16(ref_bf16_from_f32(total));
+        }
+        float g = total * inv_RD;
+        if (reduce_dtype == 1)
+            g = ref_f32_from_bf16(ref_bf16_from_f32(g));
+        adamw_one(&c, g, &master[i], &exp_avg[i], &exp_avg_sq[i]);
+        work_bf16[i] = ref_bf16_from_f32(master[i]);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* All-gather.  [P3] "AllGather vs AllReduce": GPU r holds shard r; after    */
 /* the all-gather every GPU holds [shard 0, shard 1, ..., shard D-1].        */
 /* [P2] §5.1: full_params = all_gather(local_shard) before the block runs.   */

@@ -532,6 +532,69 @@ def test_hybrid_step_composes_reduce_then_adamw():
         assert np.array_equal(a[3], bf16_torch_bits(b[0]))
 
 
+@pytest.mark.parametrize("R,D", [(2, 3), (4, 8), (3, 1), (1, 4)])
+def test_node_sums_then_fold_is_the_hybrid_step(R, D):
+    """Pin: HYBRID_SHARD split across nodes (each node's sum, then the fold of
+    the node sums with AdamW) is the pinned two-level step, bit for bit, for
+    every partition at once and for one rank in the owned layout."""
+    rng = np.random.default_rng(600 + 10 * R + D)
+    S = 23
+    contribs = [rand_bf16(rng, D * S) for _ in range(R * D)]
+    p0 = (rng.standard_normal(D * S) * 0.02).astype(np.float32)
+    for mode in (oracle.REDUCE_FP32, oracle.REDUCE_BF16):
+        ref = [p0.copy(), np.zeros(D * S, np.float32), np.zeros(D * S, np.float32), np.zeros(D * S, np.uint16)]
+        got = [p0.copy(), np.zeros(D * S, np.float32), np.zeros(D * S, np.float32), np.zeros(D * S, np.uint16)]
+        for t in (1, 2):
+            oracle.reduce_adamw_hybrid(contribs, R, S, -1, *ref, oracle.hp(step=t), reduce_dtype=mode)
+            sums = [oracle.node_sum(contribs[k * D:(k + 1) * D], S, -1, reduce_dtype=mode) for k in range(R)]
+            oracle.fold_adamw(sums, D, *got, oracle.hp(step=t), reduce_dtype=mode)
+        for a, b in zip(got, ref):
+            assert np.array_equal(a.view(np.uint8), b.view(np.uint8)), (R, D, mode)
+        r = D - 1                                               # one rank, owned slices
+        owned = [c[r * S:(r + 1) * S].copy() for c in contribs]
+        one = [p0[r * S:(r + 1) * S].copy(), np.zeros(S, np.float32), np.zeros(S, np.float32),
+               np.zeros(S, np.uint16)]
+        sums = [oracle.node_sum(owned[k * D:(k + 1) * D], S, r, oracle.LAYOUT_OWNED, mode) for k in range(R)]
+        oracle.fold_adamw(sums, D, *one, oracle.hp(step=1), reduce_dtype=mode)
+        first = [p0.copy(), np.zeros(D * S, np.float32), np.zeros(D * S, np.float32), np.zeros(D * S, np.uint16)]
+        oracle.reduce_adamw_hybrid(contribs, R, S, -1, *first, oracle.hp(step=1), reduce_dtype=mode)
+        for a, b in zip(one, first):
+            assert np.array_equal(a.view(np.uint8), b[r * S:(r + 1) * S].view(np.uint8))
+
+
+def test_hybrid_worked_examples_through_the_two_parts(golden):
+    """Pin: the hand-derived HYBRID_SHARD examples, reached through the node
+    sums and their fold (AdamW with lr = 0 and no decay leaves the master, and
+    the first moment is (1 - beta1) g, so g is read back from it)."""
+    g = golden("hybrid_worked_examples.json")
+    for case in g["cases"]:
+        R, D = case["R"], case["D"]
+        contribs = [bf16_torch_bits(np.array([x], dtype=np.float32)) for x in case["contributions"]]
+        sums = [oracle.node_sum(contribs[k * D:(k + 1) * D], 1, 0, oracle.LAYOUT_OWNED, case["reduce_dtype"])
+                for k in range(R)]
+        p, m, v, w = np.zeros(1, np.float32), np.zeros(1, np.float32), np.zeros(1, np.float32), np.zeros(1, np.uint16)
+        oracle.fold_adamw(sums, D, p, m, v, w, oracle.hp(lr=0.0, beta1=0.0, weight_decay=0.0), case["reduce_dtype"])
+        assert float(m[0]) == case["expected"], case["name"]
+
+
+@pytest.mark.parametrize("D", [1, 2, 5, 8])
+def test_node_sum_matches_torch_folds(D):
+    """Pin: the node sum is torch's own left fold, fp32 adds of the bf16 values
+    or bf16 tensor adds, with no scaling."""
+    rng = np.random.default_rng(700 + D)
+    S = 29
+    contribs = [rand_bf16(rng, D * S) for _ in range(D)]
+    t = [torch.from_numpy(c.view(np.int16)).view(torch.bfloat16) for c in contribs]
+    acc32, acc16 = t[0].float().clone(), t[0].clone()
+    for d in range(1, D):
+        acc32 = acc32 + t[d].float()
+        acc16 = acc16 + t[d]
+    got32 = oracle.node_sum(contribs, S, -1, reduce_dtype=oracle.REDUCE_FP32)
+    got16 = oracle.node_sum(contribs, S, -1, reduce_dtype=oracle.REDUCE_BF16)
+    assert np.array_equal(got32.view(np.uint32), acc32.numpy().view(np.uint32))
+    assert np.array_equal(got16.view(np.uint32), acc16.float().numpy().view(np.uint32))
+
+
 def test_hybrid_rejects_bad_arguments():
     c = [np.zeros(8, dtype=np.uint16)] * 4
     with pytest.raises(ValueError):

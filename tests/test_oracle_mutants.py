@@ -49,6 +49,18 @@ MUTANTS = [
     ("the all-gather counts the device's own shard as received",
      "return (double)n_blocks * block_bytes * (double)(D - 1) / (double)D;",
      "return (double)n_blocks * block_bytes * (double)(D) / (double)D;"),
+    ("the cross-node fold takes the node sums in reverse order",
+     "float total = node_sums[0][i];\n"
+     "        for (int32_t k = 1; k < R; ++k) {\n"
+     "            total = total + node_sums[k][i];",
+     "float total = node_sums[R - 1][i];\n"
+     "        for (int32_t k = 1; k < R; ++k) {\n"
+     "            total = total + node_sums[R - 1 - k][i];"),
+    ("the cross-node fold leaves the scaled bf16 gradient unrounded",
+     "        float g = total * inv_RD;\n"
+     "        if (reduce_dtype == 1)\n"
+     "            g = ref_f32_from_bf16(ref_bf16_from_f32(g));",
+     "        float g = total * inv_RD;"),
     ("HYBRID_SHARD folds all ranks flat, ignoring the nodes",
      "float node_sum = ref_f32_from_bf16(node[0][idx]);",
      "float node_sum = k == 0 ? ref_f32_from_bf16(node[0][idx]) : total + ref_f32_from_bf16(node[0][idx]);"
@@ -124,6 +136,9 @@ PINS = [
     lambda: pins.test_hybrid_one_rank_per_node_is_the_plain_fold_over_nodes(3, 0),
     lambda: pins.test_hybrid_one_rank_per_node_is_the_plain_fold_over_nodes(3, 1),
     lambda: pins.test_hybrid_matches_torch_two_level_fold(2, 3),
+    lambda: pins.test_hybrid_worked_examples_through_the_two_parts(golden),
+    lambda: pins.test_node_sums_then_fold_is_the_hybrid_step(2, 3),
+    lambda: pins.test_node_sum_matches_torch_folds(5),
 ]
 
 
