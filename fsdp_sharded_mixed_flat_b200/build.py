@@ -19,9 +19,10 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libzero3.so")
 
-SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "gather.cu"]
+SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "node_fold.cu", "gather.cu"]
 EXPORTS = os.path.join(CSRC, "exports.map")
-HEADERS = [os.path.join(CSRC, "plan_impl.h"), os.path.join(INCLUDE, "zero3.h"), EXPORTS]
+HEADERS = [os.path.join(CSRC, "plan_impl.h"), os.path.join(CSRC, "step_common.cuh"), os.path.join(INCLUDE, "zero3.h"),
+           EXPORTS]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xptxas", "-v",

@@ -45,18 +45,10 @@
 #include <cstring>
 
 #include "plan_impl.h"
+#include "step_common.cuh"
 #include "zero3.h"
 
 namespace {
-
-// The eight fp32 scalars of one AdamW step, in the order the C ABI documents
-// for zero3_step_scalars.
-struct AdamScalars {
-    float step_size;     // lr / (1 - b1^t)
-    float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
-    float decay;         // 1 - lr * wd
-    float b1, omb1, b2, omb2, eps;
-};
 
 struct K1Args {
     const uint16_t* c[Z3_D_MAX];  // contributions c[k*D + d] (node k, rank d), each at the launch's first element
@@ -74,97 +66,10 @@ struct K1Args {
     int32_t R;                    // nodes (HYBRID_SHARD; 1 otherwise)
 };
 
-static_assert(sizeof(AdamScalars) == Z3_SCALARS * sizeof(float), "scalar layout");
-
-// Host computation of one step's scalars: binary64, each rounded to fp32 once.
-AdamScalars step_scalars(const z3_adamw* hp) {
-    AdamScalars s;
-    const double t = double(hp->step);
-    const double bc1 = 1.0 - std::pow(hp->beta1, t);
-    const double bc2 = 1.0 - std::pow(hp->beta2, t);
-    s.step_size = float(hp->lr / bc1);
-    s.inv_sqrt_bc2 = float(1.0 / std::sqrt(bc2));
-    s.decay = float(1.0 - hp->lr * hp->weight_decay);
-    s.b1 = float(hp->beta1);
-    s.omb1 = float(1.0 - hp->beta1);
-    s.b2 = float(hp->beta2);
-    s.omb2 = float(1.0 - hp->beta2);
-    s.eps = float(hp->eps);
-    return s;
-}
-
 constexpr int kThreads = 256;
 constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: at most 80 registers per thread
 constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
-
-__device__ __forceinline__ float lo_bf16(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float hi_bf16(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }
-__device__ __forceinline__ float bf16_of(uint16_t h) { return __uint_as_float(uint32_t(h) << 16); }
-
-// 16-byte load (default caching) and streaming store.  Among the cache hints
-// measured on B200 for this kernel (streaming, read-only, last-use and
-// default loads; streaming and default stores), default loads with streaming
-// stores moved the most bytes per second at every D.
-template <class T>
-__device__ __forceinline__ T ld16(const T* p) { return *p; }
-template <class T>
-__device__ __forceinline__ void st16(T* p, const T& v) { __stcs(p, v); }
-
-// fp32 -> nearest-even bf16 -> fp32.
-__device__ __forceinline__ float round_to_bf16(float x) {
-    return __bfloat162float(__float2bfloat16_rn(x));
-}
-
-// Two fp32 values -> two nearest-even bf16 in one 32-bit word (lo in bits 0..15).
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// One AdamW element; each step a single fp32 operation rounded to nearest-even.
-__device__ __forceinline__ void adamw_elem(const AdamScalars& s, float g, float& p, float& m,
-                                           float& v) {
-    const float p1 = __fmul_rn(p, s.decay);
-    const float m1 = __fadd_rn(__fmul_rn(s.b1, m), __fmul_rn(s.omb1, g));
-    const float v1 = __fadd_rn(__fmul_rn(s.b2, v), __fmul_rn(s.omb2, __fmul_rn(g, g)));
-    const float denom = __fadd_rn(__fmul_rn(__fsqrt_rn(v1), s.inv_sqrt_bc2), s.eps);
-    const float delta = __fmul_rn(s.step_size, __fdiv_rn(m1, denom));
-    p = __fsub_rn(p1, delta);
-    m = m1;
-    v = v1;
-}
-
-// Two bf16 values added pairwise by the packed hardware add, which rounds the
-// exact sum to the nearest-even bf16.  That equals rounding the fp32 sum to
-// bf16: double rounding through a format with more than 2p + 2 significand
-// bits is innocuous (Figueroa, "When is double rounding innocuous?", 1995),
-// and fp32's 24 bits exceed 18 for bf16's p = 8, also in the shared subnormal
-// range, where both formats lose the same number of leading bits.
-__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-// Fold one rank's 8 bf16 values (one 16-byte vector) into fp32 accumulators.
-__device__ __forceinline__ void fold8_fp32(float (&acc)[8], const uint4& q, bool first) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float a = lo_bf16(w[k]), b = hi_bf16(w[k]);
-        acc[2 * k] = first ? a : __fadd_rn(acc[2 * k], a);
-        acc[2 * k + 1] = first ? b : __fadd_rn(acc[2 * k + 1], b);
-    }
-}
-
-// Fold one rank's 8 bf16 values into packed bf16 accumulators (element 2k in
-// the low half of word k).
-__device__ __forceinline__ void fold8_bf16(uint32_t (&acc)[4], const uint4& q, bool first) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = first ? w[k] : add_bf16x2(acc[k], w[k]);
-}
 
 // Fold ranks base..base+D-1 for the 8 elements starting at e into the fp32 or
 // packed-bf16 accumulators, left to right, in chunks of ranks (the chunk's
@@ -233,13 +138,6 @@ __device__ __forceinline__ void reduce8(const K1Args& a, int64_t e, float (&g)[8
     }
 }
 
-// One partial sum in the reduce dtype: the fp32 sum, rounded to bf16 in bf16 mode.
-template <int MODE>
-__device__ __forceinline__ float add_in(float x, float y) {
-    const float s = __fadd_rn(x, y);
-    return MODE == Z3_REDUCE_FP32 ? s : round_to_bf16(s);
-}
-
 // One element on the scalar path (tails and misaligned buffers).  RT = 1: the
 // rank fold; otherwise the nodes' rank folds, then the fold of the node sums.
 template <int MODE, int RT, bool GATHER>
@@ -301,15 +199,6 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
         for (int k = 0; k < Z3_GATHER_MAX; ++k)
             if (k < a.ng) st16(reinterpret_cast<uint4*>(a.g[k] + e), w);
     }
-}
-
-// The scalars of this step, (DEVS) read from device memory, so that a captured
-// CUDA graph can be replayed step after step with only the 32-byte scalar
-// buffer rewritten in between.
-__device__ __forceinline__ AdamScalars load_scalars(const AdamScalars* p) {
-    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
-    const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
-    return AdamScalars{x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
 }
 
 // Vector kernel body: every pointer 16-byte aligned.  The grid covers the
@@ -405,16 +294,6 @@ KernelFn pick_any(bool gather, bool devs, bool vec, int32_t reduce_dtype, int D,
     if (gather)
         return devs ? pick<true, true>(vec, reduce_dtype, D) : pick<true, false>(vec, reduce_dtype, D);
     return devs ? pick<false, true>(vec, reduce_dtype, D) : pick<false, false>(vec, reduce_dtype, D);
-}
-
-bool hp_valid(const z3_adamw* hp);
-
-bool is_finite(double x) { return std::isfinite(x); }
-
-bool hp_valid(const z3_adamw* hp) {
-    return hp != nullptr && hp->step >= 1 && is_finite(hp->lr) && is_finite(hp->beta1) &&
-           is_finite(hp->beta2) && is_finite(hp->eps) && is_finite(hp->weight_decay) && hp->beta1 >= 0.0 &&
-           hp->beta1 < 1.0 && hp->beta2 >= 0.0 && hp->beta2 < 1.0;
 }
 
 // Validation and launch shared by every entry point.  `gathered` holds

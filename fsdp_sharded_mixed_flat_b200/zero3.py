@@ -70,6 +70,10 @@ def _load() -> C.CDLL:
     L.zero3_reduce_adamw.restype = C.c_int
     L.zero3_reduce_adamw_hybrid.argtypes = [vp, i32, i32, vp, i32, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw_hybrid.restype = C.c_int
+    L.zero3_node_sum.argtypes = [vp, i32, vp, i32, i32, vp, vp]
+    L.zero3_node_sum.restype = C.c_int
+    L.zero3_fold_adamw.argtypes = [vp, i32, i32, vp, vp, vp, vp, vp, i32, C.POINTER(AdamW), vp]
+    L.zero3_fold_adamw.restype = C.c_int
     L.zero3_reduce_adamw_gather.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp, vp, i32, i32,
                                             C.POINTER(AdamW), vp]
     L.zero3_reduce_adamw_gather.restype = C.c_int
@@ -300,6 +304,50 @@ def zero3_reduce_adamw_hybrid(plan: Plan, rank: int, n_nodes: int, contrib: Sequ
     rc = _call_on(dev, _lib.zero3_reduce_adamw_hybrid, plan.handle, rank, n_nodes, ptrs, contrib_layout, mp, ap,
                   vp, wp, reduce_dtype, C.byref(hp), _stream_handle(stream, dev))
     _check(rc, "zero3_reduce_adamw_hybrid")
+
+
+def _node_sum_dtype(reduce_dtype: int) -> torch.dtype:
+    return torch.float32 if reduce_dtype == Z3_REDUCE_FP32 else torch.bfloat16
+
+
+def zero3_node_sum(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], node_sum: torch.Tensor,
+                   contrib_layout: int = Z3_CONTRIB_FULL, reduce_dtype: int = Z3_REDUCE_FP32, stream=None) -> None:
+    """HYBRID_SHARD across nodes, part 1: this node's rank-ordered, unscaled sum of
+    its plan.D contributions for the owned partition(s), written to node_sum
+    (float32 for the fp32 reduce, bfloat16 for the bf16 reduce; see include/zero3.h)."""
+    if len(contrib) != plan.D:
+        raise ValueError(f"need {plan.D} contributions, got {len(contrib)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * plan.D)()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    op = _dev_tensor(node_sum, _node_sum_dtype(reduce_dtype), n, "node_sum")
+    dev = _launch_device(node_sum, *contrib)
+    rc = _call_on(dev, _lib.zero3_node_sum, plan.handle, rank, ptrs, contrib_layout, reduce_dtype, op,
+                  _stream_handle(stream, dev))
+    _check(rc, "zero3_node_sum")
+
+
+def zero3_fold_adamw(plan: Plan, rank: int, node_sums: Sequence[torch.Tensor], master: torch.Tensor,
+                     exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor, work_bf16: torch.Tensor, hp: AdamW,
+                     reduce_dtype: int = Z3_REDUCE_FP32, stream=None) -> None:
+    """HYBRID_SHARD across nodes, part 2: the node sums (node order) folded, scaled
+    by 1/(len(node_sums) * plan.D), AdamW and the bf16 cast (see include/zero3.h)."""
+    if not 1 <= len(node_sums) <= Z3_D_MAX:
+        raise ValueError(f"need 1..{Z3_D_MAX} node sums, got {len(node_sums)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    sp = (C.c_void_p * len(node_sums))()
+    for k, x in enumerate(node_sums):
+        sp[k] = _dev_tensor(x, _node_sum_dtype(reduce_dtype), n, f"node_sums[{k}]")
+    mp = _dev_tensor(master, torch.float32, n, "master", host_ok=True)
+    ap = _dev_tensor(exp_avg, torch.float32, n, "exp_avg", host_ok=True)
+    vp = _dev_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq", host_ok=True)
+    wp = _dev_tensor(work_bf16, torch.bfloat16, n, "work_bf16", host_ok=True)
+    dev = _launch_device(work_bf16, master, *node_sums)
+    rc = _call_on(dev, _lib.zero3_fold_adamw, plan.handle, rank, len(node_sums), sp, mp, ap, vp, wp, reduce_dtype,
+                  C.byref(hp), _stream_handle(stream, dev))
+    _check(rc, "zero3_fold_adamw")
 
 
 def zero3_reduce_adamw_gather(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], master: torch.Tensor,

@@ -267,6 +267,43 @@ Z3_API int zero3_reduce_adamw_hybrid(const z3_plan* p, int32_t rank, int32_t n_n
                                      float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
                                      int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream);
 
+/* ------------------------------------ HYBRID_SHARD across nodes, in two parts
+ * When the R nodes are separate machines, each node's sum has to exist in
+ * memory so that it can cross the network once per step ([P3] "HYBRID_SHARD:
+ * The Multi-Node Strategy").  The two calls below split the two-level
+ * reduction of zero3_reduce_adamw_hybrid at that point; composed (node sums of
+ * nodes 0..R-1, in node order), they give its results exactly.
+ *
+ * zero3_node_sum: a node's sum for rank `rank`'s partition (S elements), or for
+ * every partition in one launch (rank = -1: N_pad elements): the node's D
+ * contributions (the plan's D) folded left to right in rank order, not scaled.
+ *   contrib, contrib_layout  as for zero3_reduce_adamw (D device pointers).
+ *   reduce_dtype  Z3_REDUCE_FP32: every partial sum rounded to fp32, node_sum is
+ *                 float; Z3_REDUCE_BF16: every partial sum rounded to bf16,
+ *                 node_sum holds bf16 (uint16_t), half the bytes to send.
+ *   node_sum      device output, S (or N_pad) elements of that type.
+ * The vector path needs node_sum and every contribution (at its partition
+ * offset) 16-byte aligned; otherwise a scalar kernel gives the same results.
+ * Errors: Z3_EINVAL (NULL pointer, rank, layout or dtype out of range, output
+ * over a contribution), Z3_EALIGN (a pointer off its element size), Z3_ECUDA.
+ *
+ * zero3_fold_adamw: for rank `rank`'s partition (or every partition, rank = -1),
+ * the n_nodes node sums folded in node order 0..n_nodes-1 (partial sums in the
+ * reduce dtype), times the fp32 constant nearest 1/(n_nodes * D), then AdamW on
+ * master / exp_avg / exp_avg_sq and the bf16 cast to work_bf16, exactly as in
+ * zero3_reduce_adamw.
+ *   node_sums  host array of n_nodes (1..Z3_D_MAX) device pointers, node k's sum
+ *              as zero3_node_sum wrote it (float or bf16 by reduce_dtype), each
+ *              S (or N_pad) elements.
+ *   master, exp_avg, exp_avg_sq, work_bf16, hp  as for zero3_reduce_adamw.
+ * Errors: Z3_EINVAL (NULL pointer, bad rank, n_nodes or dtype, invalid hp,
+ * overlapping outputs, an output over a node sum), Z3_EALIGN, Z3_ECUDA. */
+Z3_API int zero3_node_sum(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, int32_t contrib_layout,
+                          int32_t reduce_dtype, void* node_sum, void* cuda_stream);
+Z3_API int zero3_fold_adamw(const z3_plan* p, int32_t rank, int32_t n_nodes, const void* const* node_sums,
+                            float* master, float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
+                            int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream);
+
 /* ------------------------------------- scalars in device memory (graphs)
  * zero3_step_scalars: the Z3_SCALARS fp32 scalars of one AdamW step, formed in
  * binary64 from *hp and rounded to fp32 once, exactly as zero3_reduce_adamw

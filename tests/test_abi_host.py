@@ -33,7 +33,7 @@ def test_library_exports_every_declared_symbol():
     assert names == sorted(["zero3_status_string", "zero3_plan", "zero3_plan_free", "zero3_plan_info",
                             "zero3_plan_tensor", "zero3_plan_rank", "zero3_memory_bytes",
                             "zero3_transient_bytes", "zero3_allgather_bytes", "zero3_reduce_adamw",
-                            "zero3_reduce_adamw_hybrid",
+                            "zero3_reduce_adamw_hybrid", "zero3_node_sum", "zero3_fold_adamw",
                             "zero3_reduce_adamw_gather",
                             "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
@@ -238,6 +238,47 @@ def test_reduce_adamw_hybrid_argument_errors():
     e = z3.zero3_plan([], 4, 8)
     assert call_hybrid(e, 16) == z3.Z3_OK                             # 64 contributions, empty plan
     assert call_hybrid(e, 1) == z3.Z3_OK
+
+
+def test_node_sum_and_fold_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)
+    L, E, A = z3.lib(), z3.Z3_EINVAL, z3.Z3_EALIGN
+    c = [P16 * (100 + d) for d in range(4)]
+
+    def node_sum(contrib=c, rank=-1, layout=0, mode=0, out=P16 * 50):
+        arr = (C.c_void_p * 4)(*contrib)
+        return L.zero3_node_sum(p.handle, rank, arr, layout, mode, None if out is None else C.c_void_p(out), None)
+    assert node_sum(out=None) == E
+    assert node_sum(rank=4) == E
+    assert node_sum(layout=1) == E                       # owned layout needs one rank
+    assert node_sum(mode=2) == E
+    assert node_sum(contrib=c[:3] + [0]) == E
+    assert node_sum(contrib=c[:3] + [c[3] + 1]) == A
+    assert node_sum(out=P16 * 50 + 2) == A                # fp32 sums need 4-byte alignment
+    assert node_sum(out=c[2]) == E                        # over a contribution
+    hp = z3.adamw(step=1)
+
+    def fold(sums=(P16 * 200, P16 * 300), n_nodes=None, rank=-1, ptrs=None, mode=0, h=hp):
+        arr = (C.c_void_p * max(1, len(sums)))(*sums)
+        ptrs = ptrs or [P16 * 1, P16 * 2, P16 * 3, P16 * 4]
+        return L.zero3_fold_adamw(p.handle, rank, len(sums) if n_nodes is None else n_nodes, arr,
+                                  *[C.c_void_p(x) for x in ptrs], mode, None if h is None else C.byref(h), None)
+    assert fold(n_nodes=0) == E
+    assert fold(n_nodes=65) == E
+    assert fold(rank=4) == E
+    assert fold(mode=3) == E
+    assert fold(h=None) == E
+    assert fold(h=z3.adamw(step=0)) == E
+    assert fold(sums=(P16 * 200, 0)) == E
+    assert fold(sums=(P16 * 200, P16 * 300 + 2)) == A
+    assert fold(ptrs=[P16 + 2, P16 * 2, P16 * 3, P16 * 4]) == A
+    assert fold(ptrs=[P16 * 10, P16 * 10, P16 * 30, P16 * 40]) == E   # master = exp_avg
+    assert fold(sums=(P16 * 200, P16 * 3)) == E                       # exp_avg_sq over a node sum
+    e = z3.zero3_plan([], 4, 8)
+    assert L.zero3_fold_adamw(e.handle, -1, 2, (C.c_void_p * 2)(P16 * 200, P16 * 300), C.c_void_p(P16),
+                              C.c_void_p(P16 * 2), C.c_void_p(P16 * 3), C.c_void_p(P16 * 4), 0, C.byref(hp),
+                              None) == z3.Z3_OK
+    assert L.zero3_node_sum(e.handle, -1, (C.c_void_p * 4)(*c), 0, 0, C.c_void_p(P16 * 50), None) == z3.Z3_OK
 
 
 def call_fused(plan, gathered, work=P16 * 4, rank=-1, n=None):
