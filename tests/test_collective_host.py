@@ -1,8 +1,9 @@
-"""The collective D-rank step (fsdp_sharded_mixed_flat_b200/collective.py) on
-CPU: gloo groups of 2 and 4 ranks move the real bytes (the all-to-all of the
-gradients, the all-gather of the shards), and the oracle stands in for the
-fused kernel on each rank.  Every rank's state and gathered block must equal a
-single-process oracle run over all ranks, bit for bit."""
+"""The collective steps (fsdp_sharded_mixed_flat_b200/collective.py) on CPU:
+gloo groups move the real bytes (all-to-all of the gradients, all-gathers of
+the node sums and of the shards), and the oracle stands in for the kernels on
+each rank.  ZeRO-3 over 2 and 4 ranks, and HYBRID_SHARD over 2 and 3 nodes of
+2 ranks (node and replica subgroups): every rank's state and gathered block
+must equal a single-process oracle run over all ranks, bit for bit."""
 import os
 import socket
 
@@ -33,8 +34,20 @@ def _bits(t: torch.Tensor) -> np.ndarray:
 
 
 class OracleKernels:
-    """The fused kernel's entry point, computed by the oracle on host tensors."""
+    """The kernels' entry points, computed by the oracle on host tensors."""
     Z3_CONTRIB_OWNED = oracle.LAYOUT_OWNED
+
+    @staticmethod
+    def _hp(hp):
+        return oracle.hp(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, hp.step)
+
+    def zero3_node_sum(self, plan, rank, contrib, node_sum, contrib_layout, reduce_dtype):
+        vals = oracle.node_sum([_bits(c) for c in contrib], plan.S, rank, contrib_layout, reduce_dtype)
+        node_sum.copy_(torch.from_numpy(vals).to(node_sum.dtype))      # exact: bf16 sums are bf16 values
+
+    def zero3_fold_adamw(self, plan, rank, node_sums, master, exp_avg, exp_avg_sq, work, hp, reduce_dtype):
+        oracle.fold_adamw([x.float().numpy() for x in node_sums], plan.D, master.numpy(), exp_avg.numpy(),
+                          exp_avg_sq.numpy(), _bits(work), self._hp(hp), reduce_dtype=reduce_dtype)
 
     def zero3_reduce_adamw(self, plan, rank, contrib, master, exp_avg, exp_avg_sq, work, hp, contrib_layout,
                            reduce_dtype):
@@ -109,3 +122,56 @@ def test_collective_step_rejects_a_plan_for_another_group_size():
                                 torch.zeros(plan1.S), bf(plan1.S), bf(plan1.N_pad - 1))
     finally:
         dist.destroy_process_group()
+
+
+def _hybrid_worker(rank, R, D, port, mode, steps, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=R * D)
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    from fsdp_sharded_mixed_flat_b200.collective import CollectiveHybridStep, hybrid_groups
+    node_group, replica_group = hybrid_groups(R, D)
+    plan = z3.zero3_plan(SHAPES, D, 8)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    d = rank % D
+    p_full = synth.master_weights(N, N_pad, seed=SEED)
+    grad = torch.zeros(N_pad, dtype=torch.bfloat16)
+    master = p_full[d * S:(d + 1) * S].clone()
+    m, v = torch.zeros(S), torch.zeros(S)
+    work = torch.zeros(S, dtype=torch.bfloat16)
+    flat = torch.zeros(N_pad, dtype=torch.bfloat16)
+    step = CollectiveHybridStep(plan, R, grad, master, m, v, work, flat, node_group, replica_group,
+                                reduce_dtype=mode, kernels=OracleKernels())
+    for t in range(1, steps + 1):
+        grad.copy_(synth.contribution(N, N_pad, seed=SEED, step=t, rank=rank, sigma=1e-3))
+        step.step(z3.adamw(step=t))
+    out[rank] = (master.numpy().copy(), m.numpy().copy(), v.numpy().copy(), _bits(work).copy(), _bits(flat).copy())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("R,D,mode", [(2, 2, 0), (2, 2, 1), (3, 2, 0)])
+def test_collective_hybrid_step_equals_the_two_level_oracle(R, D, mode):
+    """HYBRID_SHARD over R nodes of D gloo ranks: every rank equals one oracle
+    run of the two-level reduction over all R*D ranks, bit for bit, and every
+    replica of a local rank holds the same state."""
+    steps = 3
+    with mp.Manager() as manager:
+        out = manager.dict()
+        mp.spawn(_hybrid_worker, args=(R, D, _free_port(), mode, steps, out), nprocs=R * D, join=True)
+        results = dict(out)
+    offs, N, N_pad, S = oracle.plan([int(np.prod(s)) for s in SHAPES], D, 8)
+    p = synth.master_weights(N, N_pad, seed=SEED).numpy().copy()
+    m, v, w = np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.uint16)
+    for t in range(1, steps + 1):
+        c = [synth.bf16_bits(synth.contribution(N, N_pad, seed=SEED, step=t, rank=g, sigma=1e-3))
+             for g in range(R * D)]
+        oracle.reduce_adamw_hybrid(c, R, S, -1, p, m, v, w, oracle.hp(step=t), reduce_dtype=mode)
+    for g in range(R * D):
+        rp, rm, rv, rw, rflat = results[g]
+        d = g % D
+        sl = slice(d * S, (d + 1) * S)
+        assert np.array_equal(rp.view(np.uint32), p[sl].view(np.uint32)), f"master rank {g}"
+        assert np.array_equal(rm.view(np.uint32), m[sl].view(np.uint32)), f"exp_avg rank {g}"
+        assert np.array_equal(rv.view(np.uint32), v[sl].view(np.uint32)), f"exp_avg_sq rank {g}"
+        assert np.array_equal(rw, w[sl]), f"work rank {g}"
+        assert np.array_equal(rflat, w), f"gathered block rank {g}"

@@ -1,7 +1,8 @@
-"""The collective D-rank step on one GPU: a one-rank NCCL group (the all-to-all
-and all-gather reduce to copies), with the real fused kernel, against the
-oracle.  Groups of several GPUs cannot run here (one GPU per run); the same
-step's data movement with 2 and 4 ranks is tested on CPU with gloo in
+"""The collective steps on one GPU: a one-rank NCCL group (the all-to-all and
+all-gathers reduce to copies), with the real kernels, against the oracle --
+ZeRO-3 with the fused kernel, HYBRID_SHARD with the node-sum and fold kernels.
+Groups of several GPUs cannot run here (one GPU per run); the steps' data
+movement with several ranks is tested on CPU with gloo in
 test_collective_host.py."""
 import os
 import socket
@@ -58,6 +59,34 @@ def test_one_rank_nccl_group_matches_oracle(z3, nccl_one_rank, mode):
         grad.copy_(synth.contribution(N, N_pad, seed=31, step=t, rank=0, sigma=1e-3, device="cuda"))
         step.step(z3.adamw(**hp_for(t)))
         oracle.reduce_adamw([synth.bf16_bits(grad)], S, 0, hp_, hm, hv, hw, oracle_hp(t), reduce_dtype=mode)
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(p), hp_, "master")
+    assert_f32_parity(f32_host(m), hm, "exp_avg")
+    assert_f32_parity(f32_host(v), hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
+    assert np.array_equal(synth.bf16_bits(flat), hw)
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+def test_one_rank_nccl_hybrid_step_matches_oracle(z3, nccl_one_rank, mode):
+    """The HYBRID_SHARD collective step on a one-rank NCCL group (one node of one
+    rank): node and replica groups, the node-sum and fold kernels, the gathers."""
+    from fsdp_sharded_mixed_flat_b200.collective import CollectiveHybridStep, hybrid_groups
+    node_group, replica_group = hybrid_groups(1, 1)
+    plan = z3.zero3_plan([(50000,), (77, 3), (4097,)], 1, 128)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    grad = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    p = synth.master_weights(N, N_pad, seed=32, device="cuda")
+    m, v = torch.zeros_like(p), torch.zeros_like(p)
+    w = torch.zeros(S, dtype=torch.bfloat16, device="cuda")
+    flat = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    step = CollectiveHybridStep(plan, 1, grad, p, m, v, w, flat, node_group, replica_group, reduce_dtype=mode)
+    hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(S, np.float32), np.zeros(S, np.float32), np.zeros(S, np.uint16)
+    for t in range(1, 4):
+        grad.copy_(synth.contribution(N, N_pad, seed=32, step=t, rank=0, sigma=1e-3, device="cuda"))
+        step.step(z3.adamw(**hp_for(t)))
+        oracle.reduce_adamw_hybrid([synth.bf16_bits(grad)], 1, S, 0, hp_, hm, hv, hw, oracle_hp(t),
+                                   reduce_dtype=mode)
     torch.cuda.synchronize()
     assert_f32_parity(f32_host(p), hp_, "master")
     assert_f32_parity(f32_host(m), hm, "exp_avg")
