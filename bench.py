@@ -83,6 +83,9 @@ def parse_args():
     ap.add_argument("--drift", action="store_true",
                     help="report the drift of the bf16-reduce path against the fp32-reduce path")
     ap.add_argument("--drift-elements", type=int, default=1 << 24)
+    ap.add_argument("--split", action="store_true",
+                    help="HYBRID_SHARD workload: the node sums of every node, then their fold (two kernels, what "
+                         "separate machines run) instead of the fused kernel")
     ap.add_argument("--stage", type=int, choices=[1, 2, 3], default=3,
                     help="3: ZeRO-3 step (fused reduce/AdamW/cast, then the gather of the shards); "
                          "1 or 2: the fused kernel also all-gathers into the replicated bf16 weights")
@@ -340,7 +343,7 @@ class BlockRunner:
     the replicated bf16 weights (the flat block), with no separate shard."""
 
     def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
-                 graph=False, offload=False):
+                 graph=False, offload=False, split=False):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
@@ -353,6 +356,12 @@ class BlockRunner:
         self.nodes = w.get("nodes", 1)
         if self.nodes > 1 and (stage != 3 or graph or offload):
             raise SystemExit("the HYBRID_SHARD workload runs the plain ZeRO-3 block step")
+        if split and self.nodes == 1:
+            raise SystemExit("--split needs a HYBRID_SHARD workload (llama7b_hybrid)")
+        # --split: the two-level reduction as the node sums of every node, then their fold
+        # (what separate machines run), instead of the fused kernel
+        self.split = split
+        self.mid_events = []
         self.contribs = synth.contributions(self.nodes * D, self.N, self.N_pad, seed=seed, step=1,
                                             sigma=w["sigma"], dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
                                             device=dev)
@@ -383,11 +392,24 @@ class BlockRunner:
         self.step_bytes = self.k1_bytes_per_launch + (4 * self.N_pad if stage == 3 else 0) + \
             (4 * self.N if self.tensor_out is not None else 0)
         self.launches_per_step = (2 + (1 if self.tensor_out is not None else 0)) if stage == 3 else 1
+        if split:
+            esz = 4 if reduce_dtype == 0 else 2
+            sum_dtype = torch.float32 if reduce_dtype == 0 else torch.bfloat16
+            self.node_sums = [torch.empty(self.N_pad, dtype=sum_dtype, device=dev) for _ in range(self.nodes)]
+            self.node_sum_bytes = self.nodes * (2 * D + esz) * self.N_pad      # all nodes' sums
+            self.fold_bytes = (self.nodes * esz + 26) * self.N_pad
+            self.k1_bytes_per_launch = self.node_sum_bytes + self.fold_bytes
+            self.launches_per_step = self.nodes + 2
+            self.step_bytes = self.k1_bytes_per_launch + 4 * self.N_pad
         ranks = f"{self.nodes} nodes x D={D}" if self.nodes > 1 else f"D={D}"
         self.k1_name = (f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, {ranks}"
                         f"{', gather' if stage != 3 else ''}>")
-        hybrid = (" (HYBRID_SHARD: each node's rank fold, then the node sums across %d nodes, then 1/%d)"
-                  % (self.nodes, self.nodes * D) if self.nodes > 1 else "")
+        if split:
+            self.k1_name = (f"{self.nodes} x k_node_sum_vec<D={D}> + k_fold_adamw_vec<R={self.nodes}> "
+                            f"({'fp32' if reduce_dtype == 0 else 'bf16'}; the split HYBRID_SHARD reduction)")
+        hybrid = (" (HYBRID_SHARD: each node's rank fold, then the node sums across %d nodes, then 1/%d%s)"
+                  % (self.nodes, self.nodes * D, "; split: every node's sum written, then their fold"
+                     if split else "") if self.nodes > 1 else "")
         what = ("fused reduce/AdamW/cast over all %d partitions%s + gather into the flat block%s" %
                 (D, hybrid, " and into one buffer per tensor" if self.tensor_out is not None else "")
                 if stage == 3
@@ -449,7 +471,19 @@ class BlockRunner:
                 k1_events[0][1].record(self.stream)
             return self.views(pl, flat)
         # a3 + a4: reduce-scatter reduction + AdamW + bf16 cast, every rank's partition in one launch
-        if self.nodes > 1:
+        if self.split:
+            D = self.D
+            for k in range(self.nodes):
+                z3.zero3_node_sum(pl, -1, contribs[k * D:(k + 1) * D], self.node_sums[k], reduce_dtype=self.mode,
+                                  stream=self.stream)
+            if k1_events is not None:
+                import torch
+                mid = torch.cuda.Event(enable_timing=True)
+                mid.record(self.stream)
+                self.mid_events.append((k1_events[0][0], mid, k1_events[0][1]))
+            z3.zero3_fold_adamw(pl, -1, self.node_sums, self.master, self.exp_avg, self.exp_avg_sq, self.work, hp,
+                                reduce_dtype=self.mode, stream=self.stream)
+        elif self.nodes > 1:
             z3.zero3_reduce_adamw_hybrid(pl, -1, self.nodes, contribs, self.master, self.exp_avg,
                                          self.exp_avg_sq, self.work, hp, reduce_dtype=self.mode, stream=self.stream)
         else:
@@ -623,7 +657,7 @@ def run_ours(args):
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
                         stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph,
-                        offload=args.offload)
+                        offload=args.offload, split=args.split)
     stream = R.stream
 
     for _ in range(args.warmup):
@@ -716,13 +750,22 @@ def run_ours(args):
                      "frac_of_nominal_8000": k1_gbs / 8000.0, "kernel": R.k1_name,
                      "algorithmic_bytes_per_launch": R.k1_bytes_per_launch,
                      "traffic": (profiled_traffic(args.workload)
-                                 if mode == 0 and args.stage == 3 and not args.graph else None)},
+                                 if mode == 0 and args.stage == 3 and not args.graph and not args.split
+                                 else None)},
         "clocks": clk,
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": R.launches_per_step * args.steps,
         "ledger_bytes_per_device": ledger(z3, *R.ledger_args),
     }
+    if getattr(R, "split", False) and R.mid_events:
+        ns = statistics.mean(a.elapsed_time(b) for a, b, _ in R.mid_events) / 1e3
+        fo = statistics.mean(b.elapsed_time(c) for _, b, c in R.mid_events) / 1e3
+        extra["split_hybrid"] = {"node_sums_ms": 1e3 * ns, "node_sums_gbs": R.node_sum_bytes / ns / 1e9,
+                                 "fold_ms": 1e3 * fo, "fold_gbs": R.fold_bytes / fo / 1e9,
+                                 "node_sum_bytes": R.node_sum_bytes, "fold_bytes": R.fold_bytes,
+                                 "note": "every node's sum (R launches) on one GPU, then the fold: on separate "
+                                         "machines each node runs one node sum and the fold"}
     line.update(extra)
     if getattr(R, "offload", False):
         # 12 B of state read and 12 B written per element cross PCIe; HBM carries the rest
