@@ -2,9 +2,10 @@
 fused kernel and the gather: D in 1..64, alignments 1..128, random tensor lists
 (ragged tails, empty tensors), all ranks or one rank, both contribution layouts,
 both reduce dtypes, misaligned buffers (scalar paths), 0..3 fused gathered blocks,
-scalars as launch arguments or in device memory; and the HYBRID_SHARD step over
-random node counts (R * D up to 64).  Every case runs two steps and compares
-every element; canary bands must stay intact."""
+scalars as launch arguments or in device memory; the HYBRID_SHARD step over
+random node counts (R * D up to 64); and its split form for separate machines
+(each node's sum, then the fold).  Every case runs two steps and compares every
+element; canary bands must stay intact."""
 import random
 
 import numpy as np
@@ -159,3 +160,56 @@ def test_fuzz_hybrid_against_oracle(z3, block):
     for k in range(25):
         seed = 50_000 + 1000 * block + k
         hybrid_case(z3, random.Random(seed), seed)
+
+
+def node_fold_case(z3, rnd: random.Random, seed: int):
+    """HYBRID_SHARD across nodes: each node's sum (zero3_node_sum), then their
+    fold (zero3_fold_adamw), against the oracle's two-level step."""
+    D = rnd.choice([1, 2, 3, 4, 5, 8, 16, 32])
+    R = rnd.randint(1, 8)
+    A = rnd.choice([1, 2, 8, 128])
+    shapes = [(rnd.randint(0, 3000),) for _ in range(rnd.randint(1, 4))]
+    plan = z3.zero3_plan(shapes, D, A)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    rank = -1 if rnd.random() < 0.5 else rnd.randrange(D)
+    layout = z3.Z3_CONTRIB_OWNED if rank >= 0 and rnd.random() < 0.5 else z3.Z3_CONTRIB_FULL
+    mode = rnd.choice([0, 1])
+    skew = [rnd.choice([0, 0, 0, 1]) for _ in range(4)]
+    n = N_pad if rank < 0 else S
+    desc = f"seed={seed} R={R} D={D} A={A} shapes={shapes} rank={rank} layout={layout} mode={mode} skew={skew}"
+    dt = torch.float32 if mode == 0 else torch.bfloat16
+    p_full = synth.master_weights(N, N_pad, seed=seed, device="cuda")
+    p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
+    gp = Guarded(n, torch.float32, skew[0], fill=p0)
+    gm = Guarded(n, torch.float32, 0, fill=torch.zeros(n, device="cuda"))
+    gv = Guarded(n, torch.float32, 0, fill=torch.zeros(n, device="cuda"))
+    gw = Guarded(n, torch.bfloat16, skew[1], fill=torch.zeros(n, device="cuda", dtype=torch.bfloat16))
+    sums = [Guarded(n, dt, skew[2]) for _ in range(R)]
+    hp_, hm, hv, hw = f32_host(p0).copy(), np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.uint16)
+    for t in (1, 2):
+        contribs = synth.contributions(R * D, N, N_pad, seed=seed, step=t, sigma=1e-3,
+                                       dist=rnd.choice(["normal", "student_t"]), zero_frac=0.02, device="cuda")
+        if layout == z3.Z3_CONTRIB_OWNED:
+            contribs = [c[rank * S:(rank + 1) * S].clone() for c in contribs]
+        gc = [Guarded(c.numel(), torch.bfloat16, skew[3], fill=c) for c in contribs]
+        for k in range(R):
+            z3.zero3_node_sum(plan, rank, [g.t for g in gc[k * D:(k + 1) * D]], sums[k].t, contrib_layout=layout,
+                              reduce_dtype=mode)
+        z3.zero3_fold_adamw(plan, rank, [g.t for g in sums], gp.t, gm.t, gv.t, gw.t, z3.adamw(**hp_for(t)),
+                            reduce_dtype=mode)
+        oracle.reduce_adamw_hybrid([synth.bf16_bits(c) for c in contribs], R, S, rank, hp_, hm, hv, hw,
+                                   oracle_hp(t), layout=layout, reduce_dtype=mode)
+        torch.cuda.synchronize()
+        assert_f32_parity(f32_host(gp.t), hp_, "master " + desc)
+        assert_f32_parity(f32_host(gm.t), hm, "exp_avg " + desc)
+        assert_f32_parity(f32_host(gv.t), hv, "exp_avg_sq " + desc)
+        assert_bf16_parity(synth.bf16_bits(gw.t), hw, "work " + desc)
+        for g in [gp, gm, gv, gw, *sums, *gc]:
+            assert g.guards_intact(), "canary " + desc
+
+
+@pytest.mark.parametrize("block", range(2))
+def test_fuzz_node_sums_then_fold_against_oracle(z3, block):
+    for k in range(25):
+        seed = 90_000 + 1000 * block + k
+        node_fold_case(z3, random.Random(seed), seed)
