@@ -268,10 +268,11 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
     return n * steps / dt, dt, desc, kept
 
 
-def sample_parity(z3, dev, kept: dict, reduce_dtype: int) -> dict:
+def sample_parity(z3, dev, kept: dict, reduce_dtype: int, split: bool = False) -> dict:
     """Our path, through the public API on the GPU, over the CPU baseline's own
     sample (the same contributions, master and steps, as rank 0's owned slice),
-    compared element by element with the oracle's results."""
+    compared element by element with the oracle's results.  split: the
+    HYBRID_SHARD reduction as node sums and their fold, as the benchmark ran it."""
     import numpy as np
     import torch
 
@@ -282,9 +283,16 @@ def sample_parity(z3, dev, kept: dict, reduce_dtype: int) -> dict:
     p = torch.from_numpy(kept["p0"]).to(dev)
     m, v = torch.zeros_like(p), torch.zeros_like(p)
     w = torch.zeros(n, dtype=torch.bfloat16, device=dev)
+    sums = ([torch.empty(n, dtype=torch.float32 if reduce_dtype == 0 else torch.bfloat16, device=dev)
+             for _ in range(nodes)] if split else None)
     for t in range(1, steps + 1):
         hp = z3.adamw(step=t)
-        if nodes > 1:
+        if split:
+            for k in range(nodes):
+                z3.zero3_node_sum(plan, 0, c[k * D:(k + 1) * D], sums[k], contrib_layout=z3.Z3_CONTRIB_OWNED,
+                                  reduce_dtype=reduce_dtype)
+            z3.zero3_fold_adamw(plan, 0, sums, p, m, v, w, hp, reduce_dtype=reduce_dtype)
+        elif nodes > 1:
             z3.zero3_reduce_adamw_hybrid(plan, 0, nodes, c, p, m, v, w, hp, contrib_layout=z3.Z3_CONTRIB_OWNED,
                                          reduce_dtype=reduce_dtype)
         else:
@@ -785,7 +793,8 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                 "host": host_info(),
                                 "seconds": secs_cpu,
-                                "parity_vs_oracle": sample_parity(z3, dev, kept, mode)}
+                                "parity_vs_oracle": sample_parity(z3, dev, kept, mode,
+                                                                  split=getattr(R, "split", False))}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
