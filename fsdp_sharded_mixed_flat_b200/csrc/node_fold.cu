@@ -96,8 +96,19 @@ __device__ __forceinline__ void node_sum8(const NodeSumArgs& a, int64_t e) {
     }
 }
 
+// Blocks per SM the node-sum kernel asks for (the register cap follows from it).
+// 3 blocks (80 registers) as in the fused kernel; the fp32 fold at 16 or more
+// ranks hoists the loads of every rank chunk and spilled under that cap, so it
+// gets 2 blocks (128 registers) at 16 ranks and 1 at 32: measured on B200 for
+// the 7B block, 6771 -> 7242 GB/s at 16 ranks, 6022 -> 6432 GB/s at 32.
 template <int MODE, int DT>
-__global__ void __launch_bounds__(kNfThreads, 3) k_node_sum_vec(const __grid_constant__ NodeSumArgs a) {
+constexpr int node_sum_min_blocks() {
+    return (MODE == Z3_REDUCE_FP32 && DT >= 32) ? 1 : (MODE == Z3_REDUCE_FP32 && DT >= 16) ? 2 : 3;
+}
+
+template <int MODE, int DT>
+__global__ void __launch_bounds__(kNfThreads, (node_sum_min_blocks<MODE, DT>()))
+    k_node_sum_vec(const __grid_constant__ NodeSumArgs a) {
     const int64_t n8 = a.n >> 3;
     const int64_t step = int64_t(gridDim.x) * kNfThreads;
     for (int64_t q = int64_t(blockIdx.x) * kNfThreads + threadIdx.x; q < n8; q += step) node_sum8<MODE, DT>(a, q << 3);
