@@ -7,7 +7,6 @@ Every function of the oracle has at least one pin here; a plausible mistake
 (a dropped rank, a wrong slice index, a missing 1/D, a flipped sign, a missing
 bias correction, coupled weight decay, a wrong pad) fails at least one test.
 """
-import math
 import random
 from fractions import Fraction
 
