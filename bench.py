@@ -83,6 +83,8 @@ def parse_args():
     ap.add_argument("--drift", action="store_true",
                     help="report the drift of the bf16-reduce path against the fp32-reduce path")
     ap.add_argument("--drift-elements", type=int, default=1 << 24)
+    ap.add_argument("--nodes", type=int, default=0,
+                    help="HYBRID_SHARD workload: number of nodes (default: the workload's)")
     ap.add_argument("--split", action="store_true",
                     help="HYBRID_SHARD workload: the node sums of every node, then their fold (two kernels, what "
                          "separate machines run) instead of the fused kernel")
@@ -230,7 +232,7 @@ def oracle_workload(workload: str) -> str:
 
 
 def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int = 0, reduce_dtype: int = 0,
-                  keep: bool = False):
+                  keep: bool = False, nodes: int = 0):
     """Time the oracle over `steps` passes of a `sample`-element slice of the
     workload's owned elements (all D contributions, AdamW, cast).  Returns
     (owned params/s, seconds, description, kept), where kept holds the sample's
@@ -242,7 +244,7 @@ def oracle_sample(workload: str, sample: int, steps: int, seed: int = 0, D: int 
     workload = oracle_workload(workload)
     w = synth.WORKLOADS[workload]
     D = D or w["D"]
-    nodes = w.get("nodes", 1)
+    nodes = nodes or w.get("nodes", 1)
     n = min(sample, synth.block_numel(w["tensors"]))
     contribs = [synth.bf16_bits(synth.contribution(n, n, seed=seed, step=1, rank=d, sigma=w["sigma"],
                                                    dist=w["dist"], zero_frac=w.get("zero_frac", 0.0),
@@ -351,7 +353,7 @@ class BlockRunner:
     the replicated bf16 weights (the flat block), with no separate shard."""
 
     def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
-                 graph=False, offload=False, split=False):
+                 graph=False, offload=False, split=False, nodes=0):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
@@ -361,7 +363,9 @@ class BlockRunner:
         plan = z3.zero3_plan(self.shapes, D, synth.ALIGN)
         self.N, self.N_pad, self.S = plan.N, plan.N_pad, plan.S
         # HYBRID_SHARD: `nodes` nodes of D ranks, contribution k*D + d from rank d of node k
-        self.nodes = w.get("nodes", 1)
+        self.nodes = nodes or w.get("nodes", 1)
+        if nodes and "nodes" not in w:
+            raise SystemExit("--nodes needs a HYBRID_SHARD workload (llama7b_hybrid)")
         if self.nodes > 1 and (stage != 3 or graph or offload):
             raise SystemExit("the HYBRID_SHARD workload runs the plain ZeRO-3 block step")
         if split and self.nodes == 1:
@@ -665,7 +669,7 @@ def run_ours(args):
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
                         stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph,
-                        offload=args.offload, split=args.split)
+                        offload=args.offload, split=args.split, nodes=args.nodes)
     stream = R.stream
 
     for _ in range(args.warmup):
@@ -785,11 +789,12 @@ def run_ours(args):
         line["roofline"]["traffic"] = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # calibrate on a small slice, then size the step count for about 10 s of oracle work
-        rate, _, _, _ = oracle_sample(args.workload, 1 << 16, 1, D=R.D, reduce_dtype=mode)
+        nodes = getattr(R, "nodes", 1)
+        rate, _, _, _ = oracle_sample(args.workload, 1 << 16, 1, D=R.D, reduce_dtype=mode, nodes=nodes)
         n_cpu = min(args.cpu_sample, synth.block_numel(synth.WORKLOADS[oracle_workload(args.workload)]["tensors"]))
         cpu_steps = max(1, min(args.cpu_steps, round(10.0 * rate / max(1, n_cpu))))
         v, secs_cpu, desc, kept = oracle_sample(args.workload, args.cpu_sample, cpu_steps, D=R.D,
-                                                reduce_dtype=mode, keep=True)
+                                                reduce_dtype=mode, keep=True, nodes=nodes)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                 "host": host_info(),
                                 "seconds": secs_cpu,

@@ -66,7 +66,9 @@ def run_small(z3, numels, R, D, A, rank, layout, mode, steps=6, seed=0, skew=0):
 
 
 SMALL = [
-    ([123457], 4, 8, 128),        # the specialised kernel: 4 nodes of 8
+    ([123457], 4, 8, 128),        # the specialised kernels: 2, 4 and 8 nodes of 8
+    ([60001, 7], 2, 8, 128),
+    ([30011], 8, 8, 8),
     ([5000, 77], 4, 8, 1),        # ... with a ragged tail
     ([3000, 17], 2, 3, 8),        # generic kernel
     ([20001], 3, 5, 1),
