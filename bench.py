@@ -57,6 +57,16 @@ K1_SOURCE = os.path.join(ROOT, "fsdp_sharded_mixed_flat_b200", "csrc", "reduce_a
 SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
+# How the 70B shard's per-layer contributions arrive in a transient buffer (the
+# reduce-scatter's delivery, simulated on one GPU).
+ARRIVALS = {
+    "copy": "device-to-device copy from a pool on the copy stream (read + write)",
+    "fill": "write-only fill of the transient buffer on the copy stream, as a delivery over NVLink writes it",
+    "fill_prio": "write-only fill on the copy stream, the fused kernel's stream at a higher priority",
+}
+DEFAULT_ARRIVAL = "fill"
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -73,9 +83,13 @@ def parse_args():
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
     ap.add_argument("--offload", action="store_true",
                     help="fp32 master / m / v in page-locked host memory, reached by the kernel over PCIe")
-    ap.add_argument("--refill", choices=["copy", "fill"], default="copy",
-                    help="70B shard: each layer's contributions arrive by a device-to-device copy from a "
-                         "pool (read + write) or by a write-only fill of the transient buffer")
+    ap.add_argument("--refill", choices=list(ARRIVALS), default=DEFAULT_ARRIVAL,
+                    help="70B shard: how each layer's contributions arrive in the transient buffer: "
+                         + "; ".join(f"{k}: {v}" for k, v in ARRIVALS.items()))
+    ap.add_argument("--sweep-steps", type=int, default=10,
+                    help="timed steps per configuration in the sweep of the target configurations")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the sweep of the target configurations (one GPU only)")
     ap.add_argument("--graph", action="store_true",
                     help="capture the step's launches in a CUDA graph once and replay it every step")
     ap.add_argument("--unflatten-copy", action="store_true",
@@ -567,7 +581,7 @@ class ShardRunner:
     owned contributions stream in last to first through two transient buffers
     (copy stream) while the fused kernel runs on the other buffer."""
 
-    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, refill="copy"):
+    def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, refill=DEFAULT_ARRIVAL):
         import torch
         from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
         w = synth.WORKLOADS["llama70b_layer"]
@@ -584,8 +598,11 @@ class ShardRunner:
         # the refill source: two layers' worth of owned contributions (what the reduce-scatter delivers)
         self.pool = [torch.cat([synth.contribution(S, S, seed=seed, step=1, rank=d, sigma=w["sigma"], device=dev)
                                 for d in range(D)]) for _ in range(2)]
+        if refill not in ARRIVALS:
+            raise SystemExit(f"unknown arrival {refill}")
+        hi = torch.cuda.Stream.priority_range()[1] if refill == "fill_prio" else 0   # (low, high)
         self.streamer = LayerStreamer(plan, L, 0, self.master, self.exp_avg, self.exp_avg_sq, self.work,
-                                      reduce_dtype=reduce_dtype)
+                                      reduce_dtype=reduce_dtype, compute_priority=hi)
         self.stream = torch.cuda.current_stream(dev)
         self.step_no = 0
         self.units_per_step = L * S                            # owned params of this rank
@@ -599,12 +616,13 @@ class ShardRunner:
         self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}> (owned layout)"
         self.source = lambda l: self.pool[l & 1]
         # write-only refill: the transient buffer receives a value, as an NVLink delivery would write it
-        self.fill = (lambda l, buf: buf.fill_(1e-4 * (1 + (l & 7)))) if refill == "fill" else None
+        self.fill = (lambda l, buf: buf.fill_(1e-4 * (1 + (l & 7)))) if refill != "copy" else None
+        self.arrival_desc = f"{refill}: {ARRIVALS[refill]}"
         self.desc = (f"rank 0's resident shard of 80 LLaMA-70B-shaped layers ({len(w['tensors'])} tensors, "
                      f"855,654,400 params each), D={D}, S={S} per layer, {L * S} owned params "
                      f"({L * S * 14 / 1e9:.1f} GB of master+m+v+bf16); per step the 80 layers' owned bf16 "
                      f"contributions ({2 * D * S / 1e9:.2f} GB each) stream 79->0 through two transient buffers "
-                     f"({'device-to-device copy from a pool' if refill == 'copy' else 'write-only fill'} "
+                     f"({ARRIVALS[refill]}) "
                      f"on a copy stream) while the fused kernel runs")
 
     def hp(self):
@@ -635,6 +653,100 @@ class ShardRunner:
         # contributions come from pinned host memory layer by layer; layer 0's bf16 shard goes back
         self.streamer.step(lambda l: self.host_pool[l & 1], self.hp())
         self.host_out.copy_(self.work[:self.S], non_blocking=True)
+
+
+def time_runner(R, steps: int, warmup: int, dev, clocks=None, barrier=None, step=None):
+    """W untimed warm-up steps, then `steps` steps timed with CUDA events on the
+    runner's stream between synchronisations (and barriers, with several ranks);
+    the fused kernel is timed launch by launch with its own events.  Returns
+    (seconds of the timed steps, mean seconds per fused-kernel launch)."""
+    import torch
+    step = step or R.step
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if clocks is not None:
+        clocks.start()
+    k1_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(R.k1_launches_per_step)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if barrier is not None:
+        barrier()
+    torch.cuda.synchronize(dev)
+    t0.record(R.stream)
+    for i in range(steps):
+        step(k1_ev[i])
+    t1.record(R.stream)
+    torch.cuda.synchronize(dev)
+    if barrier is not None:
+        barrier()
+    secs = t0.elapsed_time(t1) / 1e3
+    k1_ms = [a.elapsed_time(b) for step_ev in k1_ev for a, b in step_ev]
+    return secs, statistics.mean(k1_ms) / 1e3
+
+
+# The target configurations besides the headline: (key, workload, D).  Each is
+# measured in both reduce dtypes by config_sweep.
+SWEEP_BLOCKS = [("config1_llama7b_d8", "llama7b_d8", 8), ("config2_llama7b_d32", "llama7b_d32", 32),
+                ("config3_policy_D2", "llama7b_policy", 2), ("config3_policy_D4", "llama7b_policy", 4),
+                ("config3_policy_D8", "llama7b_policy", 8), ("config3_policy_D16", "llama7b_policy", 16)]
+NOMINAL_HBM_GBS = 8000.0
+
+
+def config_sweep(z3, synth, dev, steps: int, warmup: int, hbm_peak: float, refill: str) -> dict:
+    """Every target configuration on this GPU, with fewer steps than the headline:
+    the fused kernel's own time, rate and fraction of peak, and the whole step's
+    owned params/s (plan + fused kernel + gather for a block; the 80-layer
+    streamed step for the 70B shard).  Target: the fused kernel at >= 80 % of
+    nominal 8 TB/s, i.e. 6.4e12 / (2D + 26) owned params/s."""
+    import torch
+    out = {}
+    for key, workload, D in SWEEP_BLOCKS:
+        entry = {}
+        for name, mode in (("fp32", z3.Z3_REDUCE_FP32), ("bf16", z3.Z3_REDUCE_BF16)):
+            R = BlockRunner(z3, synth, workload, D, mode, 2000, dev)
+            secs, k1 = time_runner(R, steps, warmup, dev)
+            gbs = R.k1_bytes_per_launch / k1 / 1e9
+            target = 0.8 * NOMINAL_HBM_GBS * 1e9 / (2 * D + 26)
+            entry[name] = {"k1_ms": 1e3 * k1, "k1_gbs": gbs, "k1_owned_params_per_s": R.units_per_step / k1,
+                           "k1_frac": gbs / hbm_peak, "k1_frac_of_nominal_8000": gbs / NOMINAL_HBM_GBS,
+                           "target_k1_owned_params_per_s": target,
+                           "meets_80pct_of_nominal": R.units_per_step / k1 >= target,
+                           "step_ms": 1e3 * secs / steps, "step_owned_params_per_s": R.units_per_step * steps / secs}
+            del R
+            torch.cuda.empty_cache()
+        entry["workload"] = workload
+        entry["D"] = D
+        entry["bytes_per_owned_param"] = 2 * D + 26
+        out[key] = entry
+    # config 4: one rank's 80-layer 70B shard, streamed through two transient buffers
+    S4 = ShardRunner(z3, synth, "llama70b_shard", 8, z3.Z3_REDUCE_FP32, 2000, dev, refill=refill)
+    shard_steps = max(2, steps // 5)
+    secs, k1 = time_runner(S4, shard_steps, 1, dev)
+    ip_secs, ip_k1 = time_runner(S4, shard_steps, 1, dev, step=S4.step_in_place)
+    step_s = secs / shard_steps
+    k1_bytes = S4.L * S4.k1_bytes_per_launch
+    target = 0.8 * NOMINAL_HBM_GBS * 1e9 / 42
+    out["config4_llama70b_shard"] = {
+        "workload": "llama70b_shard", "D": 8, "layers": S4.L, "owned_params_per_step": S4.units_per_step,
+        "streamed": {"arrival": S4.arrival_desc, "step_ms": 1e3 * step_s,
+                     "step_owned_params_per_s": S4.units_per_step / step_s,
+                     "k1_ms_per_layer": 1e3 * k1, "k1_gbs": S4.k1_bytes_per_launch / k1 / 1e9,
+                     "k1_frac": S4.k1_bytes_per_launch / k1 / 1e9 / hbm_peak,
+                     "step_hbm_gbs": (k1_bytes + S4.refill_bytes) / step_s / 1e9,
+                     "arrival_bytes_per_step": S4.refill_bytes},
+        "in_place": {"step_ms": 1e3 * ip_secs / shard_steps,
+                     "step_owned_params_per_s": S4.units_per_step * shard_steps / ip_secs,
+                     "k1_ms_per_layer": 1e3 * ip_k1, "k1_gbs": S4.k1_bytes_per_launch / ip_k1 / 1e9,
+                     "k1_frac": S4.k1_bytes_per_launch / ip_k1 / 1e9 / hbm_peak,
+                     "k1_owned_params_per_s": S4.S / ip_k1,
+                     "meets_80pct_of_nominal": S4.S / ip_k1 >= target,
+                     "note": "the same 80 fused-kernel launches reading the contributions where they lie: the "
+                             "kernel's own rate, without the arrival of the next layer's bytes"},
+        "target_k1_owned_params_per_s": target, "steps": shard_steps}
+    del S4
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -672,31 +784,12 @@ def run_ours(args):
                         offload=args.offload, split=args.split, nodes=args.nodes)
     stream = R.stream
 
-    for _ in range(args.warmup):
-        R.step()
-    torch.cuda.synchronize(dev)
-
     props = torch.cuda.get_device_properties(dev)
     uuid = getattr(props, "uuid", None)
     clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else None)
-    clocks.start()
-    k1_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(R.k1_launches_per_step)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    t0.record(stream)
-    for i in range(args.steps):
-        R.step(k1_ev[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
+    secs, k1_avg_s = time_runner(R, args.steps, args.warmup, dev, clocks=clocks,
+                                 barrier=dist.barrier if world > 1 else None)
     clk = clocks.stop()
-    secs = t0.elapsed_time(t1) / 1e3
-    k1_ms = [a.elapsed_time(b) for step_ev in k1_ev for a, b in step_ev]
-    k1_avg_s = statistics.mean(k1_ms) / 1e3
     job_secs, job_units = aggregate(secs, float(R.units_per_step) * args.steps, world, dev)
     value = job_units / job_secs
 
@@ -787,19 +880,33 @@ def run_ours(args):
                                    "is bound by PCIe, not HBM, so the hbm roofline fields describe the kernels "
                                    "on the staged device buffers only"}
         line["roofline"]["traffic"] = None
+    run_D, run_nodes, run_split = R.D, getattr(R, "nodes", 1), getattr(R, "split", False)
+    if world == 1 and not args.no_sweep and args.workload == "llama7b_d8" and args.stage == 3 and \
+            not (args.graph or args.offload or args.unflatten_copy):
+        # every target configuration, on the same GPU after the headline (whose buffers are freed first)
+        R.__dict__.clear()
+        del R
+        torch.cuda.empty_cache()
+        sweep_clocks = ClockSampler(f"GPU-{uuid}" if uuid is not None else None)
+        sweep_clocks.start()
+        line["configs"] = config_sweep(z3, synth, dev, args.sweep_steps, max(3, min(args.warmup, 5)), hbm_peak,
+                                       args.refill)
+        line["configs"]["clocks"] = sweep_clocks.stop()
+        line["configs"]["note"] = ("the fused kernel (K1) of every target configuration timed alone with CUDA events "
+                                   "over %d steps after warm-up, both reduce dtypes; target: K1 at >= 80 %% of "
+                                   "nominal 8 TB/s; k1_frac is of the measured copy peak" % args.sweep_steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # calibrate on a small slice, then size the step count for about 10 s of oracle work
-        nodes = getattr(R, "nodes", 1)
-        rate, _, _, _ = oracle_sample(args.workload, 1 << 16, 1, D=R.D, reduce_dtype=mode, nodes=nodes)
+        nodes = run_nodes
+        rate, _, _, _ = oracle_sample(args.workload, 1 << 16, 1, D=run_D, reduce_dtype=mode, nodes=nodes)
         n_cpu = min(args.cpu_sample, synth.block_numel(synth.WORKLOADS[oracle_workload(args.workload)]["tensors"]))
         cpu_steps = max(1, min(args.cpu_steps, round(10.0 * rate / max(1, n_cpu))))
-        v, secs_cpu, desc, kept = oracle_sample(args.workload, args.cpu_sample, cpu_steps, D=R.D,
+        v, secs_cpu, desc, kept = oracle_sample(args.workload, args.cpu_sample, cpu_steps, D=run_D,
                                                 reduce_dtype=mode, keep=True, nodes=nodes)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                 "host": host_info(),
                                 "seconds": secs_cpu,
-                                "parity_vs_oracle": sample_parity(z3, dev, kept, mode,
-                                                                  split=getattr(R, "split", False))}
+                                "parity_vs_oracle": sample_parity(z3, dev, kept, mode, split=run_split)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -19,10 +19,14 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libzero3.so")
 
-SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "node_fold.cu", "gather.cu"]
+SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "node_fold.cu", "gather.cu", "host_adamw.cpp"]
+# per-source host-compiler flags: the host optimiser must round every operation
+# on its own (no contraction into fused multiply-adds); -fno-math-errno only
+# drops errno bookkeeping around sqrt, so the loop vectorises
+EXTRA_FLAGS = {"host_adamw.cpp": ["-Xcompiler", "-ffp-contract=off,-fno-math-errno,-fno-fast-math"]}
 EXPORTS = os.path.join(CSRC, "exports.map")
-HEADERS = [os.path.join(CSRC, "plan_impl.h"), os.path.join(CSRC, "step_common.cuh"), os.path.join(INCLUDE, "zero3.h"),
-           EXPORTS]
+HEADERS = [os.path.join(CSRC, "plan_impl.h"), os.path.join(CSRC, "step_common.cuh"),
+           os.path.join(CSRC, "adamw_scalars.h"), os.path.join(INCLUDE, "zero3.h"), EXPORTS]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xptxas", "-v",
@@ -54,7 +58,7 @@ def build(force: bool = False, quiet: bool = True) -> str:
     objs, logs = [], []
     for src in SOURCES:
         obj = os.path.join(OUT_DIR, src + ".o")
-        cmd = [nvcc(), *NVCC_FLAGS, "-c", os.path.join(CSRC, src), "-o", obj]
+        cmd = [nvcc(), *NVCC_FLAGS, *EXTRA_FLAGS.get(src, []), "-c", os.path.join(CSRC, src), "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         logs.append(f"$ {' '.join(cmd)}\n{r.stdout}{r.stderr}")
         if r.returncode != 0:

@@ -8,7 +8,8 @@
 //
 // Both kernels are pure copies bound by HBM bandwidth (2 bytes read + 2 bytes
 // written per element).
-//   - flat copy: grid.y = rank, grid.x covering the shard (2 independent
+//   - flat copy: grid.y = one row per shard to copy (a shard already in place
+//     inside the block is skipped), grid.x covering the shard (2 independent
 //     16-byte vectors per thread, consecutive threads on consecutive vectors),
 //     so the block scheduler balances the SMs; streaming stores.
 //   - per-tensor copy: the host cuts every tensor into segments, one per rank
@@ -40,7 +41,8 @@ constexpr int64_t kMaxBlocks = 1 << 30;   // grid.x cap; beyond it the kernels l
 constexpr int kSegMax = 100;  // segments per launch; keeps the parameter block under 4 KB
 
 struct FlatArgs {
-    const uint16_t* shard[Z3_D_MAX];
+    const uint16_t* shard[Z3_D_MAX];  // the shards to copy, in grid.y order
+    int32_t rank[Z3_D_MAX];           // the partition each of them fills
     uint16_t* flat;
     int64_t S;
 };
@@ -62,9 +64,9 @@ struct SegArgs {
 static_assert(sizeof(SegArgs) <= 4096, "segment table must fit the 4 KB parameter block");
 
 __global__ void __launch_bounds__(kThreads) k_gather_flat_vec(const __grid_constant__ FlatArgs a) {
-    const int r = blockIdx.y;
-    const uint4* src = reinterpret_cast<const uint4*>(a.shard[r]);
-    uint4* dst = reinterpret_cast<uint4*>(a.flat + int64_t(r) * a.S);
+    const int y = blockIdx.y;
+    const uint4* src = reinterpret_cast<const uint4*>(a.shard[y]);
+    uint4* dst = reinterpret_cast<uint4*>(a.flat + int64_t(a.rank[y]) * a.S);
     const int64_t n = a.S >> 3;
     const int64_t span = int64_t(kThreads) * kUnroll;
     for (int64_t i = int64_t(blockIdx.x) * span + threadIdx.x; i < n; i += int64_t(gridDim.x) * span) {
@@ -79,9 +81,9 @@ __global__ void __launch_bounds__(kThreads) k_gather_flat_vec(const __grid_const
 }
 
 __global__ void __launch_bounds__(kThreads) k_gather_flat_scalar(const __grid_constant__ FlatArgs a) {
-    const int r = blockIdx.y;
-    const uint16_t* src = a.shard[r];
-    uint16_t* dst = a.flat + int64_t(r) * a.S;
+    const int y = blockIdx.y;
+    const uint16_t* src = a.shard[y];
+    uint16_t* dst = a.flat + int64_t(a.rank[y]) * a.S;
     const int64_t stride = int64_t(gridDim.x) * kThreads;
     for (int64_t j = int64_t(blockIdx.x) * kThreads + threadIdx.x; j < a.S; j += stride) dst[j] = src[j];
 }
@@ -182,9 +184,13 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
     if (tensor_out != nullptr)
         for (int32_t i = 0; i < nt; ++i)
             if (tensor_out[i] != nullptr && !z3::aligned(tensor_out[i], 2)) return Z3_EALIGN;
-    // outputs overlap neither the shards nor each other
+    // Shard r may sit in place inside the block, at exactly flat_out + r*S (a
+    // rank's own shard as a view of its gathered block, the usual FSDP layout):
+    // that partition is already where it belongs and is not copied.  Otherwise
+    // outputs overlap neither the shards nor each other.
+    auto in_place = [&](int32_t r) { return flat_out != nullptr && shards[r] == flat_out + int64_t(r) * S; };
     for (int32_t r = 0; r < D; ++r) {
-        if (flat_out && z3::overlaps(flat_out, p->N_pad * 2, shards[r], S * 2)) return Z3_EINVAL;
+        if (flat_out && !in_place(r) && z3::overlaps(flat_out, p->N_pad * 2, shards[r], S * 2)) return Z3_EINVAL;
         if (tensor_out)
             for (int32_t i = 0; i < nt; ++i)
                 if (tensor_out[i] && z3::overlaps(tensor_out[i], p->numel[i] * 2, shards[r], S * 2))
@@ -209,13 +215,24 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
     bool vec_src = (S % 8) == 0;
     for (int32_t r = 0; r < D; ++r) vec_src = vec_src && z3::aligned(shards[r], 16);
 
-    // ---- the all-gather into the flat block
-    if (flat_out != nullptr) {
-        FlatArgs a;
-        for (int32_t r = 0; r < Z3_D_MAX; ++r) a.shard[r] = r < D ? shards[r] : nullptr;
+    // ---- the all-gather into the flat block: one grid row per shard not already in place
+    FlatArgs a;
+    int32_t n_copy = 0;
+    bool vec = (S % 8) == 0 && flat_out != nullptr && z3::aligned(flat_out, 16);
+    for (int32_t r = 0; r < D; ++r) {
+        if (flat_out == nullptr || in_place(r)) continue;
+        a.shard[n_copy] = shards[r];
+        a.rank[n_copy] = r;
+        vec = vec && z3::aligned(shards[r], 16);
+        ++n_copy;
+    }
+    if (n_copy > 0) {
+        for (int32_t k = n_copy; k < Z3_D_MAX; ++k) {
+            a.shard[k] = nullptr;
+            a.rank[k] = 0;
+        }
         a.flat = flat_out;
         a.S = S;
-        const bool vec = vec_src && z3::aligned(flat_out, 16);
         auto fn = vec ? k_gather_flat_vec : k_gather_flat_scalar;
         int64_t bx;
         if (vec) {
@@ -226,10 +243,10 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
             if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0) != cudaSuccess || per_sm < 1)
                 per_sm = 1;
             bx = (S + kThreads - 1) / kThreads;
-            const int64_t cap = std::max<int64_t>(1, (int64_t(sms) * per_sm + D - 1) / D);
+            const int64_t cap = std::max<int64_t>(1, (int64_t(sms) * per_sm + n_copy - 1) / n_copy);
             bx = std::max<int64_t>(1, std::min(bx, cap));
         }
-        fn<<<dim3(unsigned(bx), unsigned(D)), dim3(kThreads), 0, stream>>>(a);
+        fn<<<dim3(unsigned(bx), unsigned(n_copy)), dim3(kThreads), 0, stream>>>(a);
         if (cudaGetLastError() != cudaSuccess) return Z3_ECUDA;
     }
 

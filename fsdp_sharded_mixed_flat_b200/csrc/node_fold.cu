@@ -11,6 +11,11 @@
 //                 left to right in rank order, not scaled; written as fp32
 //                 (fp32 reduce) or bf16 (bf16 reduce, every partial sum
 //                 rounded).  Reads 2*D bytes, writes 4 (or 2) per element.
+//                 The same kernel with the 1/D scale is the reduce-scatter's
+//                 reduction alone (zero3_reduce_scatter): the averaged gradient
+//                 of the owned partition, for the CPU-offload step, whose
+//                 optimiser runs on the host ("7.10 — Fully-sharded data
+//                 parallel (FSDP / ZeRO-3)", §8).
 //   k_fold_adamw: the R node sums folded in node order, times fp32(1/(R*D)),
 //                 AdamW on the owned fp32 master / m / v and the bf16 cast.
 //                 Reads 4*R (or 2*R) + 12 bytes, writes 14 per element.
@@ -40,6 +45,7 @@ struct NodeSumArgs {
     void* out;                    // n node sums: float (fp32 reduce) or bf16 bits (bf16 reduce)
     int64_t n;
     int32_t D;
+    float inv_n;                  // SCALE kernels: fp32 nearest to 1/D
 };
 
 struct FoldArgs {
@@ -55,17 +61,21 @@ struct FoldArgs {
 };
 
 // ---------------------------------------------------------------- node sums
-template <int MODE>
+// SCALE = false: the node's unscaled sum.  SCALE = true: the reduce-scatter's
+// averaged gradient, the sum times fp32(1/D) (rounded to bf16 in the bf16
+// reduce), exactly the g the fused kernel hands to AdamW.
+template <int MODE, bool SCALE>
 __device__ __forceinline__ void node_sum1(const NodeSumArgs& a, int64_t i) {
     float acc = bf16_of(a.c[0][i]);
     for (int d = 1; d < a.D; ++d) acc = add_in<MODE>(acc, bf16_of(a.c[d][i]));
+    if constexpr (SCALE) acc = __fmul_rn(acc, a.inv_n);
     if constexpr (MODE == Z3_REDUCE_FP32)
         static_cast<float*>(a.out)[i] = acc;
-    else
-        static_cast<uint16_t*>(a.out)[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));  // exact: acc is bf16
+    else  // nearest-even: exact for the unscaled sum (already bf16), the rounding of g when scaled
+        static_cast<uint16_t*>(a.out)[i] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
 }
 
-template <int MODE, int DT>
+template <int MODE, int DT, bool SCALE>
 __device__ __forceinline__ void node_sum8(const NodeSumArgs& a, int64_t e) {
     const int D = DT > 0 ? DT : a.D;
     float acc[8];
@@ -87,10 +97,19 @@ __device__ __forceinline__ void node_sum8(const NodeSumArgs& a, int64_t e) {
         }
     }
     if constexpr (MODE == Z3_REDUCE_FP32) {
+        if constexpr (SCALE) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = __fmul_rn(acc[k], a.inv_n);
+        }
         float* o = static_cast<float*>(a.out) + e;
         st16(reinterpret_cast<float4*>(o), make_float4(acc[0], acc[1], acc[2], acc[3]));
         st16(reinterpret_cast<float4*>(o + 4), make_float4(acc[4], acc[5], acc[6], acc[7]));
     } else {
+        if constexpr (SCALE) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                accw[k] = pack_bf16x2(__fmul_rn(lo_bf16(accw[k]), a.inv_n), __fmul_rn(hi_bf16(accw[k]), a.inv_n));
+        }
         st16(reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + e),
              make_uint4(accw[0], accw[1], accw[2], accw[3]));
     }
@@ -106,20 +125,22 @@ constexpr int node_sum_min_blocks() {
     return (MODE == Z3_REDUCE_FP32 && DT >= 32) ? 1 : (MODE == Z3_REDUCE_FP32 && DT >= 16) ? 2 : 3;
 }
 
-template <int MODE, int DT>
+template <int MODE, int DT, bool SCALE>
 __global__ void __launch_bounds__(kNfThreads, (node_sum_min_blocks<MODE, DT>()))
     k_node_sum_vec(const __grid_constant__ NodeSumArgs a) {
     const int64_t n8 = a.n >> 3;
     const int64_t step = int64_t(gridDim.x) * kNfThreads;
-    for (int64_t q = int64_t(blockIdx.x) * kNfThreads + threadIdx.x; q < n8; q += step) node_sum8<MODE, DT>(a, q << 3);
+    for (int64_t q = int64_t(blockIdx.x) * kNfThreads + threadIdx.x; q < n8; q += step)
+        node_sum8<MODE, DT, SCALE>(a, q << 3);
     const int64_t tail = (n8 << 3) + int64_t(blockIdx.x) * kNfThreads + threadIdx.x;
-    if (tail < a.n) node_sum1<MODE>(a, tail);
+    if (tail < a.n) node_sum1<MODE, SCALE>(a, tail);
 }
 
-template <int MODE>
+template <int MODE, bool SCALE>
 __global__ void __launch_bounds__(kNfThreads) k_node_sum_scalar(const __grid_constant__ NodeSumArgs a) {
     const int64_t stride = int64_t(gridDim.x) * kNfThreads;
-    for (int64_t i = int64_t(blockIdx.x) * kNfThreads + threadIdx.x; i < a.n; i += stride) node_sum1<MODE>(a, i);
+    for (int64_t i = int64_t(blockIdx.x) * kNfThreads + threadIdx.x; i < a.n; i += stride)
+        node_sum1<MODE, SCALE>(a, i);
 }
 
 // ---------------------------------------------------- fold of the node sums
@@ -215,17 +236,17 @@ __global__ void __launch_bounds__(kNfThreads) k_fold_adamw_scalar(const __grid_c
 using NodeSumFn = void (*)(NodeSumArgs);
 using FoldFn = void (*)(FoldArgs);
 
-template <int MODE>
+template <int MODE, bool SCALE>
 NodeSumFn pick_node_sum(bool vec, int D) {
-    if (!vec) return k_node_sum_scalar<MODE>;
+    if (!vec) return k_node_sum_scalar<MODE, SCALE>;
     switch (D) {
-    case 1: return k_node_sum_vec<MODE, 1>;
-    case 2: return k_node_sum_vec<MODE, 2>;
-    case 4: return k_node_sum_vec<MODE, 4>;
-    case 8: return k_node_sum_vec<MODE, 8>;
-    case 16: return k_node_sum_vec<MODE, 16>;
-    case 32: return k_node_sum_vec<MODE, 32>;
-    default: return k_node_sum_vec<MODE, 0>;
+    case 1: return k_node_sum_vec<MODE, 1, SCALE>;
+    case 2: return k_node_sum_vec<MODE, 2, SCALE>;
+    case 4: return k_node_sum_vec<MODE, 4, SCALE>;
+    case 8: return k_node_sum_vec<MODE, 8, SCALE>;
+    case 16: return k_node_sum_vec<MODE, 16, SCALE>;
+    case 32: return k_node_sum_vec<MODE, 32, SCALE>;
+    default: return k_node_sum_vec<MODE, 0, SCALE>;
     }
 }
 
@@ -263,9 +284,11 @@ int64_t grid_for(Fn fn, bool vec, int64_t n) {
 
 }  // namespace
 
-extern "C" Z3_API int zero3_node_sum(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
-                                     int32_t contrib_layout, int32_t reduce_dtype, void* node_sum,
-                                     void* cuda_stream) {
+namespace {
+
+// zero3_node_sum (scale = false) and zero3_reduce_scatter (scale = true).
+int launch_node_sum(const z3_plan* p, int32_t rank, const uint16_t* const* contrib, int32_t contrib_layout,
+                    int32_t reduce_dtype, void* node_sum, bool scale, void* cuda_stream) {
     if (p == nullptr || contrib == nullptr || node_sum == nullptr) return Z3_EINVAL;
     const int32_t D = p->D;
     if (rank < -1 || rank >= D) return Z3_EINVAL;
@@ -288,17 +311,37 @@ extern "C" Z3_API int zero3_node_sum(const z3_plan* p, int32_t rank, const uint1
     a.out = node_sum;
     a.n = n;
     a.D = D;
+    a.inv_n = float(1.0 / double(D));
     bool vec = z3::aligned(node_sum, 16);
     for (int32_t d = 0; d < Z3_D_MAX; ++d) {
         a.c[d] = d < D ? contrib[d] + c_off : nullptr;
         if (d < D && !z3::aligned(a.c[d], 16)) vec = false;
     }
-    const NodeSumFn fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_node_sum<Z3_REDUCE_FP32>(vec, D)
-                                                        : pick_node_sum<Z3_REDUCE_BF16>(vec, D);
+    NodeSumFn fn;
+    if (scale)
+        fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_node_sum<Z3_REDUCE_FP32, true>(vec, D)
+                                            : pick_node_sum<Z3_REDUCE_BF16, true>(vec, D);
+    else
+        fn = reduce_dtype == Z3_REDUCE_FP32 ? pick_node_sum<Z3_REDUCE_FP32, false>(vec, D)
+                                            : pick_node_sum<Z3_REDUCE_BF16, false>(vec, D);
     const int64_t blocks = grid_for(fn, vec, n);
     if (blocks < 1) return Z3_ECUDA;
     fn<<<dim3(unsigned(blocks)), dim3(kNfThreads), 0, static_cast<cudaStream_t>(cuda_stream)>>>(a);
     return cudaGetLastError() == cudaSuccess ? Z3_OK : Z3_ECUDA;
+}
+
+}  // namespace
+
+extern "C" Z3_API int zero3_node_sum(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                     int32_t contrib_layout, int32_t reduce_dtype, void* node_sum,
+                                     void* cuda_stream) {
+    return launch_node_sum(p, rank, contrib, contrib_layout, reduce_dtype, node_sum, false, cuda_stream);
+}
+
+extern "C" Z3_API int zero3_reduce_scatter(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                           int32_t contrib_layout, int32_t reduce_dtype, void* grad,
+                                           void* cuda_stream) {
+    return launch_node_sum(p, rank, contrib, contrib_layout, reduce_dtype, grad, true, cuda_stream);
 }
 
 extern "C" Z3_API int zero3_fold_adamw(const z3_plan* p, int32_t rank, int32_t n_nodes, const void* const* node_sums,

@@ -1,6 +1,6 @@
 // step_common.cuh -- the pieces every optimiser-step kernel of this library
-// shares: the AdamW scalars and their host computation, the AdamW element
-// update, the bf16 conversions and the 16-byte memory accesses.
+// shares: the AdamW element update (its scalars come from adamw_scalars.h),
+// the bf16 conversions and the 16-byte memory accesses.
 //
 // Pages: "7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)", §3 (rank r
 // updates P_r from its fp32 master, m, v and gradient slice); "Building GPT
@@ -21,46 +21,10 @@
 #include <cmath>
 #include <cstdint>
 
+#include "adamw_scalars.h"
 #include "zero3.h"
 
 namespace {
-
-// The eight fp32 scalars of one AdamW step, in the order the C ABI documents
-// for zero3_step_scalars.
-struct AdamScalars {
-    float step_size;     // lr / (1 - b1^t)
-    float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
-    float decay;         // 1 - lr * wd
-    float b1, omb1, b2, omb2, eps;
-};
-
-static_assert(sizeof(AdamScalars) == Z3_SCALARS * sizeof(float), "scalar layout");
-
-// Host computation of one step's scalars: binary64, each rounded to fp32 once.
-inline AdamScalars step_scalars(const z3_adamw* hp) {
-    AdamScalars s;
-    const double t = double(hp->step);
-    const double bc1 = 1.0 - std::pow(hp->beta1, t);
-    const double bc2 = 1.0 - std::pow(hp->beta2, t);
-    s.step_size = float(hp->lr / bc1);
-    s.inv_sqrt_bc2 = float(1.0 / std::sqrt(bc2));
-    s.decay = float(1.0 - hp->lr * hp->weight_decay);
-    s.b1 = float(hp->beta1);
-    s.omb1 = float(1.0 - hp->beta1);
-    s.b2 = float(hp->beta2);
-    s.omb2 = float(1.0 - hp->beta2);
-    s.eps = float(hp->eps);
-    return s;
-}
-
-inline bool is_finite(double x) { return std::isfinite(x); }
-
-// A usable set of hyper-parameters: step >= 1, everything finite, betas in [0, 1).
-inline bool hp_valid(const z3_adamw* hp) {
-    return hp != nullptr && hp->step >= 1 && is_finite(hp->lr) && is_finite(hp->beta1) &&
-           is_finite(hp->beta2) && is_finite(hp->eps) && is_finite(hp->weight_decay) && hp->beta1 >= 0.0 &&
-           hp->beta1 < 1.0 && hp->beta2 >= 0.0 && hp->beta2 < 1.0;
-}
 
 __device__ __forceinline__ float lo_bf16(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float hi_bf16(uint32_t x) { return __uint_as_float(x & 0xFFFF0000u); }

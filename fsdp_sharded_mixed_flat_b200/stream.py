@@ -27,7 +27,11 @@ from . import zero3 as z3
 class LayerStreamer:
     def __init__(self, plan: "z3.Plan", n_layers: int, rank: int, master: torch.Tensor,
                  exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor, work_bf16: torch.Tensor,
-                 reduce_dtype: int = z3.Z3_REDUCE_FP32):
+                 reduce_dtype: int = z3.Z3_REDUCE_FP32, compute_priority: int = 0):
+        """compute_priority: CUDA stream priority of the compute stream (0 is the
+        default, negative is higher).  A higher priority than the copy stream's lets
+        the block scheduler start the fused kernel's blocks first and run the
+        arrival of the next block's bytes in the SMs it leaves free."""
         S, D = plan.S, plan.D
         for name, t in (("master", master), ("exp_avg", exp_avg), ("exp_avg_sq", exp_avg_sq),
                         ("work_bf16", work_bf16)):
@@ -41,7 +45,7 @@ class LayerStreamer:
         self.device = dev
         # two transient buffers, each the D owned contributions of one block, back to back
         self.buf = [torch.empty(D * S, dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        self.compute = torch.cuda.Stream(dev)
+        self.compute = torch.cuda.Stream(dev, priority=compute_priority)
         self.copy = torch.cuda.Stream(dev)
         self.filled = [torch.cuda.Event() for _ in range(2)]
         self.free = [torch.cuda.Event() for _ in range(2)]

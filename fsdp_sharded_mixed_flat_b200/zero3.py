@@ -83,6 +83,10 @@ def _load() -> C.CDLL:
     L.zero3_reduce_adamw_dev.restype = C.c_int
     L.zero3_gather_block.argtypes = [vp, vp, vp, vp, vp]
     L.zero3_gather_block.restype = C.c_int
+    L.zero3_reduce_scatter.argtypes = [vp, i32, vp, i32, i32, vp, vp]
+    L.zero3_reduce_scatter.restype = C.c_int
+    L.zero3_host_adamw.argtypes = [i64, vp, i32, vp, vp, vp, vp, C.POINTER(AdamW), i32]
+    L.zero3_host_adamw.restype = C.c_int
     return L
 
 
@@ -441,3 +445,50 @@ def zero3_gather_block(plan: Plan, shards: Sequence[torch.Tensor], flat_out: Opt
     dev = _launch_device(flat_out, *(tensor_out or []), *shards)
     rc = _call_on(dev, _lib.zero3_gather_block, plan.handle, sp, fp, tp, _stream_handle(stream, dev))
     _check(rc, "zero3_gather_block")
+
+
+def zero3_reduce_scatter(plan: Plan, rank: int, contrib: Sequence[torch.Tensor], grad: torch.Tensor,
+                         contrib_layout: int = Z3_CONTRIB_FULL, reduce_dtype: int = Z3_REDUCE_FP32,
+                         stream=None) -> None:
+    """The reduce-scatter's reduction alone: the averaged gradient of the owned
+    partition(s) into grad (float32 for the fp32 reduce, bfloat16 for the bf16
+    reduce; see include/zero3.h)."""
+    if len(contrib) != plan.D:
+        raise ValueError(f"need {plan.D} contributions, got {len(contrib)}")
+    n = plan.N_pad if rank < 0 else plan.S
+    c_need = plan.N_pad if contrib_layout == Z3_CONTRIB_FULL else plan.S
+    ptrs = (C.c_void_p * plan.D)()
+    for d, c in enumerate(contrib):
+        ptrs[d] = _dev_tensor(c, torch.bfloat16, c_need, f"contrib[{d}]")
+    gp = _dev_tensor(grad, _node_sum_dtype(reduce_dtype), n, "grad", host_ok=True)
+    dev = _launch_device(grad, *contrib)
+    rc = _call_on(dev, _lib.zero3_reduce_scatter, plan.handle, rank, ptrs, contrib_layout, reduce_dtype, gp,
+                  _stream_handle(stream, dev))
+    _check(rc, "zero3_reduce_scatter")
+
+
+def _host_tensor(t: torch.Tensor, dtype: torch.dtype, need: int, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < need:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {need}")
+    return t.data_ptr()
+
+
+def zero3_host_adamw(grad: torch.Tensor, master: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
+                     work_bf16: torch.Tensor, hp: AdamW, n: Optional[int] = None, n_threads: int = 0) -> None:
+    """AdamW and the bf16 cast of n elements in host memory, on host threads
+    (n defaults to grad.numel()); grad is float32 or bfloat16 (see include/zero3.h).
+    Synchronous; the GIL is released while it runs."""
+    n = grad.numel() if n is None else n
+    gdt = Z3_REDUCE_FP32 if grad.dtype == torch.float32 else Z3_REDUCE_BF16
+    gp = _host_tensor(grad, torch.float32 if gdt == Z3_REDUCE_FP32 else torch.bfloat16, n, "grad")
+    mp = _host_tensor(master, torch.float32, n, "master")
+    ap = _host_tensor(exp_avg, torch.float32, n, "exp_avg")
+    vp = _host_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
+    wp = _host_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
+    _check(_lib.zero3_host_adamw(n, gp, gdt, mp, ap, vp, wp, C.byref(hp), n_threads), "zero3_host_adamw")

@@ -193,7 +193,9 @@ Z3_API int zero3_allgather_bytes(int64_t block_params, int32_t n_blocks, int32_t
  *          then reads and writes it over PCIe; the arithmetic is unchanged).
  *   work_bf16 bf16 output, same extent as master; device or mapped host memory.
  *   reduce_dtype  Z3_REDUCE_FP32 or Z3_REDUCE_BF16.
- *   hp     host struct; hp->step >= 1, all values finite.
+ *   hp     host struct; hp->step >= 1, all values finite, betas in [0, 1),
+ *          eps > 0 (a zero eps turns the zero pad into 0/0), lr >= 0 and
+ *          weight_decay >= 0.
  *   cuda_stream  stream to enqueue on.
  * Pad elements are processed like real ones: a zero master with zero
  * contributions stays exactly zero.
@@ -304,6 +306,58 @@ Z3_API int zero3_fold_adamw(const z3_plan* p, int32_t rank, int32_t n_nodes, con
                             float* master, float* exp_avg, float* exp_avg_sq, uint16_t* work_bf16,
                             int32_t reduce_dtype, const z3_adamw* hp, void* cuda_stream);
 
+/* ------------------------------------ CPU offload: optimiser on the host
+ * The CPU-offload variant of [P2] §8: the Adam state (fp32 master, m, v)
+ * lives in host memory; every step the GPU reduces the owned gradient shard,
+ * the shard goes down over PCIe, AdamW runs on the host, and the bf16 weights
+ * go back up (4 or 2 bytes per parameter down, 2 up, instead of moving the
+ * 12 bytes of state each way).  These two calls are the GPU and host halves;
+ * composed (zero3_reduce_scatter, then zero3_host_adamw on its output) they
+ * give exactly the results of zero3_reduce_adamw.
+ *
+ * zero3_reduce_scatter: the reduce-scatter's reduction alone ([P3] "AllGather
+ * vs AllReduce": rank r receives the sum of the r-th slice of every rank's
+ * gradient; [P2] §4) for rank `rank`'s partition (S elements) or every
+ * partition (rank = -1, N_pad elements): the averaged gradient
+ *   g = (c_0 + c_1 + ... + c_{D-1}) * (1/D)
+ * folded left to right in rank order in the reduce dtype, the factor the
+ * fp32 constant nearest 1/D -- the g zero3_reduce_adamw hands to AdamW.
+ *   contrib, contrib_layout  as for zero3_reduce_adamw (D device pointers).
+ *   reduce_dtype  Z3_REDUCE_FP32: grad is float; Z3_REDUCE_BF16: every partial
+ *                 sum rounded to bf16 and g rounded to bf16, grad holds bf16
+ *                 (uint16_t) bits.
+ *   grad          device output (or mapped page-locked host memory), S (or
+ *                 N_pad) elements of that type.
+ * The vector path needs grad and every contribution (at its partition offset)
+ * 16-byte aligned; otherwise a scalar kernel gives the same results.
+ * Errors: Z3_EINVAL (NULL pointer, rank, layout or dtype out of range, grad
+ * over a contribution), Z3_EALIGN (a pointer off its element size), Z3_ECUDA.
+ *
+ * zero3_host_adamw: AdamW and the bf16 cast of n elements in HOST memory, on
+ * host threads, with the same operations in the same order as the GPU kernels
+ * (each one IEEE binary32 operation rounded to nearest-even, no fused
+ * multiply-add), so the results are bit-identical to zero3_reduce_adamw's:
+ *   p = p*(1 - lr*wd); m = b1*m + (1-b1)*g; v = b2*v + (1-b2)*g*g;
+ *   p = p - (lr/(1-b1^t)) * m / (sqrt(v)/sqrt(1-b2^t) + eps);  w = bf16(p)
+ *   grad        host array of n gradients: float (grad_dtype Z3_REDUCE_FP32)
+ *               or bf16 bits (Z3_REDUCE_BF16), e.g. zero3_reduce_scatter's
+ *               output copied down.
+ *   master, exp_avg, exp_avg_sq  host fp32 arrays of n elements, in place.
+ *   work_bf16   host bf16 output, n elements (to be copied up).
+ *   hp          as for zero3_reduce_adamw.
+ *   n_threads   host threads to use (0: all the hardware threads).  The
+ *               threads are kept in a pool for later calls; concurrent calls
+ *               run one after the other.
+ * Synchronous: returns when every element is updated.  Nothing touches the GPU.
+ * Errors: Z3_EINVAL (n < 0, n_threads < 0, NULL pointer with n > 0, bad
+ * grad_dtype, invalid hp, overlapping arrays), Z3_EALIGN (a pointer off its
+ * element size), Z3_EOVERFLOW (n beyond 2^60), Z3_ENOMEM (no thread could be
+ * started). */
+Z3_API int zero3_reduce_scatter(const z3_plan* p, int32_t rank, const uint16_t* const* contrib,
+                                int32_t contrib_layout, int32_t reduce_dtype, void* grad, void* cuda_stream);
+Z3_API int zero3_host_adamw(int64_t n, const void* grad, int32_t grad_dtype, float* master, float* exp_avg,
+                            float* exp_avg_sq, uint16_t* work_bf16, const z3_adamw* hp, int32_t n_threads);
+
 /* ------------------------------------- scalars in device memory (graphs)
  * zero3_step_scalars: the Z3_SCALARS fp32 scalars of one AdamW step, formed in
  * binary64 from *hp and rounded to fp32 once, exactly as zero3_reduce_adamw
@@ -312,7 +366,7 @@ Z3_API int zero3_fold_adamw(const z3_plan* p, int32_t rank, int32_t n_nodes, con
  *   [3] beta1   [4] 1 - beta1   [5] beta2   [6] 1 - beta2   [7] eps
  *   out: host array of Z3_SCALARS floats.
  * Errors: Z3_EINVAL (out or hp NULL, hp->step < 1, a value not finite, a beta
- * outside [0, 1)).
+ * outside [0, 1), eps <= 0, lr < 0 or weight_decay < 0).
  *
  * zero3_reduce_adamw_dev: zero3_reduce_adamw (n_gathered = 0) or
  * zero3_reduce_adamw_gather (n_gathered >= 1, up to Z3_GATHER_MAX) whose kernel
@@ -339,7 +393,10 @@ Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t
  *   shards     host array of D device pointers, shard r = rank r's S bf16
  *              working weights.
  *   flat_out   device bf16, N_pad elements: flat_out[r*S + j] = shards[r][j].
- *              May be NULL when tensor_out is given.
+ *              May be NULL when tensor_out is given.  A shard may already
+ *              sit in place inside it, shards[r] == flat_out + r*S (a rank's
+ *              own shard kept as a view of its gathered block, as FSDP lays
+ *              it out); that partition is left as it is and not copied.
  *   tensor_out host array of n_tensors device pointers, or NULL: tensor i's
  *              buffer receives its numel elements (flat elements
  *              [offset_i, offset_i + numel_i)), read straight from the shards.
@@ -347,7 +404,9 @@ Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t
  * Zero-copy views need no call: zero3_plan_tensor gives each tensor's offset
  * in flat_out.  The vector path needs S % 8 == 0 and 16-byte aligned
  * pointers; otherwise a scalar kernel gives the same bytes.
- * Errors: Z3_EINVAL (both outputs NULL, a NULL shard), Z3_EALIGN, Z3_ECUDA. */
+ * Errors: Z3_EINVAL (both outputs NULL, a NULL shard, an output overlapping a
+ * shard other than in the in-place position above, outputs overlapping each
+ * other), Z3_EALIGN, Z3_ECUDA. */
 Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
                               uint16_t* const* tensor_out, void* cuda_stream);
 

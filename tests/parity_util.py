@@ -77,6 +77,30 @@ def assert_bf16_parity(got: np.ndarray, ref: np.ndarray, what: str, exact: bool 
         assert n == 0, f"{what}: {n} of {got.size} bf16 values differ"
 
 
+class RefPlan:
+    """The oracle's plan of a tensor list: offsets, numels, N, N_pad, S."""
+
+    def __init__(self, shapes, D: int, A: int):
+        self.numels = [synth.numel(s) for s in shapes]
+        offs, self.N, self.N_pad, self.S = oracle.plan(self.numels, D, A)
+        self.offsets = [int(o) for o in offs]
+        self.D = D
+
+
+def checked_plan(z3, shapes, D: int, A: int):
+    """The product's plan and the oracle's plan of the same tensor list, after
+    asserting that they agree on every offset, numel, N, N_pad and S.  Expected
+    values are built from the oracle's plan only, so a planner mistake cannot
+    make the kernel and its expected value agree."""
+    plan = z3.zero3_plan(shapes, D, A)
+    ref = RefPlan(shapes, D, A)
+    assert (plan.N, plan.N_pad, plan.S) == (ref.N, ref.N_pad, ref.S), \
+        f"plan sizes {(plan.N, plan.N_pad, plan.S)} != oracle {(ref.N, ref.N_pad, ref.S)}"
+    assert list(plan.offsets) == ref.offsets, "tensor offsets differ from the oracle's plan"
+    assert list(plan.numels) == ref.numels, "tensor sizes differ from the oracle's plan"
+    return plan, ref
+
+
 def state_init(n_real: int, n_pad: int, seed: int):
     """fp32 master (zero pad) and zero moments, on the device."""
     p = synth.master_weights(n_real, n_pad, seed=seed, device="cuda")

@@ -35,7 +35,8 @@ def test_library_exports_every_declared_symbol():
                             "zero3_transient_bytes", "zero3_allgather_bytes", "zero3_reduce_adamw",
                             "zero3_reduce_adamw_hybrid", "zero3_node_sum", "zero3_fold_adamw",
                             "zero3_reduce_adamw_gather",
-                            "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block"]), names
+                            "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block",
+                            "zero3_reduce_scatter", "zero3_host_adamw"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -196,6 +197,11 @@ def test_reduce_adamw_argument_errors():
     assert call_reduce(p, hp=z3.adamw(beta1=1.0)) == E
     assert call_reduce(p, hp=z3.adamw(lr=float("nan"))) == E
     assert call_reduce(p, hp=z3.adamw(eps=float("inf"))) == E
+    # eps = 0 would make a zero pad element compute 0/0; negative lr or decay are not AdamW
+    assert call_reduce(p, hp=z3.adamw(eps=0.0)) == E
+    assert call_reduce(p, hp=z3.adamw(eps=-1e-8)) == E
+    assert call_reduce(p, hp=z3.adamw(lr=-1e-4)) == E
+    assert call_reduce(p, hp=z3.adamw(weight_decay=-0.1)) == E
     assert z3.lib().zero3_reduce_adamw(None, 0, None, 0, None, None, None, None, 0, None, None) == E
     # misaligned: fp32 state off a 4-byte boundary, bf16 off a 2-byte boundary
     assert call_reduce(p, ptrs=[P16 + 2, P16 * 2, P16 * 3, P16 * 4]) == z3.Z3_EALIGN
@@ -238,6 +244,28 @@ def test_reduce_adamw_hybrid_argument_errors():
     e = z3.zero3_plan([], 4, 8)
     assert call_hybrid(e, 16) == z3.Z3_OK                             # 64 contributions, empty plan
     assert call_hybrid(e, 1) == z3.Z3_OK
+
+
+def test_reduce_scatter_argument_errors():
+    p = z3.zero3_plan([(1000,)], 4, 8)
+    L, E, A = z3.lib(), z3.Z3_EINVAL, z3.Z3_EALIGN
+    c = [P16 * (100 + d) for d in range(4)]
+
+    def rs(contrib=c, rank=-1, layout=0, mode=0, out=P16 * 50):
+        arr = (C.c_void_p * 4)(*contrib)
+        return L.zero3_reduce_scatter(p.handle, rank, arr, layout, mode, None if out is None else C.c_void_p(out),
+                                      None)
+    assert rs(out=None) == E
+    assert rs(rank=4) == E
+    assert rs(rank=-2) == E
+    assert rs(layout=1) == E                             # owned layout needs one rank
+    assert rs(mode=2) == E
+    assert rs(contrib=c[:3] + [0]) == E
+    assert rs(contrib=c[:3] + [c[3] + 1]) == A
+    assert rs(out=P16 * 50 + 2) == A                      # fp32 gradient needs 4-byte alignment
+    assert rs(out=c[1]) == E                              # over a contribution
+    e = z3.zero3_plan([], 4, 8)
+    assert L.zero3_reduce_scatter(e.handle, -1, (C.c_void_p * 4)(*c), 0, 1, C.c_void_p(P16 * 50), None) == z3.Z3_OK
 
 
 def test_node_sum_and_fold_argument_errors():
@@ -321,6 +349,13 @@ def test_step_scalars_match_the_oracle():
         z3.zero3_step_scalars(z3.adamw(step=0))
     with pytest.raises(z3.Zero3Error):
         z3.zero3_step_scalars(z3.adamw(beta2=1.0))
+    for bad in (dict(eps=0.0), dict(eps=-1e-8), dict(lr=-3e-4), dict(weight_decay=-0.1)):
+        with pytest.raises(z3.Zero3Error) as e:
+            z3.zero3_step_scalars(z3.adamw(**bad))
+        assert e.value.status == z3.Z3_EINVAL, bad
+    # the edges that stay valid: no learning rate, no decay
+    z3.zero3_step_scalars(z3.adamw(lr=0.0))
+    z3.zero3_step_scalars(z3.adamw(weight_decay=0.0))
 
 
 def test_reduce_adamw_dev_argument_errors():
@@ -371,7 +406,10 @@ def test_gather_block_argument_errors():
     assert call_gather(p, shards=[P16 + 1, P16 * 2, P16 * 3, P16 * 4]) == z3.Z3_EALIGN
     assert call_gather(p, flat=P16 * 500 + 1) == z3.Z3_EALIGN
     assert call_gather(p, flat=None, tensor_out=[P16 * 700 + 1, 0]) == z3.Z3_EALIGN
-    assert call_gather(p, flat=P16 * 100) == E                    # flat over shard 0
+    S = p.S * 2                                                  # bytes per shard
+    assert call_gather(p, flat=P16 * 100 - S) == E               # shard 0 where partition 1 lies
+    assert call_gather(p, flat=P16 * 100 + 2) == E               # flat over shard 0, off its place
+    # shard 0 sitting exactly in place (flat + 0*S) is accepted: see the GPU test
     assert call_gather(p, flat=None, tensor_out=[P16 * 700, P16 * 700 + 2]) == E   # tensors overlap
     assert call_gather(p, tensor_out=[P16 * 500, 0]) == E         # tensor over flat
     assert z3.lib().zero3_gather_block(None, None, None, None, None) == E

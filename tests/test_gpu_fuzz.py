@@ -14,7 +14,8 @@ import torch
 
 import oracle
 import synth
-from parity_util import Guarded, assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp
+from parity_util import (Guarded, assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for,
+                         oracle_hp)
 
 pytestmark = pytest.mark.gpu
 SENTINEL = 0x7FAB
@@ -34,8 +35,8 @@ def one_case(z3, rnd: random.Random, seed: int):
     A = rnd.choice([1, 2, 3, 8, 16, 128])
     shapes = [(rnd.randint(0, 3000),) if rnd.random() < 0.7 else (rnd.randint(1, 30), rnd.randint(1, 90))
               for _ in range(rnd.randint(1, 6))]
-    plan = z3.zero3_plan(shapes, D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, shapes, D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     rank = -1 if rnd.random() < 0.5 else rnd.randrange(D)
     layout = z3.Z3_CONTRIB_OWNED if rank >= 0 and rnd.random() < 0.5 else z3.Z3_CONTRIB_FULL
     mode = rnd.choice([0, 1])
@@ -97,12 +98,12 @@ def one_case(z3, rnd: random.Random, seed: int):
     if rank < 0 and gw is not None:
         shards = [gw.t[r * S:(r + 1) * S] for r in range(D)]
         flat = Guarded(N_pad, torch.bfloat16, skew[4])
-        outs = [Guarded(k, torch.bfloat16, rnd.choice([0, 1, 3])) if k else None for k in plan.numels]
+        outs = [Guarded(k, torch.bfloat16, rnd.choice([0, 1, 3])) if k else None for k in ref.numels]
         z3.zero3_gather_block(plan, shards, flat.t, [None if o is None else o.t for o in outs])
         torch.cuda.synchronize()
-        ref = oracle.all_gather([hw[r * S:(r + 1) * S] for r in range(D)], S)
-        assert np.array_equal(synth.bf16_bits(flat.t), ref), "flat " + desc
-        for o, r in zip(outs, oracle.unflatten(ref, plan.offsets, plan.numels)):
+        ref_flat = oracle.all_gather([hw[r * S:(r + 1) * S] for r in range(D)], S)
+        assert np.array_equal(synth.bf16_bits(flat.t), ref_flat), "flat " + desc
+        for o, r in zip(outs, oracle.unflatten(ref_flat, ref.offsets, ref.numels)):
             if o is not None:
                 assert np.array_equal(synth.bf16_bits(o.t), r), "tensor " + desc
                 assert o.guards_intact()
@@ -121,8 +122,8 @@ def hybrid_case(z3, rnd: random.Random, seed: int):
     R = rnd.randint(1, 64 // D)
     A = rnd.choice([1, 2, 8, 128])
     shapes = [(rnd.randint(0, 3000),) for _ in range(rnd.randint(1, 4))]
-    plan = z3.zero3_plan(shapes, D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, shapes, D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     rank = -1 if rnd.random() < 0.5 else rnd.randrange(D)
     layout = z3.Z3_CONTRIB_OWNED if rank >= 0 and rnd.random() < 0.5 else z3.Z3_CONTRIB_FULL
     mode = rnd.choice([0, 1])
@@ -169,8 +170,8 @@ def node_fold_case(z3, rnd: random.Random, seed: int):
     R = rnd.randint(1, 8)
     A = rnd.choice([1, 2, 8, 128])
     shapes = [(rnd.randint(0, 3000),) for _ in range(rnd.randint(1, 4))]
-    plan = z3.zero3_plan(shapes, D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, shapes, D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     rank = -1 if rnd.random() < 0.5 else rnd.randrange(D)
     layout = z3.Z3_CONTRIB_OWNED if rank >= 0 and rnd.random() < 0.5 else z3.Z3_CONTRIB_FULL
     mode = rnd.choice([0, 1])

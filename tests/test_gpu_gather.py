@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import Guarded
+from parity_util import Guarded, checked_plan
 
 pytestmark = pytest.mark.gpu
 
@@ -31,13 +31,13 @@ def random_bits(n: int, gen: torch.Generator) -> torch.Tensor:
 
 
 def run_gather(z3, shapes, D, A, shard_skew=0, dst_skews=None, skip=(), with_flat=True, seed=0):
-    plan = z3.zero3_plan(shapes, D, A)
-    S, N_pad = plan.S, plan.N_pad
+    plan, ref = checked_plan(z3, shapes, D, A)
+    S, N_pad = ref.S, ref.N_pad
     gen = torch.Generator().manual_seed(seed)
     shards = [Guarded(S, torch.bfloat16, shard_skew, fill=random_bits(S, gen)) for _ in range(D)]
     flat = Guarded(N_pad, torch.bfloat16, 0) if with_flat else None
     dst_skews = dst_skews or [0] * len(shapes)
-    outs = [None if i in skip else Guarded(plan.numels[i], torch.bfloat16, dst_skews[i]) for i in range(len(shapes))]
+    outs = [None if i in skip else Guarded(ref.numels[i], torch.bfloat16, dst_skews[i]) for i in range(len(shapes))]
     z3.zero3_gather_block(plan, [s.t for s in shards], None if flat is None else flat.t,
                           [None if o is None else o.t for o in outs])
     torch.cuda.synchronize()
@@ -46,11 +46,11 @@ def run_gather(z3, shapes, D, A, shard_skew=0, dst_skews=None, skip=(), with_fla
     if flat is not None:
         assert np.array_equal(synth.bf16_bits(flat.t), ref_flat)
         assert flat.guards_intact()
-    ref_t = oracle.unflatten(ref_flat, plan.offsets, plan.numels)
+    ref_t = oracle.unflatten(ref_flat, ref.offsets, ref.numels)
     for i, (o, r) in enumerate(zip(outs, ref_t)):
         if o is None:
             continue
-        assert np.array_equal(synth.bf16_bits(o.t), r), f"tensor {i} (offset {plan.offsets[i]})"
+        assert np.array_equal(synth.bf16_bits(o.t), r), f"tensor {i} (offset {ref.offsets[i]})"
         assert o.guards_intact(), f"canary of tensor {i}"
     for s in shards:
         assert s.guards_intact()
@@ -120,17 +120,52 @@ def test_llama7b_block_full_size(z3):
     the 9 separate tensors, every element compared."""
     w = synth.WORKLOADS["llama7b_d8"]
     shapes = [s for _, s in w["tensors"]]
-    plan = z3.zero3_plan(shapes, 8, synth.ALIGN)
-    S = plan.S
+    plan, ref = checked_plan(z3, shapes, 8, synth.ALIGN)
+    S = ref.S
     gen = torch.Generator(device="cuda").manual_seed(5)
-    work = torch.randint(-32768, 32768, (plan.N_pad,), generator=gen, device="cuda",
+    work = torch.randint(-32768, 32768, (ref.N_pad,), generator=gen, device="cuda",
                          dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
-    flat = torch.empty(plan.N_pad, dtype=torch.bfloat16, device="cuda")
+    flat = torch.empty(ref.N_pad, dtype=torch.bfloat16, device="cuda")
     outs = [torch.empty(s, dtype=torch.bfloat16, device="cuda") for s in shapes]
     z3.zero3_gather_block(plan, [work[r * S:(r + 1) * S] for r in range(8)], flat, outs)
     torch.cuda.synchronize()
     host = synth.bf16_bits(work)
     ref_flat = oracle.all_gather([host[r * S:(r + 1) * S] for r in range(8)], S)
     assert np.array_equal(synth.bf16_bits(flat), ref_flat)
-    for o, r in zip(outs, oracle.unflatten(ref_flat, plan.offsets, plan.numels)):
+    ref_t = oracle.unflatten(ref_flat, ref.offsets, ref.numels)
+    for o, r in zip(outs, ref_t):
         assert np.array_equal(synth.bf16_bits(o).ravel(), r)
+    for view, r in zip(plan.views(flat), ref_t):                 # the zero-copy unflatten
+        assert np.array_equal(synth.bf16_bits(view).ravel(), r)
+
+
+@pytest.mark.parametrize("own", [[2], [0, 3], [0, 1, 2, 3]])
+def test_shards_in_place_inside_the_block(z3, own):
+    """A shard that already sits at its place in the block (shards[r] is the view
+    flat[r*S:(r+1)*S], how FSDP keeps a rank's own shard) is accepted and left as
+    it is; the other shards are copied around it, and the per-tensor copies read
+    it in place."""
+    shapes = [(1000,), (77, 13), (4096,), (5,)]
+    D = 4
+    plan, ref = checked_plan(z3, shapes, D, 8)
+    S, N_pad = ref.S, ref.N_pad
+    gen = torch.Generator().manual_seed(31)
+    flat = Guarded(N_pad, torch.bfloat16, 0)
+    apart = [Guarded(S, torch.bfloat16, 0, fill=random_bits(S, gen)) for _ in range(D)]
+    for r in own:
+        flat.t[r * S:(r + 1) * S].copy_(apart[r].t)            # rank r's shard lives in the block
+    shards = [flat.t[r * S:(r + 1) * S] if r in own else apart[r].t for r in range(D)]
+    outs = [Guarded(k, torch.bfloat16, 1) for k in ref.numels]
+    z3.zero3_gather_block(plan, shards, flat.t, [o.t for o in outs])
+    torch.cuda.synchronize()
+    ref_flat = oracle.all_gather([synth.bf16_bits(a.t) for a in apart], S)
+    assert np.array_equal(synth.bf16_bits(flat.t), ref_flat)
+    for o, r in zip(outs, oracle.unflatten(ref_flat, ref.offsets, ref.numels)):
+        assert np.array_equal(synth.bf16_bits(o.t), r)
+        assert o.guards_intact()
+    assert flat.guards_intact()
+    # a shard inside the block at another rank's place is refused before any work
+    bad = list(shards)
+    bad[1] = flat.t[2 * S:3 * S] if 1 not in own else flat.t[0:S]
+    with pytest.raises(z3.Zero3Error):
+        z3.zero3_gather_block(plan, bad, flat.t)

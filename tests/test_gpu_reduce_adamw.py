@@ -16,8 +16,8 @@ import torch
 
 import oracle
 import synth
-from parity_util import (Guarded, assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp,
-                         state_init)
+from parity_util import (Guarded, assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for,
+                         oracle_hp, state_init)
 
 pytestmark = pytest.mark.gpu
 
@@ -33,8 +33,8 @@ def z3():
 
 def run_small(z3, numels, D, A, rank, layout, mode, steps=10, seed=0, skew=(0, 0, 0, 0, 0),
               dist="normal", sigma=1e-3, zero_frac=0.0):
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, seed)
     p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
@@ -152,8 +152,8 @@ SENTINEL = 0x7FAB  # a bf16 NaN pattern the kernel never produces
 
 
 def run_fused(z3, numels, D, A, rank, layout, mode, n_gathered, with_work, steps=3, skew=0, seed=5):
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, seed)
     p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
@@ -219,8 +219,8 @@ def test_fused_gather_misaligned_scalar_path(z3):
 def test_offloaded_state_matches_oracle(z3, numels, D, A, rank, mode):
     """fp32 master / m / v in page-locked host memory, read and written by the kernel
     over PCIe (the CPU-offload placement): same results as in HBM."""
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, 8)
     p0 = (p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]).cpu()
@@ -252,8 +252,8 @@ def test_staged_offload_matches_oracle(z3, numels, D, A, n_stage, mode):
     """The optimiser state in pinned host memory, streamed partition by partition
     through device staging buffers: same results as the whole-block kernel."""
     from fsdp_sharded_mixed_flat_b200.offload import OffloadedState
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     p_full, _, _ = state_init(N, N_pad, 9)
     p = p_full.cpu().pin_memory()
     m, v = torch.zeros(N_pad).pin_memory(), torch.zeros(N_pad).pin_memory()
@@ -294,8 +294,8 @@ def sample_indices(n: int, S: int, D: int, k: int, seed: int) -> torch.Tensor:
 def run_sampled(z3, workload: str, D: int, rank: int, layout: int, mode: int, steps: int,
                 k: int = 200_000, seed: int = 0):
     w = synth.WORKLOADS[workload]
-    plan = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [s for _, s in w["tensors"]], D, synth.ALIGN)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, seed)
     p = (p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]).contiguous()
@@ -342,6 +342,58 @@ def test_llama7b_block_d32_padded(z3):
     assert not wk[plan.N:].view(torch.int16).any()
 
 
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+def test_llama7b_d32_sharded_equals_unsharded_full_size(z3, mode):
+    """The padded 7B block at D = 32 (N = 202,387,457, N_pad = 202,391,552, the
+    4095 pad elements in rank 31's shard), 3 steps run two ways on the same
+    contributions: 32 separate rank-r launches (full layout), each into its own
+    S-element master / m / v / bf16 buffers, and one all-ranks launch on a copy of
+    the same state.  Sharding leaves the arithmetic of DDP unchanged ("Building
+    GPT from Scratch — Part 8", "Key Takeaways"; "7.10 — Fully-sharded data
+    parallel", §3), so the 32 shards concatenated must equal the unsharded result
+    bit for bit, and both must equal the oracle on sampled elements that include
+    every shard boundary and the whole pad; the pad must stay exactly zero."""
+    w = synth.WORKLOADS["llama7b_d32"]
+    D = 32
+    plan, ref = checked_plan(z3, [s for _, s in w["tensors"]], D, synth.ALIGN)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
+    assert (N, N_pad, S) == (202_387_457, 202_391_552, 6_324_736)
+    p_full, _, _ = state_init(N, N_pad, 3)
+    big = [p_full.clone(), torch.zeros_like(p_full), torch.zeros_like(p_full),
+           torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")]
+    shard = [[p_full[r * S:(r + 1) * S].clone() for r in range(D)],
+             [torch.zeros(S, device="cuda") for _ in range(D)],
+             [torch.zeros(S, device="cuda") for _ in range(D)],
+             [torch.zeros(S, dtype=torch.bfloat16, device="cuda") for _ in range(D)]]
+    idx = torch.from_numpy(np.unique(np.concatenate([sample_indices(N_pad, S, D, 100_000, 4).cpu().numpy(),
+                                                     np.arange(N, N_pad)]))).cuda()
+    hp_, hm, hv = f32_host(p_full[idx]).copy(), np.zeros(idx.numel(), np.float32), np.zeros(idx.numel(), np.float32)
+    hw = np.zeros(idx.numel(), np.uint16)
+    del p_full
+    for t in range(1, 4):
+        c = synth.contributions(D, N, N_pad, seed=3, step=t, sigma=w["sigma"], device="cuda")
+        hp = z3.adamw(**hp_for(t))
+        for r in range(D):
+            z3.zero3_reduce_adamw(plan, r, c, shard[0][r], shard[1][r], shard[2][r], shard[3][r], hp,
+                                  contrib_layout=z3.Z3_CONTRIB_FULL, reduce_dtype=mode)
+        z3.zero3_reduce_adamw(plan, -1, c, *big, hp, reduce_dtype=mode)
+        oracle.reduce_adamw([synth.bf16_bits(x[idx]) for x in c], idx.numel(), 0, hp_, hm, hv, hw, oracle_hp(t),
+                            layout=oracle.LAYOUT_OWNED, reduce_dtype=mode)
+        del c
+    torch.cuda.synchronize()
+    for name, whole, parts in zip(("master", "exp_avg", "exp_avg_sq", "work_bf16"), big, shard):
+        bits = torch.int16 if whole.dtype == torch.bfloat16 else torch.int32
+        cat = torch.cat(parts)
+        differ = int((cat.view(bits) != whole.view(bits)).sum().item())
+        assert differ == 0, f"{name}: {differ} elements of the 32 shards differ from the unsharded step"
+        assert not whole[N:].view(bits).any(), f"{name}: the pad is no longer zero"
+    what = f"7B block D=32 mode={mode}"
+    assert_f32_parity(f32_host(big[0][idx]), hp_, "master " + what)
+    assert_f32_parity(f32_host(big[1][idx]), hm, "exp_avg " + what)
+    assert_f32_parity(f32_host(big[2][idx]), hv, "exp_avg_sq " + what)
+    assert_bf16_parity(synth.bf16_bits(big[3][idx]), hw, "work_bf16 " + what)
+
+
 @pytest.mark.parametrize("D", [2, 4, 8, 16])
 def test_llama7b_policy_sweep_bf16_reduce(z3, D):
     run_sampled(z3, "llama7b_policy", D, -1, z3.Z3_CONTRIB_FULL, 1, steps=3, k=100_000)
@@ -354,8 +406,8 @@ def test_policy_sweep_hundred_steps_every_element(z3, D):
     element compared after the last step."""
     w = synth.WORKLOADS["llama7b_policy"]
     n_real = 1 << 20
-    plan = z3.zero3_plan([(n_real,)], D, synth.ALIGN)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(n_real,)], D, synth.ALIGN)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     for mode in (0, 1):
         p, m, v = state_init(N, N_pad, 31)
         wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
@@ -384,8 +436,8 @@ def test_tiny_gpt_full_ten_steps_then_gather(z3):
     """Config of the 3.3M-parameter GPT, every element compared, then the gather."""
     w = synth.WORKLOADS["tiny_gpt"]
     shapes = [s for _, s in w["tensors"]]
-    plan = z3.zero3_plan(shapes, w["D"], synth.ALIGN)
-    N, N_pad, S, D = plan.N, plan.N_pad, plan.S, plan.D
+    plan, ref = checked_plan(z3, shapes, w["D"], synth.ALIGN)
+    N, N_pad, S, D = ref.N, ref.N_pad, ref.S, ref.D
     p, m, v = state_init(N, N_pad, 0)
     wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
     hp_, hm, hv, hw = f32_host(p).copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
@@ -405,7 +457,7 @@ def test_tiny_gpt_full_ten_steps_then_gather(z3):
     torch.cuda.synchronize()
     ref_flat = oracle.all_gather([hw[r * S:(r + 1) * S] for r in range(D)], S)
     assert np.array_equal(synth.bf16_bits(flat), ref_flat)
-    ref_t = oracle.unflatten(ref_flat, plan.offsets, plan.numels)
+    ref_t = oracle.unflatten(ref_flat, ref.offsets, ref.numels)
     for o, r, view in zip(outs, ref_t, plan.views(flat)):
         assert np.array_equal(synth.bf16_bits(o).ravel(), r)
         assert np.array_equal(synth.bf16_bits(view).ravel(), r)
@@ -420,8 +472,8 @@ def test_single_launch_beyond_2_31_elements(z3):
     free, _ = torch.cuda.mem_get_info()
     if free < 48e9:
         pytest.skip("needs about 45 GB of free device memory")
-    plan = z3.zero3_plan([(N,)], D, synth.ALIGN)
-    N_pad, S = plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(N,)], D, synth.ALIGN)
+    N_pad, S = ref.N_pad, ref.S
     p = synth.master_weights(N, N_pad, seed=21, device="cuda")
     m, v = torch.zeros_like(p), torch.zeros_like(p)
     w = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
@@ -455,8 +507,8 @@ def test_random_hyperparameters_match_oracle(z3):
     large learning rate, no decay, late steps) and both reduce dtypes."""
     import random
     rnd = random.Random(99)
-    plan = z3.zero3_plan([(30000,), (4097,)], 4, 8)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(30000,), (4097,)], 4, 8)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     for case in range(12):
         a = dict(lr=10 ** rnd.uniform(-5, -1.5), beta1=rnd.choice([0.0, 0.5, 0.9, 0.99]),
                  beta2=rnd.choice([0.5, 0.95, 0.999]), eps=10 ** rnd.uniform(-10, -2),
