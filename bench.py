@@ -6,11 +6,16 @@ memory ledger.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--D D] [--reduce-dtype fp32|bf16] [--stage 1|2|3]
-                    [--graph] [--offload] [--unflatten-copy] [--refill copy|fill] [--drift]
+                    [--graph] [--offload [state|host]] [--unflatten-copy] [--refill copy|fill|memset] [--drift]
 
-One process per GPU (torchrun for N > 1).  Each rank runs its own block
-(independent replicas: the path needs no inter-GPU exchange), so the work per
-GPU is fixed as N grows.  Rank 0 prints one JSON line.
+One process per GPU (torchrun for N > 1).  With N = 1 the block's D ranks are
+simulated on the one GPU.  With N > 1 the block is sharded over the N GPUs
+(D = N, strong scaling: one block per step in all): every rank's gradient
+crosses an NCCL all-to-all (the reduce-scatter's data movement), the fused
+kernel updates the rank's own partition, and an NCCL all-gather assembles the
+block (--transport peer: the kernels read the peers' memory through CUDA IPC
+instead); --replicas runs N independent single-GPU replicas instead.  Rank 0
+prints one JSON line.
 
 Timing: W untimed warm-up steps, then K steps between a barrier plus
 cudaDeviceSynchronize on each side, timed with CUDA events on the launching
@@ -59,12 +64,16 @@ SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 # How the 70B shard's per-layer contributions arrive in a transient buffer (the
 # reduce-scatter's delivery, simulated on one GPU).
+# Measured on B200 for the 80-layer step: copy 93.8 ms, fill 85.9 ms (torch's
+# bf16 fill kernel writes at about 3.9 TB/s), memset 70.0 ms (the driver's
+# memset writes at about 6.8 TB/s).
 ARRIVALS = {
     "copy": "device-to-device copy from a pool on the copy stream (read + write)",
-    "fill": "write-only fill of the transient buffer on the copy stream, as a delivery over NVLink writes it",
-    "fill_prio": "write-only fill on the copy stream, the fused kernel's stream at a higher priority",
+    "fill": "write-only fill of the transient buffer by torch's fill kernel on the copy stream",
+    "memset": "write-only cudaMemsetAsync of the transient buffer on the copy stream, as a delivery over NVLink "
+              "writes it",
 }
-DEFAULT_ARRIVAL = "fill"
+DEFAULT_ARRIVAL = "memset"
 
 
 def parse_args():
@@ -81,11 +90,19 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--D", type=int, default=0, help="simulated ranks (default: the workload's)")
     ap.add_argument("--reduce-dtype", choices=["fp32", "bf16"], default="fp32")
-    ap.add_argument("--offload", action="store_true",
-                    help="fp32 master / m / v in page-locked host memory, reached by the kernel over PCIe")
+    ap.add_argument("--offload", nargs="?", const="state", default=None, choices=["state", "host"],
+                    help="fp32 master / m / v in page-locked host memory: 'state' streams it through the GPU, "
+                         "which keeps the arithmetic (24 B per param over PCIe); 'host' runs AdamW on the host, "
+                         "with the averaged gradient down and the bf16 weights up (6 B per param, 4 in bf16)")
     ap.add_argument("--refill", choices=list(ARRIVALS), default=DEFAULT_ARRIVAL,
                     help="70B shard: how each layer's contributions arrive in the transient buffer: "
                          + "; ".join(f"{k}: {v}" for k, v in ARRIVALS.items()))
+    ap.add_argument("--replicas", action="store_true",
+                    help="N > 1: run N independent single-GPU replicas (each simulating its own D ranks) instead "
+                         "of the real D-GPU step with D = N")
+    ap.add_argument("--transport", choices=["nccl", "peer"], default="nccl",
+                    help="N > 1: how the D-GPU step moves its bytes: NCCL all-to-all and all-gather around the "
+                         "fused kernel, or the kernels' own plain loads of the peers' memory (CUDA IPC)")
     ap.add_argument("--sweep-steps", type=int, default=10,
                     help="timed steps per configuration in the sweep of the target configurations")
     ap.add_argument("--no-sweep", action="store_true",
@@ -396,13 +413,18 @@ class BlockRunner:
         self.offload = offload
         self.work = torch.zeros(self.N_pad, dtype=torch.bfloat16, device=dev)
         self.offloaded = None
+        self.host_seconds = []
         if offload:
-            # the optimiser state leaves the GPU: page-locked host memory, streamed through the GPU
-            from fsdp_sharded_mixed_flat_b200.offload import OffloadedState
+            # the optimiser state leaves the GPU: page-locked host memory
+            from fsdp_sharded_mixed_flat_b200.offload import HostAdamWOffload, OffloadedState
             self.master, self.exp_avg, self.exp_avg_sq = (t.cpu().pin_memory() for t in
                                                           (self.master, self.exp_avg, self.exp_avg_sq))
-            self.offloaded = OffloadedState(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
-                                            reduce_dtype=reduce_dtype)
+            if offload == "host":
+                self.offloaded = HostAdamWOffload(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
+                                                  reduce_dtype=reduce_dtype)
+            else:
+                self.offloaded = OffloadedState(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
+                                                reduce_dtype=reduce_dtype)
         self.flat = torch.empty(self.N_pad, dtype=torch.bfloat16, device=dev)
         self.shards = [self.work[r * self.S:(r + 1) * self.S] for r in range(D)]
         self.stream = torch.cuda.current_stream(dev)
@@ -451,13 +473,24 @@ class BlockRunner:
             # events around the replay time every kernel of the graph
             self.k1_bytes_per_launch = self.step_bytes
             self.k1_name = "CUDA graph of the step (%s)" % ("fused kernel + gather" if stage == 3 else "fused kernel")
-        if offload:
+        if offload == "state":
             what += ("; fp32 master/m/v in page-locked host memory, streamed partition by partition through "
                      "device staging buffers (copy-in, kernel, copy-out on three streams)")
             self.k1_name += " (rank-partition launches on staged state)"
             self.k1_launches_per_step = D
             self.k1_bytes_per_launch = (2 * D + 26) * self.S
             self.launches_per_step = D + 1
+        elif offload == "host":
+            gb = 4 if reduce_dtype == 0 else 2
+            what += ("; fp32 master/m/v in page-locked host memory and AdamW on the host: per partition the "
+                     "averaged gradient is reduced on the GPU, copied down, updated by libzero3's host threads, "
+                     "and the bf16 weights copied up (pipelined over partitions)")
+            self.k1_name = (f"k_node_sum_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}, scaled> "
+                            "(the reduce-scatter's reduction alone, one launch per partition)")
+            self.k1_launches_per_step = D
+            self.k1_bytes_per_launch = (2 * D + gb) * self.S
+            self.launches_per_step = D + 1
+            self.step_bytes = self.k1_bytes_per_launch * D + 4 * self.N_pad
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
                      f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
                      f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + {what}")
@@ -486,7 +519,10 @@ class BlockRunner:
         if k1_events is not None:
             k1_events[0][0].record(self.stream)
         if self.offloaded is not None:
-            self.offloaded.step(contribs, hp, k1_events)
+            if self.offload == "host":
+                self.offloaded.step(contribs, hp, k1_events, host_seconds=self.host_seconds)
+            else:
+                self.offloaded.step(contribs, hp, k1_events)
             z3.zero3_gather_block(pl, self.shards, flat, self.tensor_out, stream=self.stream)
             return self.views(pl, flat)
         if self.stage != 3:
@@ -600,9 +636,8 @@ class ShardRunner:
                                 for d in range(D)]) for _ in range(2)]
         if refill not in ARRIVALS:
             raise SystemExit(f"unknown arrival {refill}")
-        hi = torch.cuda.Stream.priority_range()[1] if refill == "fill_prio" else 0   # (low, high)
         self.streamer = LayerStreamer(plan, L, 0, self.master, self.exp_avg, self.exp_avg_sq, self.work,
-                                      reduce_dtype=reduce_dtype, compute_priority=hi)
+                                      reduce_dtype=reduce_dtype)
         self.stream = torch.cuda.current_stream(dev)
         self.step_no = 0
         self.units_per_step = L * S                            # owned params of this rank
@@ -616,7 +651,19 @@ class ShardRunner:
         self.k1_name = f"k_reduce_adamw_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}> (owned layout)"
         self.source = lambda l: self.pool[l & 1]
         # write-only refill: the transient buffer receives a value, as an NVLink delivery would write it
-        self.fill = (lambda l, buf: buf.fill_(1e-4 * (1 + (l & 7)))) if refill != "copy" else None
+        self.fill = None
+        if refill == "fill":
+            self.fill = lambda l, buf: buf.fill_(1e-4 * (1 + (l & 7)))
+        elif refill == "memset":
+            from cuda.bindings import runtime as cudart
+
+            def memset(l, buf):
+                # bytes 0x38..0x3F: bf16 values 4.4e-5 .. 1.9, finite, a different one per layer
+                err, = cudart.cudaMemsetAsync(buf.data_ptr(), 0x38 + (l & 7), buf.numel() * buf.element_size(),
+                                              torch.cuda.current_stream(buf.device).cuda_stream)
+                if err != cudart.cudaError_t.cudaSuccess:
+                    raise RuntimeError(f"cudaMemsetAsync: {err}")
+            self.fill = memset
         self.arrival_desc = f"{refill}: {ARRIVALS[refill]}"
         self.desc = (f"rank 0's resident shard of 80 LLaMA-70B-shaped layers ({len(w['tensors'])} tensors, "
                      f"855,654,400 params each), D={D}, S={S} per layer, {L * S} owned params "
@@ -693,6 +740,68 @@ SWEEP_BLOCKS = [("config1_llama7b_d8", "llama7b_d8", 8), ("config2_llama7b_d32",
 NOMINAL_HBM_GBS = 8000.0
 
 
+def prefetch_sweep(z3, synth, dev, steps: int, L: int = 32, D: int = 8) -> dict:
+    """The backward sweep of one rank over the L = 32 blocks of LLaMA-7B at D = 8
+    with the next block's all-gather prefetched into one of two transient
+    buffers (PrefetchSweep), timed against the same sweep with every gather
+    serialised in front of its block.  Per block: the gather of the block's 8
+    shards (4 B per element of the block) and the fused kernel on this rank's
+    partition (42 B per owned element)."""
+    import torch
+    from fsdp_sharded_mixed_flat_b200.stream import PrefetchSweep
+    w = synth.WORKLOADS["llama7b_d8"]
+    plan = z3.zero3_plan([sh for _, sh in w["tensors"]], D, synth.ALIGN)
+    S, N_pad = plan.S, plan.N_pad
+    g = torch.Generator(device=dev).manual_seed(77)
+    flat = torch.randn(L * N_pad, generator=g, device=dev).mul_(0.02).to(torch.bfloat16)   # every rank's shards
+    shards = [[flat[l * N_pad + d * S:l * N_pad + (d + 1) * S] for d in range(D)] for l in range(L)]
+    master = torch.randn(L * S, generator=g, device=dev).mul_(0.02)
+    m, v = torch.zeros_like(master), torch.zeros_like(master)
+    pool = torch.cat([synth.contribution(S, S, seed=77, step=1, rank=d, sigma=w["sigma"], device=dev)
+                      for d in range(D)])
+    contribs = [pool[d * S:(d + 1) * S] for d in range(D)]
+    sweep = PrefetchSweep(plan, shards, 0, master, m, v)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    t = [0]
+
+    def hp():
+        t[0] += 1
+        return z3.adamw(step=t[0], **synth.ADAMW)
+    for prefetch in (True, False):
+        sweep.step(lambda l: contribs, hp(), prefetch=prefetch)
+        torch.cuda.synchronize(dev)
+        ev = {}
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            sweep.step(lambda l: contribs, hp(), prefetch=prefetch, events=ev)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        res[prefetch] = (a.elapsed_time(b) / 1e3 / steps,
+                         statistics.mean(x.elapsed_time(y) for x, y in ev["gather"]) / 1e3,
+                         statistics.mean(x.elapsed_time(y) for x, y in ev["k1"]) / 1e3)
+    t_pre, g_pre, k_pre = res[True]
+    t_ser, g_ser, k_ser = res[False]
+    out = {"blocks": L, "D": D, "rank": 0, "transient_gathered_buffers": 2,
+           "transient_bytes": sweep.transient_bytes,
+           "ledger_transient_bytes_2_blocks": z3.zero3_transient_bytes(N_pad, 2),
+           "sweep_ms_prefetch": 1e3 * t_pre, "sweep_ms_serial": 1e3 * t_ser,
+           "gather_ms_serial": 1e3 * g_ser, "k1_ms_serial": 1e3 * k_ser,
+           "gather_gbs_serial": 4 * N_pad / g_ser / 1e9, "k1_gbs_serial": 42 * S / k_ser / 1e9,
+           "gather_ms_overlapped": 1e3 * g_pre, "k1_ms_overlapped": 1e3 * k_pre,
+           "hidden_fraction_of_gather": (t_ser - t_pre) / (L * g_ser),
+           "owned_params_per_s_prefetch": L * S / t_pre,
+           "sweep_hbm_gbs_prefetch": L * (4 * N_pad + 42 * S) / t_pre / 1e9,
+           "note": "one GPU holds every rank's shards, so each gather reads HBM like the fused kernel does and "
+                   "both are bound by the same HBM: the prefetch can only fill the gaps between launches. On D "
+                   "GPUs the gather reads the peers' shards over NVLink, a separate resource, which is what the "
+                   "prefetch hides"}
+    del sweep, flat, shards, master, m, v, pool, contribs
+    torch.cuda.empty_cache()
+    return out
+
+
 def config_sweep(z3, synth, dev, steps: int, warmup: int, hbm_peak: float, refill: str) -> dict:
     """Every target configuration on this GPU, with fewer steps than the headline:
     the fused kernel's own time, rate and fraction of peak, and the whole step's
@@ -746,7 +855,171 @@ def config_sweep(z3, synth, dev, steps: int, warmup: int, hbm_peak: float, refil
         "target_k1_owned_params_per_s": target, "steps": shard_steps}
     del S4
     torch.cuda.empty_cache()
+    out["next2_prefetch_llama7b_L32_d8"] = prefetch_sweep(z3, synth, dev, max(2, steps // 5))
     return out
+
+
+class Clock:
+    """Time marks: CUDA events recorded on the current stream, or the host clock
+    when the step runs on the CPU (the host tests of the multi-rank path)."""
+
+    def __init__(self, device):
+        import torch
+        self.torch, self.device, self.cuda = torch, device, device.type == "cuda"
+
+    def mark(self):
+        if self.cuda:
+            e = self.torch.cuda.Event(enable_timing=True)
+            e.record(self.torch.cuda.current_stream(self.device))
+            return e
+        return time.perf_counter()
+
+    def seconds(self, a, b) -> float:
+        return a.elapsed_time(b) / 1e3 if self.cuda else b - a
+
+    def sync(self):
+        if self.cuda:
+            self.torch.cuda.synchronize(self.device)
+
+
+class CollectiveRunner:
+    """Rank r's share of the real D-GPU ZeRO-3 step, D = the world size, one
+    process per GPU: this rank's full bf16 gradient of the block goes through an
+    all-to-all (the reduce-scatter's data movement: rank r receives P_r of every
+    rank's gradient, in rank order), the fused kernel reduces it in rank order and
+    updates this rank's fp32 state and bf16 shard (owned layout), and an
+    all-gather assembles the block ("7.10 — Fully-sharded data parallel", §4,
+    §5.1).  With transport "peer" the kernels read the peers' gradients and
+    shards through CUDA IPC mappings with plain loads instead (peer.py)."""
+
+    def __init__(self, z3, synth, workload, world, rank, reduce_dtype, dev, kernels=None, transport="nccl"):
+        import torch
+        from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
+        w = synth.WORKLOADS[workload]
+        self.shapes = [s for _, s in w["tensors"]]
+        plan = z3.zero3_plan(self.shapes, world, synth.ALIGN)
+        self.plan, self.D, self.rank, self.mode, self.device = plan, world, rank, reduce_dtype, dev
+        N, N_pad, S = plan.N, plan.N_pad, plan.S
+        self.N, self.N_pad, self.S = N, N_pad, S
+        self.grad = synth.contribution(N, N_pad, seed=1000, step=1, rank=rank, sigma=w["sigma"], dist=w["dist"],
+                                       zero_frac=w.get("zero_frac", 0.0), device=dev)
+        self.master = synth.master_weights(N, N_pad, seed=1000, device=dev)[rank * S:(rank + 1) * S].clone()
+        self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
+        self.work = torch.zeros(S, dtype=torch.bfloat16, device=dev)
+        self.flat = torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)
+        self.transport = transport
+        if transport == "peer":
+            from fsdp_sharded_mixed_flat_b200.peer import PeerGroup, PeerZero3Step
+            self.stepper = PeerZero3Step(PeerGroup(), plan, self.grad, self.master, self.exp_avg, self.exp_avg_sq,
+                                         self.work, self.flat, reduce_dtype=reduce_dtype, kernels=kernels or z3)
+        else:
+            self.stepper = CollectiveZero3Step(plan, self.grad, self.master, self.exp_avg, self.exp_avg_sq,
+                                               self.work, self.flat, reduce_dtype=reduce_dtype, kernels=kernels or z3)
+        self.z3, self.synth = z3, synth
+        self.clock = Clock(dev)
+        self.marks = []
+        self.step_no = 0
+        self.units_per_step = S                         # owned params of this rank
+        self.k1_bytes_per_launch = (2 * world + 26) * S
+        self.gather_bytes = 2 * N_pad * (world - 1) // world   # bytes this rank receives in the all-gather
+        self.a2a_bytes = 2 * S * (world - 1)                     # gradient bytes it receives in the all-to-all
+
+    def step(self, timed: bool = False):
+        a = self.synth.ADAMW
+        self.step_no += 1
+        hp = self.z3.adamw(step=self.step_no, **a)
+        if self.transport == "peer":
+            m0 = self.clock.mark() if timed else None
+            self.stepper.step(hp)
+            if timed:
+                m1 = self.clock.mark()
+                self.marks.append((m0, m0, m1, m1))
+        else:
+            self.stepper.step(hp, mark=self.clock.mark if timed else None, marks=self.marks)
+
+
+def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, clocks=None, barrier=None):
+    """bench.py --gpus N, N > 1: the real D-GPU step with D = N, the block's
+    ranks on N GPUs (strong scaling: one block's N_pad owned params per step in
+    all, S = N_pad / N per rank).  Returns (the JSON line, the runner); only rank
+    0's line is printed."""
+    import torch
+    mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
+    R = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport=args.transport)
+    barrier = barrier or (lambda: torch.distributed.barrier())
+    for _ in range(args.warmup):
+        R.step()
+    R.clock.sync()
+    barrier()
+    if clocks is not None:
+        clocks.start()
+    t0 = R.clock.mark()
+    R.marks.clear()
+    for _ in range(args.steps):
+        R.step(timed=True)
+    t1 = R.clock.mark()
+    R.clock.sync()
+    barrier()
+    clk = clocks.stop() if clocks is not None else None
+    secs = R.clock.seconds(t0, t1)
+    phase = [[R.clock.seconds(m[k], m[k + 1]) for m in R.marks] for k in range(3)]
+    a2a_s, k1_s, ag_s = (statistics.mean(x) for x in phase)
+    job_secs, job_units = aggregate(secs, float(R.units_per_step) * args.steps, world,
+                                    dev if dev.type == "cuda" else None)
+
+    # ---- end to end: this rank's gradient from pinned host memory, its new shard back
+    pin = dev.type == "cuda"
+    host_grad = R.grad.cpu().pin_memory() if pin else R.grad.clone()
+    host_shard = torch.empty(R.S, dtype=torch.bfloat16, pin_memory=pin)
+    e2e_steps = max(1, args.e2e_steps)
+    barrier()
+    e0 = R.clock.mark()
+    for _ in range(e2e_steps):
+        R.grad.copy_(host_grad, non_blocking=True)
+        R.step()
+        host_shard.copy_(R.work, non_blocking=True)
+    e1 = R.clock.mark()
+    R.clock.sync()
+    barrier()
+    e2e_secs, e2e_units = aggregate(R.clock.seconds(e0, e1), float(R.units_per_step) * e2e_steps, world,
+                                    dev if dev.type == "cuda" else None)
+    hbm_peak, peak_kind = measured_peaks()
+    k1_gbs = R.k1_bytes_per_launch / k1_s / 1e9
+    step_s = secs / args.steps
+    line = {
+        "metric": METRIC, "value": job_units / job_secs, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: one block of {R.N} params ({R.N_pad} padded) sharded over the "
+                               f"{world} GPUs, S={R.S} owned per rank; bf16 gradients of every rank, fp32 master "
+                               f"N(0,0.02), AdamW lr=3e-4 b=(0.9,0.95) eps=1e-8 wd=0.1",
+                   "D": world, "reduce_dtype": args.reduce_dtype, "owned_params_per_step": R.N_pad,
+                   "transport": args.transport,
+                   "l2": "each rank streams its %.2f GB gradient and the gathered block per step (L2 126 MB), "
+                         "no flush" % (2 * R.N_pad / 1e9),
+                   "parallelism": (f"ZeRO-3 dp{world}: all-to-all of the gradients (NCCL), fused reduce/AdamW/cast "
+                                   f"on the owned partition, all-gather of the bf16 shards (NCCL)"
+                                   if args.transport == "nccl" else
+                                   f"ZeRO-3 dp{world}: the fused kernel reads every rank's gradient slice and the "
+                                   f"gather kernel every rank's shard through CUDA IPC mappings (plain loads)")},
+        "per_rank_owned_params_per_s": R.units_per_step / step_s,
+        "comm_nranks": world,
+        "collective": {"all_to_all_ms": 1e3 * a2a_s, "reduce_adamw_ms": 1e3 * k1_s, "all_gather_ms": 1e3 * ag_s,
+                       "collective_share_of_step": (a2a_s + ag_s) / max(step_s, 1e-12),
+                       "all_to_all_bytes_in_per_rank": R.a2a_bytes, "all_gather_bytes_in_per_rank": R.gather_bytes,
+                       "note": "with transport peer the whole step is one phase (reduce_adamw_ms holds it)"},
+        "kernels": {"reduce_adamw_ms": 1e3 * k1_s, "reduce_adamw_gbs": k1_gbs},
+        "roofline": {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
+                     "kernel": f"k_reduce_adamw_vec<{'fp32' if mode == 0 else 'bf16'}, D={world}> (owned layout)",
+                     "algorithmic_bytes_per_launch": R.k1_bytes_per_launch, "traffic": None},
+        "clocks": clk,
+        "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": 2 * R.N_pad,
+                "d2h_bytes_per_step": 2 * R.S, "steps": e2e_steps},
+        "gpu_launches": args.steps * (1 if args.transport == "nccl" else 2),
+        "ledger_bytes_per_device": ledger(z3, R.N, R.N_pad, world, R.N_pad),
+    }
+    return line, R
 
 
 def run_ours(args):
@@ -771,6 +1044,17 @@ def run_ours(args):
     from fsdp_sharded_mixed_flat_b200 import zero3 as z3
 
     mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
+    if world > 1 and not args.replicas:
+        props = torch.cuda.get_device_properties(dev)
+        uuid = getattr(props, "uuid", None)
+        line, R = run_collective(args, rank, world, dev, z3, synth,
+                                 clocks=ClockSampler(f"GPU-{uuid}" if uuid is not None else None))
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        del R
+        dist.barrier()
+        dist.destroy_process_group()
+        return 0
     if args.graph and (args.unflatten_copy or args.workload == "llama70b_shard"):
         raise SystemExit("--graph covers the block step without --unflatten-copy")
     if args.offload and (args.graph or args.stage != 3 or args.workload == "llama70b_shard"):
@@ -844,7 +1128,8 @@ def run_ours(args):
                    "reduce_dtype": "bf16" if mode == z3.Z3_REDUCE_BF16 else "fp32",
                    "owned_params_per_step": R.units_per_step,
                    "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (R.step_bytes / 1e9),
-                   "parallelism": f"replicas x{world} (one block per GPU, no collective)"},
+                   "parallelism": f"replicas x{world} (one block per GPU, its {R.D} ranks simulated on it; "
+                                  f"no collective)"},
         "step_hbm_gbs": R.step_bytes * args.steps * world / job_secs / 1e9,
         "kernels": {"reduce_adamw_ms": 1e3 * k1_avg_s, "reduce_adamw_gbs": k1_gbs,
                     "reduce_adamw_params_per_s": R.units_per_step / R.k1_launches_per_step / k1_avg_s,
@@ -872,13 +1157,29 @@ def run_ours(args):
                                  "note": "every node's sum (R launches) on one GPU, then the fold: on separate "
                                          "machines each node runs one node sum and the fold"}
     line.update(extra)
-    if getattr(R, "offload", False):
+    if getattr(R, "offload", None) == "state":
         # 12 B of state read and 12 B written per element cross PCIe; HBM carries the rest
         step_s = job_secs / args.steps
-        line["offload"] = {"pcie_gbs_per_direction": 12 * R.N_pad / step_s / 1e9,
+        line["offload"] = {"placement": "state streamed through the GPU, AdamW on the GPU",
+                           "pcie_bytes_per_param": 24, "pcie_gbs_per_direction": 12 * R.N_pad / step_s / 1e9,
                            "note": "fp32 master/m/v (12 B per element) cross PCIe each way every step; the step "
                                    "is bound by PCIe, not HBM, so the hbm roofline fields describe the kernels "
                                    "on the staged device buffers only"}
+        line["roofline"]["traffic"] = None
+    elif getattr(R, "offload", None) == "host":
+        step_s = job_secs / args.steps
+        down = R.offloaded.bytes_down
+        host_s = R.host_seconds[-args.steps * R.D:]
+        line["offload"] = {"placement": "AdamW on the host (the page's CPU-offload variant)",
+                           "pcie_bytes_per_param": (down + R.offloaded.bytes_up) / R.N_pad,
+                           "pcie_gbs_down": down / step_s / 1e9, "pcie_gbs_up": R.offloaded.bytes_up / step_s / 1e9,
+                           "host_adamw_ms_per_step": 1e3 * sum(host_s) / args.steps,
+                           "host_adamw_params_per_s": R.N_pad * args.steps / sum(host_s),
+                           "host_threads": os.cpu_count(),
+                           "note": "the averaged gradient (4 B, or 2 with the bf16 reduce) goes down and the bf16 "
+                                   "weights (2 B) come up per param; the step is bound by the host's AdamW "
+                                   "(30 B of host memory traffic per param), so the hbm roofline fields describe "
+                                   "the GPU's reduce kernels only"}
         line["roofline"]["traffic"] = None
     run_D, run_nodes, run_split = R.D, getattr(R, "nodes", 1), getattr(R, "split", False)
     if world == 1 and not args.no_sweep and args.workload == "llama7b_d8" and args.stage == 3 and \

@@ -33,6 +33,8 @@ the node sums have to cross between machines.
 """
 from __future__ import annotations
 
+from typing import Optional
+
 import torch
 import torch.distributed as dist
 
@@ -67,12 +69,21 @@ class CollectiveZero3Step:
         self.recv = torch.empty(D * S, dtype=torch.bfloat16, device=grad.device)
         self.slices = [self.recv[d * S:(d + 1) * S] for d in range(D)]
 
-    def step(self, hp: "z3.AdamW") -> None:
+    def step(self, hp: "z3.AdamW", mark=None, marks: Optional[list] = None) -> None:
+        """One step.  With mark (a callable returning a time mark, e.g. a CUDA
+        event recorded on the current stream) and marks (a list), the four marks
+        around the all-to-all, the fused kernel and the all-gather are appended to
+        marks as one tuple."""
         k = self.k
+        m0 = mark() if mark else None
         dist.all_to_all_single(self.recv, self.grad, group=self.group)
+        m1 = mark() if mark else None
         k.zero3_reduce_adamw(self.plan, self.rank, self.slices, self.master, self.exp_avg, self.exp_avg_sq,
                              self.work, hp, contrib_layout=k.Z3_CONTRIB_OWNED, reduce_dtype=self.reduce_dtype)
+        m2 = mark() if mark else None
         dist.all_gather_into_tensor(self.flat, self.work, group=self.group)
+        if mark:
+            marks.append((m0, m1, m2, mark()))
 
 
 def hybrid_groups(n_nodes: int, D: int, world_group=None):

@@ -1,6 +1,7 @@
 """Host logic of the benchmark on CPU: the whole-job aggregation over ranks
 (max of the per-rank times, sum of the units) on a world-size-2 gloo group,
-and the clock-sample parsing."""
+the multi-GPU path (the D-GPU step with D = N) end to end on two gloo ranks
+with the oracle standing in for the kernels, and the clock-sample parsing."""
 import os
 import socket
 
@@ -76,3 +77,77 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["metric"] == bench.METRIC
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["cpu_baseline"]["cores"] == 1
+
+
+def _collective_worker(rank, world, port, mode, out):
+    import argparse
+
+    import numpy as np
+    import torch
+
+    import synth
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    from test_collective_host import OracleKernels
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    args = argparse.Namespace(workload="tiny_gpt", steps=2, warmup=1, e2e_steps=1,
+                              reduce_dtype="bf16" if mode else "fp32", transport="nccl")
+    line, R = bench.run_collective(args, rank, world, torch.device("cpu"), z3, synth, kernels=OracleKernels(),
+                                   barrier=dist.barrier)
+    out[rank] = (line, R.master.numpy().copy(), R.exp_avg.numpy().copy(), R.exp_avg_sq.numpy().copy(),
+                 R.work.view(torch.int16).numpy().view(np.uint16).copy(),
+                 R.flat.view(torch.int16).numpy().view(np.uint16).copy(), R.step_no)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode):
+    """bench.py's N > 1 path (run_collective: the D-GPU step, warm-up, timed
+    steps, max-over-ranks aggregation, the end-to-end leg, the JSON line) on two
+    gloo ranks; the oracle stands in for the kernels, the collectives move the
+    real bytes.  Every rank's state equals one oracle run over both ranks."""
+    import numpy as np
+
+    import oracle
+    import synth
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as m:
+        out = m.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_collective_worker, args=(r, world, port, mode, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(300)
+            assert p.exitcode == 0
+        res = dict(out)
+    line = res[0][0]
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "comm_nranks",
+              "collective", "per_rank_owned_params_per_s"):
+        assert k in line, k
+    assert line["n_gpus"] == 2 and line["comm_nranks"] == 2 and line["scaling"] == "strong"
+    assert line["config"]["D"] == 2 and line["value"] > 0 and line["e2e"]["value"] > 0
+    assert line["metric"] == bench.METRIC and line["steps"] == 2 and line["warmup"] == 1
+    w = synth.WORKLOADS["tiny_gpt"]
+    numels = [synth.numel(s) for _, s in w["tensors"]]
+    _, N, N_pad, S = oracle.plan(numels, world, synth.ALIGN)
+    assert line["config"]["owned_params_per_step"] == N_pad
+    steps = res[0][6]
+    assert steps == 1 + 2 + 1                          # warm-up, timed, end to end
+    p = synth.master_weights(N, N_pad, seed=1000).numpy().copy()
+    mm, vv, ww = np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.uint16)
+    c = [synth.bf16_bits(synth.contribution(N, N_pad, seed=1000, step=1, rank=d, sigma=w["sigma"]))
+         for d in range(world)]
+    for t in range(1, steps + 1):
+        oracle.reduce_adamw(c, S, -1, p, mm, vv, ww, oracle.hp(step=t), reduce_dtype=mode)
+    for r in range(world):
+        _, rp, rm, rv, rw, rflat, _ = res[r]
+        sl = slice(r * S, (r + 1) * S)
+        assert np.array_equal(rp.view(np.uint32), p[sl].view(np.uint32)), f"master rank {r}"
+        assert np.array_equal(rm.view(np.uint32), mm[sl].view(np.uint32)), f"exp_avg rank {r}"
+        assert np.array_equal(rv.view(np.uint32), vv[sl].view(np.uint32)), f"exp_avg_sq rank {r}"
+        assert np.array_equal(rw, ww[sl]), f"work rank {r}"
+        assert np.array_equal(rflat, ww), f"gathered block rank {r}"

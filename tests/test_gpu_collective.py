@@ -93,3 +93,32 @@ def test_one_rank_nccl_hybrid_step_matches_oracle(z3, nccl_one_rank, mode):
     assert_f32_parity(f32_host(v), hv, "exp_avg_sq")
     assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16")
     assert np.array_equal(synth.bf16_bits(flat), hw)
+
+
+def test_bench_multi_gpu_path_on_a_one_rank_nccl_group(z3, nccl_one_rank):
+    """bench.py's N > 1 path (run_collective) on a one-rank NCCL group with the
+    real kernels: CUDA-event timing of the all-to-all, the fused kernel and the
+    all-gather, the end-to-end leg, the JSON line; the rank's state after every
+    step equals the oracle's."""
+    import argparse
+
+    import bench
+    args = argparse.Namespace(workload="tiny_gpt", steps=3, warmup=2, e2e_steps=2, reduce_dtype="fp32",
+                              transport="nccl")
+    line, R = bench.run_collective(args, 0, 1, torch.device("cuda", 0), z3, synth)
+    assert line["n_gpus"] == 1 and line["comm_nranks"] == 1 and line["value"] > 0 and line["e2e"]["value"] > 0
+    assert line["collective"]["reduce_adamw_ms"] > 0 and line["gpu_launches"] == 3
+    w = synth.WORKLOADS["tiny_gpt"]
+    numels = [synth.numel(s) for _, s in w["tensors"]]
+    _, N, N_pad, S = oracle.plan(numels, 1, synth.ALIGN)
+    p = synth.master_weights(N, N_pad, seed=1000, device="cuda").cpu().numpy().copy()
+    m, v, wk = np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.uint16)
+    c = [synth.bf16_bits(synth.contribution(N, N_pad, seed=1000, step=1, rank=0, sigma=w["sigma"], device="cuda"))]
+    for t in range(1, R.step_no + 1):
+        oracle.reduce_adamw(c, S, -1, p, m, v, wk, oracle_hp(t))
+    torch.cuda.synchronize()
+    assert_f32_parity(f32_host(R.master), p, "master")
+    assert_f32_parity(f32_host(R.exp_avg), m, "exp_avg")
+    assert_f32_parity(f32_host(R.exp_avg_sq), v, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(R.work), wk, "work_bf16")
+    assert np.array_equal(synth.bf16_bits(R.flat), wk)
