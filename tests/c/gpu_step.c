@@ -14,7 +14,10 @@
  *     ("7.10 — Fully-sharded data parallel (FSDP / ZeRO-3)", §3 and §5.1);
  *   - 3 steps of zero3_reduce_adamw_hybrid with 3 nodes of 4 ranks
  *     ("Building GPT from Scratch — Part 8", "HYBRID_SHARD: The Multi-Node
- *     Strategy").
+ *     Strategy");
+ *   - 3 steps of the CPU-offload step ("7.10", §8): zero3_reduce_scatter of
+ *     every rank's partition on the GPU, the gradient copied down, and
+ *     zero3_host_adamw on host memory.
  * Inputs are drawn from splitmix64 (Steele, Lea and Flood, "Fast splittable
  * pseudorandom number generators", 2014), keyed by (step, contributor,
  * element), and fed identically to both sides.  Exit status 0 means every
@@ -40,6 +43,8 @@ int ref_reduce_adamw(int32_t D, int64_t S, int32_t rank, const uint16_t* const* 
 int ref_reduce_adamw_hybrid(int32_t R, int32_t D, int64_t S, int32_t rank, const uint16_t* const* contrib,
                             int32_t layout, float* master, float* exp_avg, float* exp_avg_sq,
                             uint16_t* work_bf16, int32_t reduce_dtype, const oracle_hp* hp);
+int ref_reduce_scatter(int32_t D, int64_t S, int32_t rank, const uint16_t* const* contrib, int32_t layout,
+                       int32_t reduce_dtype, float* out);
 void ref_all_gather(int32_t D, int64_t S, const uint16_t* const* shards, uint16_t* flat);
 void ref_unflatten(const uint16_t* flat, int32_t n_tensors, const int64_t* offset, const int64_t* numel,
                    uint16_t* const* out);
@@ -223,6 +228,89 @@ static void run(int32_t mode, int32_t nodes)
            (long long)N_pad, failures ? "MISMATCH" : "bit-identical to the oracle");
 }
 
+/* The CPU-offload step: per rank partition, the averaged gradient on the GPU
+ * (compared with the oracle's reduce-scatter), copied down, then AdamW and
+ * the cast on the host; the host state is compared with the oracle's step. */
+static void run_offload(int32_t mode)
+{
+    const z3_tensor_spec t[NT] = {spec(1000, 1), spec(257, 33), spec(4097, 1)};
+    z3_plan* plan = NULL;
+    CHECK(zero3_plan(t, NT, D, 8, &plan) == Z3_OK);
+    int64_t N = 0, N_pad = 0, S = 0;
+    zero3_plan_info(plan, NULL, NULL, NULL, &N, &N_pad, &S);
+    const size_t gsz = mode == Z3_REDUCE_FP32 ? 4 : 2;
+
+    float* hp_ = calloc((size_t)N_pad, 4); /* the oracle's state */
+    float* hm = calloc((size_t)N_pad, 4);
+    float* hv = calloc((size_t)N_pad, 4);
+    uint16_t* hw = calloc((size_t)N_pad, 2);
+    float* op = calloc((size_t)N_pad, 4); /* the offloaded state, on the host */
+    float* om = calloc((size_t)N_pad, 4);
+    float* ov = calloc((size_t)N_pad, 4);
+    uint16_t* ow = calloc((size_t)N_pad, 2);
+    void* hg = calloc((size_t)S, gsz);
+    float* ref_g = calloc((size_t)S, 4);
+    uint16_t* hc[D];
+    const uint16_t* dc[D];
+    for (int64_t i = 0; i < N; ++i) hp_[i] = op[i] = (float)((uniform(0, 998, (uint64_t)i) - 0.5) * 0.08);
+    for (int c = 0; c < D; ++c) {
+        hc[c] = calloc((size_t)N_pad, 2);
+        dc[c] = dalloc((size_t)N_pad * 2);
+    }
+    void* dg = dalloc((size_t)S * gsz);
+
+    for (int64_t step = 1; step <= 3; ++step) {
+        for (int c = 0; c < D; ++c) {
+            for (int64_t i = 0; i < N; ++i) hc[c][i] = grad_bits((uint64_t)step + 10, (uint64_t)c, (uint64_t)i);
+            CUDA(cudaMemcpy((void*)dc[c], hc[c], (size_t)N_pad * 2, cudaMemcpyHostToDevice));
+        }
+        const z3_adamw hp = {3e-4, 0.9, 0.95, 1e-8, 0.1, step};
+        const oracle_hp ohp = {3e-4, 0.9, 0.95, 1e-8, 0.1, step};
+        for (int32_t r = 0; r < D; ++r) {
+            CHECK(zero3_reduce_scatter(plan, r, dc, Z3_CONTRIB_FULL, mode, dg, NULL) == Z3_OK);
+            CUDA(cudaMemcpy(hg, dg, (size_t)S * gsz, cudaMemcpyDeviceToHost));
+            CHECK(ref_reduce_scatter(D, S, r, (const uint16_t* const*)hc, 0, mode, ref_g) == 0);
+            for (int64_t j = 0; j < S; ++j) {
+                float g;
+                if (mode == Z3_REDUCE_FP32) {
+                    g = ((const float*)hg)[j];
+                } else {
+                    const uint32_t u = (uint32_t)((const uint16_t*)hg)[j] << 16;
+                    memcpy(&g, &u, sizeof g);
+                }
+                if (memcmp(&g, &ref_g[j], 4) != 0) {
+                    CHECK(!"reduce-scatter output differs from the oracle");
+                    break;
+                }
+            }
+            CHECK(zero3_host_adamw(S, hg, mode, op + r * S, om + r * S, ov + r * S, ow + r * S, &hp, 3) == Z3_OK);
+        }
+        CHECK(ref_reduce_adamw(D, S, -1, (const uint16_t* const*)hc, 0, hp_, hm, hv, hw, mode, &ohp) == 0);
+        CHECK(memcmp(op, hp_, (size_t)N_pad * 4) == 0);
+        CHECK(memcmp(om, hm, (size_t)N_pad * 4) == 0);
+        CHECK(memcmp(ov, hv, (size_t)N_pad * 4) == 0);
+        CHECK(memcmp(ow, hw, (size_t)N_pad * 2) == 0);
+    }
+    for (int c = 0; c < D; ++c) {
+        CUDA(cudaFree((void*)dc[c]));
+        free(hc[c]);
+    }
+    CUDA(cudaFree(dg));
+    free(hp_);
+    free(hm);
+    free(hv);
+    free(hw);
+    free(op);
+    free(om);
+    free(ov);
+    free(ow);
+    free(hg);
+    free(ref_g);
+    zero3_plan_free(plan);
+    printf("mode %d, CPU offload (GPU reduce-scatter, host AdamW), N=%lld N_pad=%lld: %s\n", (int)mode,
+           (long long)N, (long long)N_pad, failures ? "MISMATCH" : "bit-identical to the oracle");
+}
+
 int main(void)
 {
     int count = 0;
@@ -233,6 +321,7 @@ int main(void)
     for (int32_t mode = Z3_REDUCE_FP32; mode <= Z3_REDUCE_BF16; ++mode) {
         run(mode, 1);
         run(mode, NODES);
+        run_offload(mode);
     }
     return failures ? 1 : 0;
 }
