@@ -83,7 +83,7 @@ def _worker(rank, world, port, mode, steps, out):
 @pytest.mark.parametrize("world,mode", [(2, 0), (4, 0), (4, 1)])
 def test_collective_step_equals_one_oracle_run_over_all_ranks(world, mode):
     steps = 3
-    with mp.Manager() as manager:
+    with mp.get_context("spawn").Manager() as manager:
         out = manager.dict()
         mp.spawn(_worker, args=(world, _free_port(), mode, steps, out), nprocs=world, join=True)
         results = dict(out)
@@ -155,7 +155,7 @@ def test_collective_hybrid_step_equals_the_two_level_oracle(R, D, mode):
     run of the two-level reduction over all R*D ranks, bit for bit, and every
     replica of a local rank holds the same state."""
     steps = 3
-    with mp.Manager() as manager:
+    with mp.get_context("spawn").Manager() as manager:
         out = manager.dict()
         mp.spawn(_hybrid_worker, args=(R, D, _free_port(), mode, steps, out), nprocs=R * D, join=True)
         results = dict(out)
