@@ -76,7 +76,7 @@ ARRIVALS = {
 DEFAULT_ARRIVAL = "memset"
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
@@ -122,7 +122,7 @@ def parse_args():
     ap.add_argument("--stage", type=int, choices=[1, 2, 3], default=3,
                     help="3: ZeRO-3 step (fused reduce/AdamW/cast, then the gather of the shards); "
                          "1 or 2: the fused kernel also all-gathers into the replicated bf16 weights")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def host_info() -> dict:
@@ -353,22 +353,57 @@ def sample_parity(z3, dev, kept: dict, reduce_dtype: int, split: bool = False) -
             "work_bf16_max_ulp": ulps(gw, kept["wk"]), "bit_exact": bool(exact)}
 
 
+L2_NOTE = ("inputs larger than L2 (126 MB): every step streams the block's contributions and fp32 state "
+           "through HBM, so no flush is needed between steps")
+
+
+def contract_config(args, world: int, D: int, nodes: int, owned: int) -> dict:
+    """The `config` both arms print (ours and the reference arm): the workload and
+    the options that define the step, so that the two lines can be matched."""
+    multi = world > 1 and not args.replicas
+    if multi:
+        par = (f"ZeRO-3 dp{world}: NCCL all-to-all of the gradients, fused reduce/AdamW/cast on each rank's "
+               f"partition, NCCL all-gather of the bf16 shards" if args.transport == "nccl" else
+               f"ZeRO-3 dp{world}: the kernels read every rank's gradient slice and shard through CUDA IPC "
+               f"mappings (plain loads)")
+    else:
+        par = (f"replicas x{world}" if world > 1 else "one GPU") + \
+            f", the block's {D if nodes == 1 else f'{nodes} x {D}'} ranks simulated on each GPU (no collective)"
+    options = [o for o, on in (("graph", args.graph), ("unflatten_copy", args.unflatten_copy),
+                               ("split", args.split)) if on]
+    if args.offload:
+        options.append(f"offload_{args.offload}")
+    if args.workload == "llama70b_shard":
+        options.append(f"arrival_{args.refill}")
+    return {"workload": args.workload, "D": D, "nodes": nodes, "stage": args.stage,
+            "reduce_dtype": args.reduce_dtype, "owned_params_per_step": owned, "options": options,
+            "l2": L2_NOTE, "parallelism": par}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
+    import oracle
+    import synth
     steps = max(1, args.steps)
     # each step is a bounded sample (2^20 elements) so that K steps stay within minutes
     sample = min(args.cpu_sample, 1 << 20)
     mode = 1 if args.reduce_dtype == "bf16" else 0
+    multi = world > 1 and not args.replicas
+    w = synth.WORKLOADS[oracle_workload(args.workload)]
+    D = world if multi else (args.D or (8 if args.workload == "llama70b_shard" else w["D"]))
+    nodes = 1 if multi else (args.nodes or w.get("nodes", 1))
+    _, _, N_pad, S = oracle.plan([synth.numel(sh) for _, sh in w["tensors"]], D, synth.ALIGN)
+    owned = w["layers"] * S if args.workload == "llama70b_shard" else N_pad
     if args.warmup > 0:
-        oracle_sample(args.workload, min(sample, 1 << 16), 1, D=args.D, reduce_dtype=mode)
-    value, secs, desc, _ = oracle_sample(args.workload, sample, steps, D=args.D, reduce_dtype=mode)
+        oracle_sample(args.workload, min(sample, 1 << 16), 1, D=D, reduce_dtype=mode, nodes=nodes)
+    value, secs, desc, _ = oracle_sample(args.workload, sample, steps, D=D, reduce_dtype=mode, nodes=nodes)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic", "config": {"workload": args.workload, "sample_elements": sample,
-                                                      "D": args.D or None, "reduce_dtype": args.reduce_dtype},
+            "higher_is_better": True, "scaling": "strong" if multi else "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic", "config": contract_config(args, world, D, nodes, owned),
+            "sample_elements_per_step": sample,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                              "host": host_info()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -990,18 +1025,10 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
         "metric": METRIC, "value": job_units / job_secs, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: one block of {R.N} params ({R.N_pad} padded) sharded over the "
-                               f"{world} GPUs, S={R.S} owned per rank; bf16 gradients of every rank, fp32 master "
-                               f"N(0,0.02), AdamW lr=3e-4 b=(0.9,0.95) eps=1e-8 wd=0.1",
-                   "D": world, "reduce_dtype": args.reduce_dtype, "owned_params_per_step": R.N_pad,
-                   "transport": args.transport,
-                   "l2": "each rank streams its %.2f GB gradient and the gathered block per step (L2 126 MB), "
-                         "no flush" % (2 * R.N_pad / 1e9),
-                   "parallelism": (f"ZeRO-3 dp{world}: all-to-all of the gradients (NCCL), fused reduce/AdamW/cast "
-                                   f"on the owned partition, all-gather of the bf16 shards (NCCL)"
-                                   if args.transport == "nccl" else
-                                   f"ZeRO-3 dp{world}: the fused kernel reads every rank's gradient slice and the "
-                                   f"gather kernel every rank's shard through CUDA IPC mappings (plain loads)")},
+        "config": contract_config(args, world, world, 1, R.N_pad),
+        "workload_desc": (f"{args.workload}: one block of {R.N} params ({R.N_pad} padded) sharded over the {world} "
+                          f"GPUs, S={R.S} owned per rank; bf16 gradients of every rank, fp32 master N(0,0.02), "
+                          f"AdamW lr=3e-4 b=(0.9,0.95) eps=1e-8 wd=0.1; transport {args.transport}"),
         "per_rank_owned_params_per_s": R.units_per_step / step_s,
         "comm_nranks": world,
         "collective": {"all_to_all_ms": 1e3 * a2a_s, "reduce_adamw_ms": 1e3 * k1_s, "all_gather_ms": 1e3 * ag_s,
@@ -1123,13 +1150,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {R.desc}", "D": R.D, "nodes": getattr(R, "nodes", 1),
-                   "stage": getattr(R, "stage", 3),
-                   "reduce_dtype": "bf16" if mode == z3.Z3_REDUCE_BF16 else "fp32",
-                   "owned_params_per_step": R.units_per_step,
-                   "l2": "inputs larger than L2: each step streams %.2f GB (L2 126 MB), no flush" % (R.step_bytes / 1e9),
-                   "parallelism": f"replicas x{world} (one block per GPU, its {R.D} ranks simulated on it; "
-                                  f"no collective)"},
+        "config": contract_config(args, world, R.D, getattr(R, "nodes", 1), R.units_per_step),
+        "workload_desc": f"{args.workload}: {R.desc}; each step streams {R.step_bytes / 1e9:.2f} GB",
         "step_hbm_gbs": R.step_bytes * args.steps * world / job_secs / 1e9,
         "kernels": {"reduce_adamw_ms": 1e3 * k1_avg_s, "reduce_adamw_gbs": k1_gbs,
                     "reduce_adamw_params_per_s": R.units_per_step / R.k1_launches_per_step / k1_avg_s,

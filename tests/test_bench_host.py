@@ -77,11 +77,11 @@ def test_reference_arm_prints_one_contract_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["metric"] == bench.METRIC
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["cpu_baseline"]["cores"] == 1
+    # the same config our arm prints for the default workload (7B block, D = 8, one GPU)
+    assert d["config"] == bench.contract_config(bench.parse_args([]), 1, 8, 1, 202_383_360)
 
 
 def _collective_worker(rank, world, port, mode, out):
-    import argparse
-
     import numpy as np
     import torch
 
@@ -90,8 +90,8 @@ def _collective_worker(rank, world, port, mode, out):
     from test_collective_host import OracleKernels
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
-    args = argparse.Namespace(workload="tiny_gpt", steps=2, warmup=1, e2e_steps=1,
-                              reduce_dtype="bf16" if mode else "fp32", transport="nccl")
+    args = bench.parse_args(["--gpus", str(world), "--workload", "tiny_gpt", "--steps", "2", "--warmup", "1",
+                             "--e2e-steps", "1", "--reduce-dtype", "bf16" if mode else "fp32"])
     line, R = bench.run_collective(args, rank, world, torch.device("cpu"), z3, synth, kernels=OracleKernels(),
                                    barrier=dist.barrier)
     out[rank] = (line, R.master.numpy().copy(), R.exp_avg.numpy().copy(), R.exp_avg_sq.numpy().copy(),

@@ -100,11 +100,8 @@ def test_bench_multi_gpu_path_on_a_one_rank_nccl_group(z3, nccl_one_rank):
     real kernels: CUDA-event timing of the all-to-all, the fused kernel and the
     all-gather, the end-to-end leg, the JSON line; the rank's state after every
     step equals the oracle's."""
-    import argparse
-
     import bench
-    args = argparse.Namespace(workload="tiny_gpt", steps=3, warmup=2, e2e_steps=2, reduce_dtype="fp32",
-                              transport="nccl")
+    args = bench.parse_args(["--workload", "tiny_gpt", "--steps", "3", "--warmup", "2", "--e2e-steps", "2"])
     line, R = bench.run_collective(args, 0, 1, torch.device("cuda", 0), z3, synth)
     assert line["n_gpus"] == 1 and line["comm_nranks"] == 1 and line["value"] > 0 and line["e2e"]["value"] > 0
     assert line["collective"]["reduce_adamw_ms"] > 0 and line["gpu_launches"] == 3
