@@ -521,11 +521,12 @@ class BlockRunner:
                      "averaged gradient is reduced on the GPU, copied down, updated by libzero3's host threads, "
                      "and the bf16 weights copied up (pipelined over partitions)")
             self.k1_name = (f"k_node_sum_vec<{'fp32' if reduce_dtype == 0 else 'bf16'}, D={D}, scaled> "
-                            "(the reduce-scatter's reduction alone, one launch per partition)")
-            self.k1_launches_per_step = D
-            self.k1_bytes_per_launch = (2 * D + gb) * self.S
-            self.launches_per_step = D + 1
-            self.step_bytes = self.k1_bytes_per_launch * D + 4 * self.N_pad
+                            "(the reduce-scatter's reduction alone, one launch per pipeline unit)")
+            units = len(self.offloaded.units)
+            self.k1_launches_per_step = units
+            self.k1_bytes_per_launch = (2 * D + gb) * self.N_pad / units      # the mean unit
+            self.launches_per_step = units + 1
+            self.step_bytes = (2 * D + gb) * self.N_pad + 4 * self.N_pad
         self.desc = (f"{len(self.shapes)} tensors, N={self.N}, N_pad={self.N_pad}, S={self.S} per rank, D={D}, "
                      f"bf16 grads {w['dist']}(sigma={w['sigma']}), fp32 master N(0,0.02), AdamW lr=3e-4 "
                      f"b=(0.9,0.95) eps=1e-8 wd=0.1; step = plan + ledger + {what}")
@@ -1191,7 +1192,7 @@ def run_ours(args):
     elif getattr(R, "offload", None) == "host":
         step_s = job_secs / args.steps
         down = R.offloaded.bytes_down
-        host_s = R.host_seconds[-args.steps * R.D:]
+        host_s = R.host_seconds[-args.steps * len(R.offloaded.units):]
         line["offload"] = {"placement": "AdamW on the host (the page's CPU-offload variant)",
                            "pcie_bytes_per_param": (down + R.offloaded.bytes_up) / R.N_pad,
                            "pcie_gbs_down": down / step_s / 1e9, "pcie_gbs_up": R.offloaded.bytes_up / step_s / 1e9,

@@ -99,87 +99,108 @@ class HostAdamWOffload:
     over PCIe -- 4 bytes per parameter down (2 with the bf16 reduce) and 2 up,
     against the 12 bytes of state each way that OffloadedState moves.
 
-    Per step, partition by partition (P_0 .. P_{D-1}), pipelined:
-      compute stream  zero3_reduce_scatter(rank r) -> one of `n_stage` device
-                      staging buffers (the averaged gradient of P_r);
-      copy-down       the staging buffer -> P_r's slot of a pinned host
+    Per step, unit by unit (each partition P_0 .. P_{D-1} cut into `chunks`
+    consecutive pieces), pipelined:
+      compute stream  zero3_reduce_scatter of the unit -> one of `n_stage`
+                      device staging buffers (the unit's averaged gradient);
+      copy-down       the staging buffer -> the unit's slot of a pinned host
                       gradient buffer;
-      host            waits for that copy only, then zero3_host_adamw on P_r
-                      (libzero3's host threads: same operations, same bits as
-                      the GPU kernels) writing P_r's bf16 weights to a pinned
+      host            waits for that copy only, then zero3_host_adamw on the
+                      unit (libzero3's host threads: same operations, same bits
+                      as the GPU kernels) writing its bf16 weights to a pinned
                       host buffer;
-      copy-up         P_r's bf16 weights -> the device working shard.
-    The GPU reduces P_{r+1} and copies it down while the host updates P_r, and
-    P_r's weights go up while the host updates P_{r+1}.  The step returns once
-    the last host update has run; the caller's stream is ordered after the
-    last copy up, so kernels it enqueues next see every new weight.
+      copy-up         the unit's bf16 weights -> the device working shard.
+    The GPU reduces and copies the next units down while the host updates this
+    one, and this unit's weights go up while the host updates the next.  Smaller
+    units start the host sooner and leave a shorter copy up at the end.  A unit
+    of rank r's partition is reduced as a plan of its own (D ranks of the
+    unit's length, the contributions in the owned layout at the unit's offset),
+    so the arithmetic is the partition's, element for element.  The step
+    returns once the last host update has run; the caller's stream is ordered
+    after the last copy up, so kernels it enqueues next see every new weight.
     """
 
     def __init__(self, plan: "z3.Plan", master: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
-                 work_bf16: torch.Tensor, device, n_stage: int = 2, reduce_dtype: int = z3.Z3_REDUCE_FP32,
-                 n_threads: int = 0):
+                 work_bf16: torch.Tensor, device, n_stage: int = 3, reduce_dtype: int = z3.Z3_REDUCE_FP32,
+                 n_threads: int = 0, chunks: int = 4):
         S, N_pad = plan.S, plan.N_pad
         for name, t in (("master", master), ("exp_avg", exp_avg), ("exp_avg_sq", exp_avg_sq)):
             if t.device.type != "cpu" or t.dtype != torch.float32 or t.numel() < N_pad or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous host float32 tensor of N_pad elements")
         if work_bf16.device.type != "cuda" or work_bf16.numel() < N_pad:
             raise ValueError("work_bf16 must be a device bf16 tensor of N_pad elements")
-        if n_stage < 1:
-            raise ValueError("n_stage must be >= 1")
+        if n_stage < 1 or chunks < 1:
+            raise ValueError("n_stage and chunks must be >= 1")
         self.plan, self.reduce_dtype, self.n_threads = plan, reduce_dtype, n_threads
         self.host = (master, exp_avg, exp_avg_sq)
         self.work = work_bf16
         self.device = torch.device(device)
+        # units: (rank, first element within the partition, length); cuts on 128-element
+        # boundaries keep every unit's vectors 16-byte aligned
+        step = max(128, -(-(-(-S // chunks)) // 128) * 128)
+        self.units = [(r, c0, min(step, S - c0)) for r in range(plan.D) for c0 in range(0, S, step)]
+        self._plans = {}
         gdt = torch.float32 if reduce_dtype == z3.Z3_REDUCE_FP32 else torch.bfloat16
         self.grad_host = torch.empty(N_pad, dtype=gdt, pin_memory=True)
         self.work_host = torch.empty(N_pad, dtype=torch.bfloat16, pin_memory=True)
-        self.stage = [torch.empty(S, dtype=gdt, device=self.device) for _ in range(n_stage)]
+        self.stage = [torch.empty(min(step, max(S, 1)), dtype=gdt, device=self.device) for _ in range(n_stage)]
         self.compute = torch.cuda.Stream(self.device)
         self.down = torch.cuda.Stream(self.device)
         self.up = torch.cuda.Stream(self.device)
         self.reduced = [torch.cuda.Event() for _ in range(n_stage)]
         self.staged_free = [torch.cuda.Event() for _ in range(n_stage)]
-        self.arrived = [torch.cuda.Event() for _ in range(plan.D)]      # P_r's gradient is on the host
+        self.arrived = [torch.cuda.Event() for _ in self.units]      # the unit's gradient is on the host
         self.bytes_down = N_pad * self.grad_host.element_size()
         self.bytes_up = N_pad * 2
 
-    def _reduce_and_send(self, contribs, r: int, k_events) -> None:
-        plan, S = self.plan, self.plan.S
-        b = r % len(self.stage)
+    def _unit_plan(self, length: int) -> "z3.Plan":
+        if length not in self._plans:
+            self._plans[length] = z3.zero3_plan([(length * self.plan.D,)], self.plan.D, 1)
+        return self._plans[length]
+
+    def _reduce_and_send(self, contribs, u: int, k_events) -> None:
+        r, c0, n = self.units[u]
+        lo = r * self.plan.S + c0
+        b = u % len(self.stage)
         self.compute.wait_event(self.staged_free[b])   # the staging buffer's previous copy down is done
         if k_events is not None:
-            k_events[r][0].record(self.compute)
-        z3.zero3_reduce_scatter(plan, r, contribs, self.stage[b], contrib_layout=z3.Z3_CONTRIB_FULL,
-                                reduce_dtype=self.reduce_dtype, stream=self.compute)
+            k_events[u][0].record(self.compute)
+        z3.zero3_reduce_scatter(self._unit_plan(n), 0, [c[lo:lo + n] for c in contribs], self.stage[b],
+                                contrib_layout=z3.Z3_CONTRIB_OWNED, reduce_dtype=self.reduce_dtype,
+                                stream=self.compute)
         if k_events is not None:
-            k_events[r][1].record(self.compute)
+            k_events[u][1].record(self.compute)
         self.reduced[b].record(self.compute)
         with torch.cuda.stream(self.down):
             self.down.wait_event(self.reduced[b])
-            self.grad_host[r * S:(r + 1) * S].copy_(self.stage[b], non_blocking=True)
+            self.grad_host[lo:lo + n].copy_(self.stage[b][:n], non_blocking=True)
             self.staged_free[b].record(self.down)
-            self.arrived[r].record(self.down)
+            self.arrived[u].record(self.down)
 
     def step(self, contribs: Sequence[torch.Tensor], hp: "z3.AdamW", k_events: Optional[Sequence] = None,
              host_seconds: Optional[list] = None) -> None:
         """One optimiser step over every partition.  contribs: the D device bf16
-        contributions in the full layout.  k_events, if given, holds D (start, end)
-        event pairs recorded around the reduce kernels; host_seconds, if given,
-        receives the wall time of each partition's host update."""
+        contributions in the full layout.  k_events, if given, holds one (start,
+        end) event pair per unit (len(self.units)), recorded around the reduce
+        kernels; host_seconds, if given, receives the wall time of each unit's
+        host update."""
         import time
-        plan, S, D = self.plan, self.plan.S, self.plan.D
+        if len(contribs) != self.plan.D:
+            raise ValueError(f"need {self.plan.D} contributions")
         caller = torch.cuda.current_stream(self.device)
         for s in (self.compute, self.down, self.up):
             s.wait_stream(caller)
         n = len(self.stage)
-        for r in range(min(n, D)):
-            self._reduce_and_send(contribs, r, k_events)
+        U = len(self.units)
+        for u in range(min(n, U)):
+            self._reduce_and_send(contribs, u, k_events)
         master, exp_avg, exp_avg_sq = self.host
-        for r in range(D):
-            self.arrived[r].synchronize()                # only this partition's copy down
-            if r + n < D:
-                self._reduce_and_send(contribs, r + n, k_events)
-            sl = slice(r * S, (r + 1) * S)
+        for u in range(U):
+            self.arrived[u].synchronize()                # only this unit's copy down
+            if u + n < U:
+                self._reduce_and_send(contribs, u + n, k_events)
+            r, c0, length = self.units[u]
+            sl = slice(r * self.plan.S + c0, r * self.plan.S + c0 + length)
             t0 = time.perf_counter()
             z3.zero3_host_adamw(self.grad_host[sl], master[sl], exp_avg[sl], exp_avg_sq[sl], self.work_host[sl], hp,
                                 n_threads=self.n_threads)

@@ -59,10 +59,10 @@ def test_reduce_scatter_matches_oracle(z3, numels, D, A, mode):
 
 
 @pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
-@pytest.mark.parametrize("numels,D,A,n_stage", [([300, 77, 1000], 4, 8, 2), ([123457], 8, 128, 1),
-                                                ([4097, 33], 32, 128, 3), ([999], 5, 1, 2),
-                                                ([2 ** 20 + 5], 8, 128, 2)])
-def test_host_adamw_offload_matches_oracle(z3, numels, D, A, n_stage, mode):
+@pytest.mark.parametrize("numels,D,A,n_stage,chunks", [([300, 77, 1000], 4, 8, 2, 1), ([123457], 8, 128, 1, 4),
+                                                       ([4097, 33], 32, 128, 3, 2), ([999], 5, 1, 2, 3),
+                                                       ([2 ** 20 + 5], 8, 128, 2, 4), ([2 ** 20 + 5], 8, 128, 3, 7)])
+def test_host_adamw_offload_matches_oracle(z3, numels, D, A, n_stage, chunks, mode):
     from fsdp_sharded_mixed_flat_b200.offload import HostAdamWOffload
     plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
     N, N_pad, S = ref.N, ref.N_pad, ref.S
@@ -70,7 +70,8 @@ def test_host_adamw_offload_matches_oracle(z3, numels, D, A, n_stage, mode):
     p = p_dev.cpu().pin_memory()
     m, v = torch.zeros(N_pad).pin_memory(), torch.zeros(N_pad).pin_memory()
     w = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
-    off = HostAdamWOffload(plan, p, m, v, w, "cuda", n_stage=n_stage, reduce_dtype=mode, n_threads=4)
+    off = HostAdamWOffload(plan, p, m, v, w, "cuda", n_stage=n_stage, reduce_dtype=mode, n_threads=4, chunks=chunks)
+    assert sum(n for _, _, n in off.units) == N_pad and len(off.units) >= D
     hp_, hm, hv, hw = p.numpy().copy(), np.zeros(N_pad, np.float32), np.zeros(N_pad, np.float32), \
         np.zeros(N_pad, np.uint16)
     for t in range(1, 5):
