@@ -97,6 +97,8 @@ def parse_args(argv=None):
     ap.add_argument("--refill", choices=list(ARRIVALS), default=DEFAULT_ARRIVAL,
                     help="70B shard: how each layer's contributions arrive in the transient buffer: "
                          + "; ".join(f"{k}: {v}" for k, v in ARRIVALS.items()))
+    ap.add_argument("--offload-chunks", type=int, default=4,
+                    help="--offload host: pipeline units per rank partition")
     ap.add_argument("--replicas", action="store_true",
                     help="N > 1: run N independent single-GPU replicas (each simulating its own D ranks) instead "
                          "of the real D-GPU step with D = N")
@@ -419,7 +421,7 @@ class BlockRunner:
     the replicated bf16 weights (the flat block), with no separate shard."""
 
     def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
-                 graph=False, offload=False, split=False, nodes=0):
+                 graph=False, offload=False, split=False, nodes=0, offload_chunks=4):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype
@@ -456,7 +458,7 @@ class BlockRunner:
                                                           (self.master, self.exp_avg, self.exp_avg_sq))
             if offload == "host":
                 self.offloaded = HostAdamWOffload(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
-                                                  reduce_dtype=reduce_dtype)
+                                                  reduce_dtype=reduce_dtype, chunks=offload_chunks)
             else:
                 self.offloaded = OffloadedState(plan, self.master, self.exp_avg, self.exp_avg_sq, self.work, dev,
                                                 reduce_dtype=reduce_dtype)
@@ -1093,7 +1095,7 @@ def run_ours(args):
     else:
         R = BlockRunner(z3, synth, args.workload, args.D or synth.WORKLOADS[args.workload]["D"], mode, seed, dev,
                         stage=args.stage, unflatten_copy=args.unflatten_copy, graph=args.graph,
-                        offload=args.offload, split=args.split, nodes=args.nodes)
+                        offload=args.offload, split=args.split, nodes=args.nodes, offload_chunks=args.offload_chunks)
     stream = R.stream
 
     props = torch.cuda.get_device_properties(dev)
@@ -1194,6 +1196,7 @@ def run_ours(args):
         down = R.offloaded.bytes_down
         host_s = R.host_seconds[-args.steps * len(R.offloaded.units):]
         line["offload"] = {"placement": "AdamW on the host (the page's CPU-offload variant)",
+                           "pipeline_units": len(R.offloaded.units),
                            "pcie_bytes_per_param": (down + R.offloaded.bytes_up) / R.N_pad,
                            "pcie_gbs_down": down / step_s / 1e9, "pcie_gbs_up": R.offloaded.bytes_up / step_s / 1e9,
                            "host_adamw_ms_per_step": 1e3 * sum(host_s) / args.steps,

@@ -20,14 +20,16 @@
 // elements: one 16-byte load per rank, two per state array, all issued before
 // the arithmetic so that (D + 6) x 16 bytes per thread are in flight; the
 // ranks are folded in order 0..D-1 in chunks (8 ranks, 16 for the bf16 fold at
-// D = 32) to bound registers at large D.  The grid covers the whole range
+// D = 32) to bound registers at large D.  The bf16 fold at D = 16 takes 4
+// elements per thread instead (see k1_elems).  The grid covers the whole range
 // rather than looping over a resident grid: HBM bandwidth does not divide
 // evenly over the SMs, and a resident grid leaves the SMs that finish first
 // idle, while the block scheduler keeps every SM fed until the end.  Stores carry the streaming cache hint: every
 // byte is written exactly once.  Asking for three resident blocks per SM caps
 // the registers at 80 (65,536 / (3 x 256), rounded down to the allocation
 // granularity; left alone the compiler takes up to 128 at D >= 16); measured
-// on B200 this never loses and gains up to 12 % (bf16 reduce at D = 16).
+// on B200 this never loses and gains up to 12 % (bf16 reduce at D = 16, before
+// that instantiation moved to 4 elements per thread and 4 blocks per SM).
 //
 // Every arithmetic step is an explicitly rounded fp32 intrinsic, so nothing is
 // contracted into an FMA and the results are fixed by the stated operation
@@ -67,9 +69,26 @@ struct K1Args {
 };
 
 constexpr int kThreads = 256;
-constexpr int kMinBlocks = 3;               // >= 3 blocks per SM: at most 80 registers per thread
 constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
+
+// Elements per thread.  8 (16-byte loads of each contribution) everywhere but
+// the bf16 fold of 16 ranks in one node without a fused gather, which takes 4
+// (8-byte loads of each contribution): with 8 its 16 contribution vectors and
+// the state did not fit 80 registers and spilled 28 bytes per thread; with 4 it
+// needs 64 registers and no spill, and runs 4 blocks per SM.  Measured on B200
+// for the 7B block: 7066 -> 7276 GB/s, the fp32 fold's 7278; the same change
+// did not help any other instantiation (D = 2, 4, 8 and the fp32 folds were
+// within 0.5 % or slower).
+__host__ __device__ constexpr int k1_elems(int mode, int dt, int rt, bool gather) {
+    return (mode == Z3_REDUCE_BF16 && dt == 16 && rt == 1 && !gather) ? 4 : 8;
+}
+
+// Blocks per SM each vector kernel asks for (the register cap follows from it):
+// 3 (80 registers) with 8 elements per thread, 4 (64 registers) with 4.
+__host__ __device__ constexpr int k1_min_blocks(int mode, int dt, int rt, bool gather) {
+    return k1_elems(mode, dt, rt, gather) == 4 ? 4 : 3;
+}
 
 // Fold ranks base..base+D-1 for the 8 elements starting at e into the fp32 or
 // packed-bf16 accumulators, left to right, in chunks of ranks (the chunk's
@@ -201,6 +220,57 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
     }
 }
 
+// The 4 elements starting at e (the k1_elems == 4 instantiations): one 8-byte
+// load per rank, one 16-byte load per state array; the same operations in the
+// same order as process8.
+template <int MODE, int DT>
+__device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc, int64_t e) {
+    const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
+    const float4 m0 = ld16(reinterpret_cast<const float4*>(a.m + e));
+    const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
+    float acc[4];
+    uint32_t accw[2];
+    constexpr int CH = 8;
+#pragma unroll
+    for (int d0 = 0; d0 < DT; d0 += CH) {
+        uint2 q[CH];
+#pragma unroll
+        for (int k = 0; k < CH; ++k) q[k] = ld16(reinterpret_cast<const uint2*>(a.c[d0 + k] + e));
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+            const bool first = d0 + k == 0;
+            if constexpr (MODE == Z3_REDUCE_FP32) {
+                const float x[4] = {lo_bf16(q[k].x), hi_bf16(q[k].x), lo_bf16(q[k].y), hi_bf16(q[k].y)};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = first ? x[i] : __fadd_rn(acc[i], x[i]);
+            } else {
+                accw[0] = first ? q[k].x : add_bf16x2(accw[0], q[k].x);
+                accw[1] = first ? q[k].y : add_bf16x2(accw[1], q[k].y);
+            }
+        }
+    }
+    float g[4];
+    if constexpr (MODE == Z3_REDUCE_FP32) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) g[k] = __fmul_rn(acc[k], a.inv_n);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            g[2 * k] = round_to_bf16(__fmul_rn(lo_bf16(accw[k]), a.inv_n));
+            g[2 * k + 1] = round_to_bf16(__fmul_rn(hi_bf16(accw[k]), a.inv_n));
+        }
+    }
+    float p[4] = {p0.x, p0.y, p0.z, p0.w};
+    float m[4] = {m0.x, m0.y, m0.z, m0.w};
+    float v[4] = {v0.x, v0.y, v0.z, v0.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) adamw_elem(sc, g[k], p[k], m[k], v[k]);
+    st16(reinterpret_cast<float4*>(a.p + e), make_float4(p[0], p[1], p[2], p[3]));
+    st16(reinterpret_cast<float4*>(a.m + e), make_float4(m[0], m[1], m[2], m[3]));
+    st16(reinterpret_cast<float4*>(a.v + e), make_float4(v[0], v[1], v[2], v[3]));
+    st16(reinterpret_cast<uint2*>(a.w + e), make_uint2(pack_bf16x2(p[0], p[1]), pack_bf16x2(p[2], p[3])));
+}
+
 // Vector kernel body: every pointer 16-byte aligned.  The grid covers the
 // whole range (kChunks 8-element chunks per thread, consecutive threads on
 // consecutive chunks), so the block scheduler hands blocks to whichever SM is
@@ -209,6 +279,15 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
 // go through the scalar path.
 template <int MODE, int DT, int RT, bool GATHER>
 __device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc) {
+    if constexpr (k1_elems(MODE, DT, RT, GATHER) == 4) {
+        const int64_t n4 = a.n >> 2;
+        const int64_t step4 = int64_t(gridDim.x) * kThreads;
+        for (int64_t q = int64_t(blockIdx.x) * kThreads + threadIdx.x; q < n4; q += step4)
+            process4<MODE, DT>(a, sc, q << 2);
+        const int64_t tail4 = (n4 << 2) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
+        if (tail4 < a.n) scalar_elem<MODE, RT, GATHER>(a, sc, tail4);
+        return;
+    }
     const int64_t n8 = a.n >> 3;
     const int64_t span = int64_t(kThreads) * kChunks;
     const int64_t step = int64_t(gridDim.x) * span;
@@ -224,7 +303,8 @@ __device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc)
 }
 
 template <int MODE, int DT, int RT, bool GATHER, bool DEVS>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
+__global__ void __launch_bounds__(kThreads, (k1_min_blocks(MODE, DT, RT, GATHER)))
+    k_reduce_adamw_vec(const __grid_constant__ K1Args a) {
     if constexpr (DEVS) {
         const AdamScalars sc = load_scalars(a.s_dev);
         vec_body<MODE, DT, RT, GATHER>(a, sc);
@@ -397,8 +477,11 @@ int launch_k1(const z3_plan* p, int32_t rank, int32_t R, const uint16_t* const* 
     const KernelFn fn = pick_any(n_gathered > 0, dev_scalars != nullptr, vec, reduce_dtype, D, R);
     int64_t blocks;
     if (vec) {
-        const int64_t span = int64_t(kThreads) * kChunks;
-        blocks = ((n >> 3) + span - 1) / span;
+        // the template rank count of the picked kernel: D where D has its own instantiation
+        const int dt = (R == 1 && (D == 1 || D == 2 || D == 4 || D == 8 || D == 16 || D == 32)) ? D : 0;
+        const int elems = k1_elems(reduce_dtype, dt, R == 1 ? 1 : 0, n_gathered > 0);
+        const int64_t span = int64_t(kThreads) * (elems == 4 ? 1 : kChunks);
+        blocks = ((n / elems) + span - 1) / span;
         if (blocks > kMaxBlocks) blocks = kMaxBlocks;
     } else {
         int per_sm = 0;
