@@ -97,7 +97,7 @@ def parse_args(argv=None):
     ap.add_argument("--refill", choices=list(ARRIVALS), default=DEFAULT_ARRIVAL,
                     help="70B shard: how each layer's contributions arrive in the transient buffer: "
                          + "; ".join(f"{k}: {v}" for k, v in ARRIVALS.items()))
-    ap.add_argument("--offload-chunks", type=int, default=4,
+    ap.add_argument("--offload-chunks", type=int, default=1,
                     help="--offload host: pipeline units per rank partition")
     ap.add_argument("--replicas", action="store_true",
                     help="N > 1: run N independent single-GPU replicas (each simulating its own D ranks) instead "
@@ -421,7 +421,7 @@ class BlockRunner:
     the replicated bf16 weights (the flat block), with no separate shard."""
 
     def __init__(self, z3, synth, workload, D, reduce_dtype, seed, dev, stage=3, unflatten_copy=False,
-                 graph=False, offload=False, split=False, nodes=0, offload_chunks=4):
+                 graph=False, offload=False, split=False, nodes=0, offload_chunks=1):
         import torch
         w = synth.WORKLOADS[workload]
         self.z3, self.synth, self.w, self.D, self.mode = z3, synth, w, D, reduce_dtype

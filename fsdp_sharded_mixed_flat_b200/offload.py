@@ -122,7 +122,7 @@ class HostAdamWOffload:
 
     def __init__(self, plan: "z3.Plan", master: torch.Tensor, exp_avg: torch.Tensor, exp_avg_sq: torch.Tensor,
                  work_bf16: torch.Tensor, device, n_stage: int = 3, reduce_dtype: int = z3.Z3_REDUCE_FP32,
-                 n_threads: int = 0, chunks: int = 4):
+                 n_threads: int = 0, chunks: int = 1):
         S, N_pad = plan.S, plan.N_pad
         for name, t in (("master", master), ("exp_avg", exp_avg), ("exp_avg_sq", exp_avg_sq)):
             if t.device.type != "cpu" or t.dtype != torch.float32 or t.numel() < N_pad or not t.is_contiguous():
