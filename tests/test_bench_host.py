@@ -151,3 +151,33 @@ def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode):
         assert np.array_equal(rv.view(np.uint32), vv[sl].view(np.uint32)), f"exp_avg_sq rank {r}"
         assert np.array_equal(rw, ww[sl]), f"work rank {r}"
         assert np.array_equal(rflat, ww), f"gathered block rank {r}"
+
+
+def test_config_sweep_records_a_failing_entry_and_goes_on(monkeypatch):
+    """The sweep after the headline: an entry that raises (e.g. memory taken by
+    another process) is recorded as an error and the other entries still run."""
+    import torch
+
+    class FakeRunner:
+        k1_bytes_per_launch, units_per_step, S, L = 42.0e9, 1.0e9, 1.0e8, 80
+        refill_bytes, arrival_desc = 1.0e9, "memset"
+
+        def __init__(self, z3, synth, workload, D, *a, **k):
+            if workload == "llama7b_d32":
+                raise RuntimeError("CUDA out of memory (simulated)")
+
+        def step_in_place(self, *a):
+            pass
+
+    monkeypatch.setattr(bench, "BlockRunner", FakeRunner)
+    monkeypatch.setattr(bench, "ShardRunner", FakeRunner)
+    monkeypatch.setattr(bench, "time_runner", lambda R, steps, warmup, dev, step=None: (0.01 * steps, 0.006))
+    monkeypatch.setattr(bench, "prefetch_sweep", lambda *a, **k: {"sweep_ms_prefetch": 1.0})
+    z3 = type("Z3", (), {"Z3_REDUCE_FP32": 0, "Z3_REDUCE_BF16": 1})
+    out = bench.config_sweep(z3, None, torch.device("cpu"), 10, 3, 6650.0, "memset")
+    assert out["config2_llama7b_d32"] == {"error": "RuntimeError: CUDA out of memory (simulated)"}
+    assert out["config1_llama7b_d8"]["fp32"]["k1_gbs"] == pytest.approx(7000.0)
+    assert out["config1_llama7b_d8"]["fp32"]["meets_80pct_of_nominal"] is True
+    assert set(out) == {k for k, _, _ in bench.SWEEP_BLOCKS} | {"config4_llama70b_shard",
+                                                                 "next2_prefetch_llama7b_L32_d8"}
+    assert out["config4_llama70b_shard"]["streamed"]["arrival"] == "memset"
