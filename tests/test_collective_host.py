@@ -175,3 +175,57 @@ def test_collective_hybrid_step_equals_the_two_level_oracle(R, D, mode):
         assert np.array_equal(rv.view(np.uint32), v[sl].view(np.uint32)), f"exp_avg_sq rank {g}"
         assert np.array_equal(rw, w[sl]), f"work rank {g}"
         assert np.array_equal(rflat, w), f"gathered block rank {g}"
+
+
+def _failing_worker(rank, world, port, how, out):
+    import time
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=3))
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
+    plan = z3.zero3_plan(SHAPES, world, 8)
+    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    grad = synth.contribution(N, N_pad, seed=SEED, step=1, rank=rank, sigma=1e-3)
+    master = synth.master_weights(N, N_pad, seed=SEED)[rank * S:(rank + 1) * S].clone()
+    m, v = torch.zeros(S), torch.zeros(S)
+    work, flat = torch.zeros(S, dtype=torch.bfloat16), torch.zeros(N_pad, dtype=torch.bfloat16)
+    step = CollectiveZero3Step(plan, grad, master, m, v, work, flat, kernels=OracleKernels())
+    step.step(z3.adamw(step=1))                      # a whole step with every rank
+    if rank == world - 1:                            # the failing rank leaves between steps
+        if how == "stall":
+            time.sleep(15)
+        out[rank] = "left"
+        os._exit(0)                                  # no goodbye to the group
+    t0 = time.monotonic()
+    try:
+        step.step(z3.adamw(step=2))
+        out[rank] = ("no error", time.monotonic() - t0)
+    except Exception as e:                           # noqa: BLE001
+        out[rank] = (type(e).__name__, time.monotonic() - t0)
+    os._exit(0)
+
+
+@pytest.mark.parametrize("how", ["exit", "stall"])
+def test_collective_step_surfaces_a_lost_rank_as_an_error(how):
+    """A rank that exits, or stops answering, between steps: the surviving ranks'
+    next step ends with an error from the process group (a closed connection, or
+    its 3-second timeout), well before the lost rank would have come back; no rank
+    waits forever.  (Failure detection made on the host, with gloo ranks.)"""
+    world = 3
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as manager:
+        out = manager.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_failing_worker, args=(r, world, port, how, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0, "a rank did not end"
+        res = dict(out)
+    assert res[world - 1] == "left"
+    for r in range(world - 1):
+        kind, secs = res[r]
+        assert kind != "no error", f"rank {r} finished a step without the lost rank"
+        assert secs < 14, f"rank {r} took {secs:.1f} s to notice"
