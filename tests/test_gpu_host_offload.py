@@ -109,3 +109,36 @@ def test_reduce_scatter_composed_with_host_adamw_equals_the_fused_kernel(z3):
         for a, b in ((fp, hp_), (fm, hm), (fv, hv)):
             assert torch.equal(a.cpu().view(torch.int32), b.view(torch.int32))
         assert torch.equal(fw.cpu().view(torch.int16), hw.view(torch.int16))
+
+
+@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
+def test_host_adamw_offload_full_size_llama7b_block(z3, mode):
+    """The benchmark's offload step at full size: the LLaMA-7B block at D = 8, the
+    state in pinned host memory, AdamW on the host, 2 steps; every element of the
+    state and of the bf16 weights compared with the oracle on a sample that
+    includes every partition boundary."""
+    from fsdp_sharded_mixed_flat_b200.offload import HostAdamWOffload
+    w = synth.WORKLOADS["llama7b_d8"]
+    plan, ref = checked_plan(z3, [s for _, s in w["tensors"]], 8, synth.ALIGN)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
+    p = synth.master_weights(N, N_pad, seed=17, device="cuda").cpu().pin_memory()
+    m, v = torch.zeros(N_pad).pin_memory(), torch.zeros(N_pad).pin_memory()
+    wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
+    rng = np.random.default_rng(17)
+    idx = np.unique(np.concatenate([rng.choice(N_pad, 100_000, replace=False)] +
+                                   [np.arange(max(0, r * S - 16), min(N_pad, r * S + 16)) for r in range(9)]))
+    ti = torch.from_numpy(idx).cuda()
+    hp_, hm, hv = p.numpy()[idx].copy(), np.zeros(idx.size, np.float32), np.zeros(idx.size, np.float32)
+    hw = np.zeros(idx.size, np.uint16)
+    off = HostAdamWOffload(plan, p, m, v, wk, "cuda", reduce_dtype=mode)
+    for t in (1, 2):
+        c = synth.contributions(8, N, N_pad, seed=17, step=t, sigma=w["sigma"], device="cuda")
+        off.step(c, z3.adamw(**hp_for(t)))
+        oracle.reduce_adamw([synth.bf16_bits(x[ti]) for x in c], idx.size, 0, hp_, hm, hv, hw, oracle_hp(t),
+                            layout=oracle.LAYOUT_OWNED, reduce_dtype=mode)
+        del c
+    torch.cuda.synchronize()
+    assert_f32_parity(p.numpy()[idx], hp_, "master")
+    assert_f32_parity(m.numpy()[idx], hm, "exp_avg")
+    assert_f32_parity(v.numpy()[idx], hv, "exp_avg_sq")
+    assert_bf16_parity(synth.bf16_bits(wk[ti]), hw, "work_bf16")
