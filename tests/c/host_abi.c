@@ -151,6 +151,47 @@ static void check_scalars(void)
     CHECK(zero3_step_scalars(&hp, s) == Z3_EINVAL);
 }
 
+/* The host optimiser of the CPU-offload step, from C: one step from m = v = 0
+ * moves every weight by about lr against the sign of its gradient (the
+ * update is lr * g / (|g| + eps * sqrt(1 - beta2)) once the bias corrections
+ * cancel), a zero pad with a zero gradient stays exactly zero, the bf16
+ * weights are the masters rounded to bf16, and the work is the same on 1 and
+ * on 7 threads. */
+static void check_host_adamw(void)
+{
+    enum { n = 5000, pad = 96 };
+    static float g[n], p1[n], m1[n], v1[n], p7[n], m7[n], v7[n];
+    static uint16_t w1[n], w7[n];
+    for (int i = 0; i < n; ++i) {
+        g[i] = i >= n - pad ? 0.0f : (i % 2 ? 1e-3f : -2e-3f) * (float)(1 + i % 7);
+        p1[i] = p7[i] = i >= n - pad ? 0.0f : 0.01f * (float)((i % 11) - 5);
+        m1[i] = m7[i] = v1[i] = v7[i] = 0.0f;
+    }
+    const z3_adamw hp = {3e-4, 0.9, 0.95, 1e-8, 0.0, 1};
+    CHECK(zero3_host_adamw(n, g, Z3_REDUCE_FP32, p1, m1, v1, w1, &hp, 1) == Z3_OK);
+    CHECK(zero3_host_adamw(n, g, Z3_REDUCE_FP32, p7, m7, v7, w7, &hp, 7) == Z3_OK);
+    CHECK(memcmp(p1, p7, sizeof p1) == 0 && memcmp(m1, m7, sizeof m1) == 0 && memcmp(v1, v7, sizeof v1) == 0);
+    CHECK(memcmp(w1, w7, sizeof w1) == 0);
+    for (int i = 0; i < n; ++i) {
+        const float p0 = i >= n - pad ? 0.0f : 0.01f * (float)((i % 11) - 5);
+        if (i >= n - pad) {
+            CHECK(p1[i] == 0.0f && m1[i] == 0.0f && v1[i] == 0.0f && w1[i] == 0);
+            continue;
+        }
+        const double step = (double)p1[i] - (double)p0;
+        CHECK(fabs(fabs(step) - 3e-4) < 3e-6);          /* |update| = lr, within eps's share */
+        CHECK((step < 0) == (g[i] > 0));                 /* against the gradient */
+        uint32_t u;
+        memcpy(&u, &p1[i], sizeof u);
+        const uint32_t lsb = (u >> 16) & 1u;
+        CHECK(w1[i] == (uint16_t)((u + 0x7FFFu + lsb) >> 16));   /* nearest-even bf16 */
+    }
+    CHECK(zero3_host_adamw(-1, g, Z3_REDUCE_FP32, p1, m1, v1, w1, &hp, 1) == Z3_EINVAL);
+    CHECK(zero3_host_adamw(n, g, 7, p1, m1, v1, w1, &hp, 1) == Z3_EINVAL);
+    CHECK(zero3_host_adamw(n, g, Z3_REDUCE_FP32, p1, p1, v1, w1, &hp, 1) == Z3_EINVAL);   /* master = exp_avg */
+    CHECK(zero3_host_adamw(0, NULL, Z3_REDUCE_FP32, NULL, NULL, NULL, NULL, &hp, 0) == Z3_OK);
+}
+
 static void check_errors(void)
 {
     z3_tensor_spec t = spec2(3, 5);
@@ -184,6 +225,7 @@ int main(void)
     check_ledger();
     check_scalars();
     check_errors();
+    check_host_adamw();
     if (failures) {
         fprintf(stderr, "%d check(s) failed\n", failures);
         return 1;
