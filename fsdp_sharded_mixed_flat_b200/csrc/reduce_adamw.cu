@@ -73,21 +73,24 @@ constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
 
 // Elements per thread.  8 (16-byte loads of each contribution) everywhere but
-// the bf16 fold of 16 ranks in one node without a fused gather, which takes 4
-// (8-byte loads of each contribution): with 8 its 16 contribution vectors and
-// the state did not fit 80 registers and spilled 28 bytes per thread; with 4 it
-// needs 64 registers and no spill, and runs 4 blocks per SM.  Measured on B200
-// for the 7B block: 7066 -> 7276 GB/s, the fp32 fold's 7278; the same change
-// did not help any other instantiation (D = 2, 4, 8 and the fp32 folds were
-// within 0.5 % or slower).
+// in three bf16 folds without a fused gather, which take 4 (8-byte loads of
+// each contribution): 16 ranks in one node, and 4 or 8 nodes of 8 ranks
+// (HYBRID_SHARD).  With 8 elements their contribution vectors and the state
+// did not fit 80 registers and spilled 24-36 bytes per thread; with 4 nothing
+// spills.  Measured on B200 for the 7B block: one node of 16 ranks 7066 ->
+// 7276 GB/s (at 4 blocks per SM; 3 blocks lost there), 4 nodes of 8 7107 ->
+// 7204, 8 nodes of 8 7076 -> 7234 (at 3 blocks per SM).  The same change did
+// not help any other instantiation (the fp32 folds, D = 2, 4, 8 and 2 nodes of
+// 8 were within 0.5 % or slower).
 __host__ __device__ constexpr int k1_elems(int mode, int dt, int rt, bool gather) {
-    return (mode == Z3_REDUCE_BF16 && dt == 16 && rt == 1 && !gather) ? 4 : 8;
+    return (mode == Z3_REDUCE_BF16 && !gather &&
+            ((dt == 16 && rt == 1) || (dt == 8 && (rt == 4 || rt == 8)))) ? 4 : 8;
 }
 
 // Blocks per SM each vector kernel asks for (the register cap follows from it):
-// 3 (80 registers) with 8 elements per thread, 4 (64 registers) with 4.
+// 3 (80 registers), or 4 (64 registers) for the one-node 16-rank bf16 fold.
 __host__ __device__ constexpr int k1_min_blocks(int mode, int dt, int rt, bool gather) {
-    return k1_elems(mode, dt, rt, gather) == 4 ? 4 : 3;
+    return (k1_elems(mode, dt, rt, gather) == 4 && rt == 1) ? 4 : 3;
 }
 
 // Fold ranks base..base+D-1 for the 8 elements starting at e into the fp32 or
@@ -220,24 +223,19 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
     }
 }
 
-// The 4 elements starting at e (the k1_elems == 4 instantiations): one 8-byte
-// load per rank, one 16-byte load per state array; the same operations in the
-// same order as process8.
+// Fold ranks base..base+DT-1 for the 4 elements starting at e into fp32 or
+// packed-bf16 accumulators, left to right, in chunks of 8 ranks (the chunk's
+// 8-byte loads all issued before its folds).
 template <int MODE, int DT>
-__device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc, int64_t e) {
-    const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
-    const float4 m0 = ld16(reinterpret_cast<const float4*>(a.m + e));
-    const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
-    float acc[4];
-    uint32_t accw[2];
-    constexpr int CH = 8;
+__device__ __forceinline__ void fold_ranks4(const K1Args& a, int base, int64_t e, float (&acc)[4],
+                                            uint32_t (&accw)[2]) {
 #pragma unroll
-    for (int d0 = 0; d0 < DT; d0 += CH) {
-        uint2 q[CH];
+    for (int d0 = 0; d0 < DT; d0 += 8) {
+        uint2 q[8];
 #pragma unroll
-        for (int k = 0; k < CH; ++k) q[k] = ld16(reinterpret_cast<const uint2*>(a.c[d0 + k] + e));
+        for (int k = 0; k < 8; ++k) q[k] = ld16(reinterpret_cast<const uint2*>(a.c[base + d0 + k] + e));
 #pragma unroll
-        for (int k = 0; k < CH; ++k) {
+        for (int k = 0; k < 8; ++k) {
             const bool first = d0 + k == 0;
             if constexpr (MODE == Z3_REDUCE_FP32) {
                 const float x[4] = {lo_bf16(q[k].x), hi_bf16(q[k].x), lo_bf16(q[k].y), hi_bf16(q[k].y)};
@@ -246,6 +244,36 @@ __device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc,
             } else {
                 accw[0] = first ? q[k].x : add_bf16x2(accw[0], q[k].x);
                 accw[1] = first ? q[k].y : add_bf16x2(accw[1], q[k].y);
+            }
+        }
+    }
+}
+
+// The 4 elements starting at e (the k1_elems == 4 instantiations): one 8-byte
+// load per rank, one 16-byte load per state array; the same operations in the
+// same order as process8 (RT = 1: the rank fold; otherwise each node's rank
+// fold, then the node sums in node order).
+template <int MODE, int DT, int RT>
+__device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc, int64_t e) {
+    const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
+    const float4 m0 = ld16(reinterpret_cast<const float4*>(a.m + e));
+    const float4 v0 = ld16(reinterpret_cast<const float4*>(a.v + e));
+    float acc[4];
+    uint32_t accw[2];
+    if constexpr (RT == 1) {
+        fold_ranks4<MODE, DT>(a, 0, e, acc, accw);
+    } else {
+        float node[4];
+        uint32_t nodew[2];
+#pragma unroll
+        for (int k = 0; k < RT; ++k) {
+            fold_ranks4<MODE, DT>(a, k * DT, e, node, nodew);
+            if constexpr (MODE == Z3_REDUCE_FP32) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = k == 0 ? node[i] : __fadd_rn(acc[i], node[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) accw[i] = k == 0 ? nodew[i] : add_bf16x2(accw[i], nodew[i]);
             }
         }
     }
@@ -283,7 +311,7 @@ __device__ __forceinline__ void vec_body(const K1Args& a, const AdamScalars& sc)
         const int64_t n4 = a.n >> 2;
         const int64_t step4 = int64_t(gridDim.x) * kThreads;
         for (int64_t q = int64_t(blockIdx.x) * kThreads + threadIdx.x; q < n4; q += step4)
-            process4<MODE, DT>(a, sc, q << 2);
+            process4<MODE, DT, RT>(a, sc, q << 2);
         const int64_t tail4 = (n4 << 2) + int64_t(blockIdx.x) * kThreads + threadIdx.x;
         if (tail4 < a.n) scalar_elem<MODE, RT, GATHER>(a, sc, tail4);
         return;
@@ -477,9 +505,17 @@ int launch_k1(const z3_plan* p, int32_t rank, int32_t R, const uint16_t* const* 
     const KernelFn fn = pick_any(n_gathered > 0, dev_scalars != nullptr, vec, reduce_dtype, D, R);
     int64_t blocks;
     if (vec) {
-        // the template rank count of the picked kernel: D where D has its own instantiation
-        const int dt = (R == 1 && (D == 1 || D == 2 || D == 4 || D == 8 || D == 16 || D == 32)) ? D : 0;
-        const int elems = k1_elems(reduce_dtype, dt, R == 1 ? 1 : 0, n_gathered > 0);
+        // the template rank and node counts of the picked kernel (pick_vec, pick_hybrid_vec)
+        int dt = 0, rt = 1;
+        if (R == 1) {
+            if (D == 1 || D == 2 || D == 4 || D == 8 || D == 16 || D == 32) dt = D;
+        } else if (D == 8 && (R == 2 || R == 4 || R == 8)) {
+            dt = 8;
+            rt = R;
+        } else {
+            rt = 0;
+        }
+        const int elems = k1_elems(reduce_dtype, dt, rt, n_gathered > 0);
         const int64_t span = int64_t(kThreads) * (elems == 4 ? 1 : kChunks);
         blocks = ((n / elems) + span - 1) / span;
         if (blocks > kMaxBlocks) blocks = kMaxBlocks;
