@@ -65,7 +65,7 @@ SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 # How the 70B shard's per-layer contributions arrive in a transient buffer (the
 # reduce-scatter's delivery, simulated on one GPU).
 # Measured on B200 for the 80-layer step: copy 93.8 ms, fill 85.9 ms (torch's
-# bf16 fill kernel writes at about 3.9 TB/s), memset 70.0 ms (the driver's
+# bf16 fill kernel writes at about 3.9 TB/s), memset 70.0 ms (the CUDA driver's
 # memset writes at about 6.8 TB/s).
 ARRIVALS = {
     "copy": "device-to-device copy from a pool on the copy stream (read + write)",

@@ -152,7 +152,7 @@ def build_mutant(src: str, out_dir: str, tag: int) -> str:
 
 
 def killed_by(so_path: str):
-    """The index of the first pin that fails against this build, or None."""
+    """The index of the first pin that fails against the given library, or None."""
     previous = oracle.use_library(so_path)
     try:
         for k, pin in enumerate(PINS):
