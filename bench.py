@@ -904,12 +904,45 @@ def config_sweep(z3, synth, dev, steps: int, warmup: int, hbm_peak: float, refil
             torch.cuda.synchronize(dev)
             torch.cuda.empty_cache()
 
+    def sweep_step_variant(key, label, make, reps):
+        """A whole block step of one of the NEXT rows: owned params/s and ms per step,
+        with the fused kernel's own time and rate (or, offloaded, the PCIe figures)."""
+        R = make()
+        secs, k1 = time_runner(R, reps, 2, dev)
+        entry = {"what": label, "step_ms": 1e3 * secs / reps, "step_owned_params_per_s": R.units_per_step * reps / secs,
+                 "kernel": R.k1_name, "kernel_ms": 1e3 * k1, "kernel_gbs": R.k1_bytes_per_launch / k1 / 1e9,
+                 "steps": reps}
+        if getattr(R, "offload", None) == "host":
+            host_s = R.host_seconds[-reps * len(R.offloaded.units):]
+            entry.update(pcie_bytes_per_param=(R.offloaded.bytes_down + R.offloaded.bytes_up) / R.N_pad,
+                         host_adamw_ms_per_step=1e3 * sum(host_s) / reps)
+        elif getattr(R, "offload", None) == "state":
+            entry.update(pcie_bytes_per_param=24)
+        out.setdefault(key, {})[label] = entry
+        del R
+
     for key, workload, D in SWEEP_BLOCKS:
         guarded(key, lambda key=key, workload=workload, D=D: sweep_block(key, workload, D))
     guarded("config4_llama70b_shard", sweep_shard)
     guarded("next2_prefetch_llama7b_L32_d8",
             lambda: out.__setitem__("next2_prefetch_llama7b_L32_d8",
                                     prefetch_sweep(z3, synth, dev, max(2, steps // 5))))
+    # NEXT-3: the ZeRO-1/2 step (all-gather fused into the kernel), HYBRID_SHARD over 4 nodes of 8
+    guarded("next3_zero12_llama7b_d8", lambda: sweep_step_variant(
+        "next3_zero12_llama7b_d8", "fp32", lambda: BlockRunner(z3, synth, "llama7b_d8", 8, 0, 2000, dev, stage=2),
+        steps))
+    for name, mode in (("fp32", 0), ("bf16", 1)):
+        guarded("next3_hybrid_llama7b_4x8", lambda name=name, mode=mode: sweep_step_variant(
+            "next3_hybrid_llama7b_4x8", name, lambda: BlockRunner(z3, synth, "llama7b_hybrid", 8, mode, 2000, dev),
+            steps))
+    # NEXT-4: the CPU-offload step, AdamW on the host (the page's design) and the state
+    # streamed through the GPU
+    for place in ("host", "state"):
+        guarded("next4_offload_llama7b_d8", lambda place=place: sweep_step_variant(
+            "next4_offload_llama7b_d8", place,
+            lambda: BlockRunner(z3, synth, "llama7b_d8", 8, 0, 2000, dev, offload=place), 3))
+    # config 3's bf16-vs-fp32 drift over 100 steps (reported, not asserted)
+    guarded("config3_drift", lambda: out.__setitem__("config3_drift", drift_measure(z3, synth, dev, 100, 1 << 24)))
     return out
 
 
@@ -1258,21 +1291,15 @@ def run_ours(args):
     return 0
 
 
-def run_drift(args):
+def drift_measure(z3, synth, dev, steps: int, n: int) -> dict:
     """The policy sweep's drift: the same heavy-tailed contributions (Student-t nu=3,
     1% exact zeros, fresh every step) drive two copies of the same master, one
-    reduced in bf16 and one in fp32, for --steps steps at each D; report how far
-    the bf16 path's master and bf16 weights end up from the fp32 path's."""
+    reduced in bf16 and one in fp32, for `steps` steps at each D; how far the bf16
+    path's master and bf16 weights end up from the fp32 path's.  The pages give no
+    value for it: it is reported, not asserted."""
     import torch
-
-    import synth
-    from fsdp_sharded_mixed_flat_b200 import build
-    build.build()
-    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
-    dev = torch.device("cuda", 0)
     w = synth.WORKLOADS["llama7b_policy"]
-    n = args.drift_elements
-    out = {"drift": {}, "steps": args.steps, "elements": n,
+    out = {"drift": {}, "steps": steps, "elements": n,
            "workload": "first %d elements of the LLaMA-7B block, Student-t nu=3 x %g, %g%% exact zeros, "
                        "fresh contributions every step" % (n, w["sigma"], 100 * w["zero_frac"])}
     for D in w["Ds"]:
@@ -1281,7 +1308,7 @@ def run_drift(args):
         p0 = synth.master_weights(n, N_pad, seed=11, device=dev)
         state = {mode: [p0.clone(), torch.zeros_like(p0), torch.zeros_like(p0),
                         torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)] for mode in (0, 1)}
-        for t in range(1, args.steps + 1):
+        for t in range(1, steps + 1):
             c = synth.contributions(D, n, N_pad, seed=11, step=t, sigma=w["sigma"], dist=w["dist"],
                                     zero_frac=w["zero_frac"], device=dev)
             for mode in (0, 1):
@@ -1299,7 +1326,17 @@ def run_drift(args):
             "diff_rms_over_update_rms": (diff.pow(2).mean().sqrt() / upd_rms).item(),
             "bf16_weights_differing": (wf != wb).double().mean().item(),
         }
-    print(json.dumps(out), flush=True)
+    return out
+
+
+def run_drift(args):
+    import torch
+
+    import synth
+    from fsdp_sharded_mixed_flat_b200 import build
+    build.build()
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    print(json.dumps(drift_measure(z3, synth, torch.device("cuda", 0), args.steps, args.drift_elements)), flush=True)
     return 0
 
 

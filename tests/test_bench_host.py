@@ -160,11 +160,13 @@ def test_config_sweep_records_a_failing_entry_and_goes_on(monkeypatch):
 
     class FakeRunner:
         k1_bytes_per_launch, units_per_step, S, L = 42.0e9, 1.0e9, 1.0e8, 80
-        refill_bytes, arrival_desc = 1.0e9, "memset"
+        refill_bytes, arrival_desc, k1_name = 1.0e9, "memset", "fake"
 
         def __init__(self, z3, synth, workload, D, *a, **k):
             if workload == "llama7b_d32":
                 raise RuntimeError("CUDA out of memory (simulated)")
+            self.offload, self.N_pad, self.host_seconds = k.get("offload"), 1.0e9, [0.01] * 64
+            self.offloaded = type("O", (), {"units": [0] * 8, "bytes_down": 4.0e9, "bytes_up": 2.0e9})
 
         def step_in_place(self, *a):
             pass
@@ -173,11 +175,17 @@ def test_config_sweep_records_a_failing_entry_and_goes_on(monkeypatch):
     monkeypatch.setattr(bench, "ShardRunner", FakeRunner)
     monkeypatch.setattr(bench, "time_runner", lambda R, steps, warmup, dev, step=None: (0.01 * steps, 0.006))
     monkeypatch.setattr(bench, "prefetch_sweep", lambda *a, **k: {"sweep_ms_prefetch": 1.0})
+    monkeypatch.setattr(bench, "drift_measure", lambda *a, **k: {"drift": {}})
     z3 = type("Z3", (), {"Z3_REDUCE_FP32": 0, "Z3_REDUCE_BF16": 1})
     out = bench.config_sweep(z3, None, torch.device("cpu"), 10, 3, 6650.0, "memset")
     assert out["config2_llama7b_d32"] == {"error": "RuntimeError: CUDA out of memory (simulated)"}
     assert out["config1_llama7b_d8"]["fp32"]["k1_gbs"] == pytest.approx(7000.0)
     assert out["config1_llama7b_d8"]["fp32"]["meets_80pct_of_nominal"] is True
-    assert set(out) == {k for k, _, _ in bench.SWEEP_BLOCKS} | {"config4_llama70b_shard",
-                                                                 "next2_prefetch_llama7b_L32_d8"}
+    assert set(out) == {k for k, _, _ in bench.SWEEP_BLOCKS} | {
+        "config4_llama70b_shard", "next2_prefetch_llama7b_L32_d8", "next3_zero12_llama7b_d8",
+        "next3_hybrid_llama7b_4x8", "next4_offload_llama7b_d8", "config3_drift"}
     assert out["config4_llama70b_shard"]["streamed"]["arrival"] == "memset"
+    assert set(out["next3_hybrid_llama7b_4x8"]) == {"fp32", "bf16"}
+    assert set(out["next4_offload_llama7b_d8"]) == {"host", "state"}
+    assert out["next4_offload_llama7b_d8"]["state"]["pcie_bytes_per_param"] == 24
+    assert out["next4_offload_llama7b_d8"]["host"]["pcie_bytes_per_param"] == pytest.approx(6.0)
