@@ -740,6 +740,40 @@ class ShardRunner:
         self.host_out.copy_(self.work[:self.S], non_blocking=True)
 
 
+def mix_ceilings(dev, reps: int = 10) -> dict:
+    """HBM bandwidth of plain torch kernels on this GPU, per read/write mix, best
+    of `reps` launches timed with CUDA events on 1 GiB fp32 buffers (well beyond
+    L2): write-only (fill), read-only (sum), copy (1 read : 1 write) and add (2
+    reads : 1 write, the fused kernel's mix at D = 8).  Library kernels, so a
+    kernel of ours can sit a little above them; they place its rate against the
+    mix it moves."""
+    import torch
+    n = 1 << 28
+    a = torch.rand(n, device=dev)
+    b = torch.rand(n, device=dev)
+    c = torch.empty(n, device=dev)
+    ops = {"write_only_fill": (lambda: c.fill_(1.0), 4 * n),
+           "read_only_sum": (lambda: a.sum(), 4 * n),
+           "copy_1r_1w": (lambda: c.copy_(a), 8 * n),
+           "add_2r_1w": (lambda: torch.add(a, b, out=c), 12 * n)}
+    out = {}
+    for name, (fn, nbytes) in ops.items():
+        fn()
+        best = None
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            t = e0.elapsed_time(e1) / 1e3
+            best = t if best is None else min(best, t)
+        out[name] = nbytes / best / 1e9
+    del a, b, c
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_runner(R, steps: int, warmup: int, dev, clocks=None, barrier=None, step=None):
     """W untimed warm-up steps, then `steps` steps timed with CUDA events on the
     runner's stream between synchronisations (and barriers, with several ranks);
@@ -1256,6 +1290,11 @@ def run_ours(args):
                                    "(30 B of host memory traffic per param), so the hbm roofline fields describe "
                                    "the GPU's reduce kernels only"}
         line["roofline"]["traffic"] = None
+    if world == 1 and not args.no_sweep:
+        # the K1 of the default workload reads 2 bytes per byte written (28 : 14 at D = 8)
+        ceil = mix_ceilings(dev)
+        line["roofline"]["mix_ceilings_torch_gbs"] = ceil
+        line["roofline"]["frac_of_2r1w_ceiling"] = k1_gbs / ceil["add_2r_1w"]
     run_D, run_nodes, run_split = R.D, getattr(R, "nodes", 1), getattr(R, "split", False)
     if world == 1 and not args.no_sweep and args.workload == "llama7b_d8" and args.stage == 3 and \
             not (args.graph or args.offload or args.unflatten_copy):
