@@ -16,7 +16,8 @@
  *     device.  The caller owns and allocates every device buffer; the library
  *     never allocates, frees or keeps device memory.  Host arrays of device
  *     pointers (contrib, gathered, shards, tensor_out) are read during the
- *     call only.
+ *     call only.  zero3_host_adamw alone works on host memory, synchronously;
+ *     it keeps a pool of host threads for later calls.
  *   - Device work is enqueued on `cuda_stream` (a cudaStream_t; NULL means the
  *     legacy default stream) and the call returns without synchronising.
  *     Argument and alignment errors are reported synchronously, before any
