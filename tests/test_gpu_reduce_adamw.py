@@ -531,3 +531,18 @@ def test_random_hyperparameters_match_oracle(z3):
         assert_f32_parity(f32_host(m), hm, "exp_avg " + what)
         assert_f32_parity(f32_host(v), hv, "exp_avg_sq " + what)
         assert_bf16_parity(synth.bf16_bits(w), hw, "work_bf16 " + what)
+
+
+@pytest.mark.parametrize("extra", [1, 2, 3, 4, 5, 7])
+def test_four_element_folds_every_tail_residue(z3, extra):
+    """The instantiations that take 4 elements per thread (the bf16 fold of 16 ranks,
+    and of 4 and 8 nodes of 8 ranks): single-rank launches whose partition length
+    leaves every remainder mod 4 and mod 8 for the scalar tail, owned and full
+    layouts, against the oracle."""
+    S = 1000 + extra                       # partition length; A = 1 keeps it unpadded
+    run_small(z3, [16 * S], 16, 1, 0, z3.Z3_CONTRIB_FULL, 1, steps=2)       # rank 0: aligned at offset 0
+    run_small(z3, [16 * S], 16, 1, 11, z3.Z3_CONTRIB_OWNED, 1, steps=2)
+    from test_gpu_hybrid import run_small as run_hybrid
+    for R in (4, 8):
+        run_hybrid(z3, [8 * S], R, 8, 1, 0, z3.Z3_CONTRIB_FULL, 1, steps=2)
+        run_hybrid(z3, [8 * S], R, 8, 1, 5, z3.Z3_CONTRIB_OWNED, 1, steps=2)
