@@ -860,6 +860,7 @@ def prefetch_sweep(z3, synth, dev, steps: int, L: int = 32, D: int = 8) -> dict:
            "ledger_transient_bytes_2_blocks": z3.zero3_transient_bytes(N_pad, 2),
            "sweep_ms_prefetch": 1e3 * t_pre, "sweep_ms_serial": 1e3 * t_ser,
            "gather_ms_serial": 1e3 * g_ser, "k1_ms_serial": 1e3 * k_ser,
+           "sum_of_serial_kernels_ms": 1e3 * L * (g_ser + k_ser),
            "gather_gbs_serial": 4 * N_pad / g_ser / 1e9, "k1_gbs_serial": 42 * S / k_ser / 1e9,
            "gather_ms_overlapped": 1e3 * g_pre, "k1_ms_overlapped": 1e3 * k_pre,
            "hidden_fraction_of_gather": (t_ser - t_pre) / (L * g_ser),
