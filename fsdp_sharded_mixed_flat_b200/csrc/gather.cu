@@ -253,16 +253,20 @@ extern "C" Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const
     // ---- the per-tensor copies, straight from the shards
     if (tensor_out != nullptr) {
         std::vector<Seg> segs;
-        for (int32_t i = 0; i < nt; ++i) {
-            if (!tensor_out[i] || p->numel[i] == 0) continue;
-            const int64_t b = p->offset[i], e = b + p->numel[i];
-            for (int64_t r = b / S; r < D && r * S < e; ++r) {
-                const int64_t lo = std::max(b, r * S), hi = std::min(e, (r + 1) * S);
-                if (hi <= lo) continue;
-                Seg g{shards[r] + (lo - r * S), tensor_out[i] + (lo - b), hi - lo, 0, 0};
-                g.src_aligned = z3::aligned(g.src, 16) && z3::aligned(g.dst, 16) ? 1 : 0;
-                segs.push_back(g);
+        try {  // the segment list is host memory: an allocation failure is a status, not an exception
+            for (int32_t i = 0; i < nt; ++i) {
+                if (!tensor_out[i] || p->numel[i] == 0) continue;
+                const int64_t b = p->offset[i], e = b + p->numel[i];
+                for (int64_t r = b / S; r < D && r * S < e; ++r) {
+                    const int64_t lo = std::max(b, r * S), hi = std::min(e, (r + 1) * S);
+                    if (hi <= lo) continue;
+                    Seg g{shards[r] + (lo - r * S), tensor_out[i] + (lo - b), hi - lo, 0, 0};
+                    g.src_aligned = z3::aligned(g.src, 16) && z3::aligned(g.dst, 16) ? 1 : 0;
+                    segs.push_back(g);
+                }
             }
+        } catch (...) {
+            return Z3_ENOMEM;
         }
         for (size_t first = 0; first < segs.size(); first += kSegMax) {
             SegArgs a;

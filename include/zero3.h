@@ -51,7 +51,7 @@ enum {
     Z3_OK = 0,
     Z3_EINVAL = -1,    /* a NULL pointer, a value out of range, overlapping buffers */
     Z3_EALIGN = -2,    /* a pointer not aligned to its element size */
-    Z3_ENOMEM = -3,    /* host allocation failed (the plan object) */
+    Z3_ENOMEM = -3,    /* host allocation failed (a plan, a segment list, a host thread) */
     Z3_ECUDA = -4,     /* a CUDA runtime call or kernel launch failed */
     Z3_EOVERFLOW = -5  /* a size does not fit in int64_t */
 };
@@ -407,7 +407,8 @@ Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t
  * pointers; otherwise a scalar kernel gives the same bytes.
  * Errors: Z3_EINVAL (both outputs NULL, a NULL shard, an output overlapping a
  * shard other than in the in-place position above, outputs overlapping each
- * other), Z3_EALIGN, Z3_ECUDA. */
+ * other), Z3_EALIGN, Z3_ENOMEM (the host list of per-tensor segments could not
+ * be allocated), Z3_ECUDA. */
 Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
                               uint16_t* const* tensor_out, void* cuda_stream);
 
