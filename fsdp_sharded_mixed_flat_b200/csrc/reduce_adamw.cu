@@ -72,25 +72,30 @@ constexpr int kThreads = 256;
 constexpr int kChunks = 1;                  // 8-element chunks per thread
 constexpr int64_t kMaxBlocks = 1 << 30;     // grid.x cap; beyond it the kernel loops
 
-// Elements per thread.  8 (16-byte loads of each contribution) everywhere but
-// in three bf16 folds without a fused gather, which take 4 (8-byte loads of
-// each contribution): 16 ranks in one node, and 4 or 8 nodes of 8 ranks
-// (HYBRID_SHARD).  With 8 elements their contribution vectors and the state
-// did not fit 80 registers and spilled 24-36 bytes per thread; with 4 nothing
-// spills.  Measured on B200 for the 7B block: one node of 16 ranks 7066 ->
-// 7276 GB/s (at 4 blocks per SM; 3 blocks lost there), 4 nodes of 8 7107 ->
-// 7204, 8 nodes of 8 7076 -> 7234 (at 3 blocks per SM).  The same change did
-// not help any other instantiation (the fp32 folds, D = 2, 4, 8 and 2 nodes of
-// 8 were within 0.5 % or slower).
+// Elements per thread.  8 (16-byte loads of each contribution) by default; 4
+// (8-byte loads of each contribution) where it measured faster on B200 (7B
+// block), i.e. where 8 elements' contribution vectors and state did not fit the
+// register cap and spilled, without a fused gather:
+//   - the bf16 fold of one node of 16 ranks: 7066 -> 7276 GB/s;
+//   - the bf16 folds of 4 and 8 nodes of 8 ranks: 7107 -> 7204, 7076 -> 7234;
+//   - the generic one-node fp32 fold (rank counts without their own
+//     instantiation): D = 3 / 6 / 12 / 24: 6088 / 6263 / 6658 / 6746 ->
+//     6712 / 6978 / 6868 / 6997;
+//   - the generic HYBRID_SHARD fold (any node count and D), both dtypes:
+//     3 x 5 fp32 5764 -> 5976, 2 x 3 bf16 5346 -> 5889.
+// It did not help elsewhere: the fp32 folds of D = 2, 4, 8, 16, 32, 2 nodes of 8
+// and the generic one-node bf16 fold were within 0.5 % or slower with 4.
 __host__ __device__ constexpr int k1_elems(int mode, int dt, int rt, bool gather) {
-    return (mode == Z3_REDUCE_BF16 && !gather &&
-            ((dt == 16 && rt == 1) || (dt == 8 && (rt == 4 || rt == 8)))) ? 4 : 8;
+    return gather ? 8
+         : dt == 0 ? ((rt == 0 || mode == Z3_REDUCE_FP32) ? 4 : 8)
+         : (mode == Z3_REDUCE_BF16 && ((dt == 16 && rt == 1) || (dt == 8 && (rt == 4 || rt == 8)))) ? 4 : 8;
 }
 
 // Blocks per SM each vector kernel asks for (the register cap follows from it):
-// 3 (80 registers), or 4 (64 registers) for the one-node 16-rank bf16 fold.
+// 3 (80 registers), or 4 (64 registers) for the 4-element folds other than the
+// specialised HYBRID_SHARD ones (where 3 measured better).
 __host__ __device__ constexpr int k1_min_blocks(int mode, int dt, int rt, bool gather) {
-    return (k1_elems(mode, dt, rt, gather) == 4 && rt == 1) ? 4 : 3;
+    return (k1_elems(mode, dt, rt, gather) == 4 && (rt == 1 || rt == 0)) ? 4 : 3;
 }
 
 // Fold ranks base..base+D-1 for the 8 elements starting at e into the fp32 or
@@ -223,19 +228,23 @@ __device__ __forceinline__ void process8(const K1Args& a, const AdamScalars& sc,
     }
 }
 
-// Fold ranks base..base+DT-1 for the 4 elements starting at e into fp32 or
+// Fold ranks base..base+D-1 for the 4 elements starting at e into fp32 or
 // packed-bf16 accumulators, left to right, in chunks of 8 ranks (the chunk's
-// 8-byte loads all issued before its folds).
+// 8-byte loads all issued before its folds).  DT = 0: D from the arguments.
 template <int MODE, int DT>
 __device__ __forceinline__ void fold_ranks4(const K1Args& a, int base, int64_t e, float (&acc)[4],
                                             uint32_t (&accw)[2]) {
+    const int D = DT > 0 ? DT : a.D;
 #pragma unroll
-    for (int d0 = 0; d0 < DT; d0 += 8) {
+    for (int d0 = 0; d0 < (DT > 0 ? DT : Z3_D_MAX); d0 += 8) {
+        if (DT == 0 && d0 >= D) break;
         uint2 q[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) q[k] = ld16(reinterpret_cast<const uint2*>(a.c[base + d0 + k] + e));
+        for (int k = 0; k < 8; ++k)
+            if (d0 + k < D) q[k] = ld16(reinterpret_cast<const uint2*>(a.c[base + d0 + k] + e));
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
+            if (d0 + k >= D) continue;
             const bool first = d0 + k == 0;
             if constexpr (MODE == Z3_REDUCE_FP32) {
                 const float x[4] = {lo_bf16(q[k].x), hi_bf16(q[k].x), lo_bf16(q[k].y), hi_bf16(q[k].y)};
@@ -252,7 +261,8 @@ __device__ __forceinline__ void fold_ranks4(const K1Args& a, int base, int64_t e
 // The 4 elements starting at e (the k1_elems == 4 instantiations): one 8-byte
 // load per rank, one 16-byte load per state array; the same operations in the
 // same order as process8 (RT = 1: the rank fold; otherwise each node's rank
-// fold, then the node sums in node order).
+// fold, then the node sums in node order; DT = 0 / RT = 0: counts from the
+// arguments).
 template <int MODE, int DT, int RT>
 __device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc, int64_t e) {
     const float4 p0 = ld16(reinterpret_cast<const float4*>(a.p + e));
@@ -263,11 +273,13 @@ __device__ __forceinline__ void process4(const K1Args& a, const AdamScalars& sc,
     if constexpr (RT == 1) {
         fold_ranks4<MODE, DT>(a, 0, e, acc, accw);
     } else {
+        const int D = DT > 0 ? DT : a.D;
+        const int R = RT > 0 ? RT : a.R;
         float node[4];
         uint32_t nodew[2];
-#pragma unroll
-        for (int k = 0; k < RT; ++k) {
-            fold_ranks4<MODE, DT>(a, k * DT, e, node, nodew);
+#pragma unroll(RT > 0 ? RT : 1)
+        for (int k = 0; k < R; ++k) {
+            fold_ranks4<MODE, DT>(a, k * D, e, node, nodew);
             if constexpr (MODE == Z3_REDUCE_FP32) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) acc[i] = k == 0 ? node[i] : __fadd_rn(acc[i], node[i]);
