@@ -14,7 +14,7 @@ import torch.distributed as dist
 
 import oracle
 import synth
-from parity_util import assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp
+from parity_util import assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for, oracle_hp
 
 pytestmark = pytest.mark.gpu
 
@@ -46,8 +46,8 @@ def nccl_one_rank():
 @pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
 def test_one_rank_nccl_group_matches_oracle(z3, nccl_one_rank, mode):
     from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
-    plan = z3.zero3_plan([(50000,), (77, 3), (4097,)], 1, 128)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(50000,), (77, 3), (4097,)], 1, 128)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     grad = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
     p = synth.master_weights(N, N_pad, seed=31, device="cuda")
     m, v = torch.zeros_like(p), torch.zeros_like(p)
@@ -73,8 +73,8 @@ def test_one_rank_nccl_hybrid_step_matches_oracle(z3, nccl_one_rank, mode):
     rank): node and replica groups, the node-sum and fold kernels, the gathers."""
     from fsdp_sharded_mixed_flat_b200.collective import CollectiveHybridStep, hybrid_groups
     node_group, replica_group = hybrid_groups(1, 1)
-    plan = z3.zero3_plan([(50000,), (77, 3), (4097,)], 1, 128)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(50000,), (77, 3), (4097,)], 1, 128)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     grad = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
     p = synth.master_weights(N, N_pad, seed=32, device="cuda")
     m, v = torch.zeros_like(p), torch.zeros_like(p)

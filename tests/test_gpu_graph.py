@@ -11,7 +11,8 @@ import torch
 
 import oracle
 import synth
-from parity_util import assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp, state_init
+from parity_util import (assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for, oracle_hp,
+                         state_init)
 
 pytestmark = pytest.mark.gpu
 
@@ -29,8 +30,8 @@ def z3():
 @pytest.mark.parametrize("numels,D,A,rank", [([300, 77, 1000], 4, 8, -1), ([123457], 8, 128, -1),
                                              ([13], 3, 1, -1), ([4097, 33], 32, 128, 5), ([999], 5, 1, 2)])
 def test_device_scalars_match_oracle(z3, numels, D, A, rank, mode):
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, 3)
     p = (p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]).clone()
@@ -60,8 +61,8 @@ def test_graphed_step_matches_oracle(z3, stage, mode):
     from fsdp_sharded_mixed_flat_b200.graph import GraphedStep
     w_ = synth.WORKLOADS["tiny_gpt"]
     shapes = [s for _, s in w_["tensors"]]
-    plan = z3.zero3_plan(shapes, w_["D"], synth.ALIGN)
-    N, N_pad, S, D = plan.N, plan.N_pad, plan.S, plan.D
+    plan, ref = checked_plan(z3, shapes, w_["D"], synth.ALIGN)
+    N, N_pad, S, D = ref.N, ref.N_pad, ref.S, plan.D
     p, m, v = state_init(N, N_pad, 0)
     work = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda") if stage == 3 else None
     flat = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")

@@ -16,8 +16,8 @@ import torch
 
 import oracle
 import synth
-from parity_util import (Guarded, assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp,
-                         state_init)
+from parity_util import (assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, Guarded, hp_for,
+                         oracle_hp, state_init)
 
 pytestmark = pytest.mark.gpu
 
@@ -32,8 +32,8 @@ def z3():
 
 
 def run_small(z3, numels, R, D, A, rank, layout, mode, steps=6, seed=0, skew=0):
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     n = N_pad if rank < 0 else S
     p_full, _, _ = state_init(N, N_pad, seed)
     p0 = p_full if rank < 0 else p_full[rank * S:(rank + 1) * S]
@@ -125,8 +125,8 @@ def test_llama7b_block_4_nodes_of_8_bench_configuration(z3, mode, steps):
     launch, full layout; sampled elements against the oracle."""
     w = synth.WORKLOADS["llama7b_hybrid"]
     R, D = w["nodes"], w["D"]
-    plan = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [s for _, s in w["tensors"]], D, synth.ALIGN)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     p, m, v = state_init(N, N_pad, 0)
     wk = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
     rng = np.random.default_rng(1)

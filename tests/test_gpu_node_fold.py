@@ -11,7 +11,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import Guarded, f32_host, hp_for, oracle_hp, state_init
+from parity_util import checked_plan, f32_host, Guarded, hp_for, oracle_hp, state_init
 
 pytestmark = pytest.mark.gpu
 
@@ -36,8 +36,8 @@ def sum_bits(t: torch.Tensor) -> np.ndarray:
     ([4097, 33], 32, 128, 0), ([2 ** 12 + 5], 64, 8, 0), ([777], 1, 1, 0), ([5000, 77], 8, 8, 1),
 ])
 def test_node_sum_matches_oracle(z3, numels, D, A, skew, mode):
-    plan = z3.zero3_plan([(k,) for k in numels], D, A)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(k,) for k in numels], D, A)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     c = synth.contributions(D, N, N_pad, seed=D, step=1, sigma=1e-3, dist="student_t", zero_frac=0.02,
                             device="cuda")
     dt = torch.float32 if mode == 0 else torch.bfloat16
@@ -47,9 +47,9 @@ def test_node_sum_matches_oracle(z3, numels, D, A, skew, mode):
         gc = [Guarded(x.numel(), torch.bfloat16, skew, fill=x) for x in src]
         out = Guarded(n, dt, skew)
         z3.zero3_node_sum(plan, rank, [g.t for g in gc], out.t, contrib_layout=layout, reduce_dtype=mode)
-        ref = oracle.node_sum([synth.bf16_bits(x) for x in src], S, rank, layout, mode)
+        want = oracle.node_sum([synth.bf16_bits(x) for x in src], S, rank, layout, mode)
         torch.cuda.synchronize()
-        assert np.array_equal(sum_bits(out.t), ref.view(np.uint32)), (numels, D, rank, layout, mode)
+        assert np.array_equal(sum_bits(out.t), want.view(np.uint32)), (numels, D, rank, layout, mode)
         assert out.guards_intact() and all(g.guards_intact() for g in gc)
 
 
@@ -57,8 +57,8 @@ def test_node_sum_matches_oracle(z3, numels, D, A, skew, mode):
 @pytest.mark.parametrize("R,skew", [(1, 0), (2, 0), (3, 0), (4, 0), (8, 0), (16, 0), (4, 1)])
 def test_fold_adamw_matches_oracle(z3, R, skew, mode):
     D = 4
-    plan = z3.zero3_plan([(20000,), (4097,)], D, 8)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(20000,), (4097,)], D, 8)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     dt = torch.float32 if mode == 0 else torch.bfloat16
     for rank in (-1, 2):
         n = N_pad if rank < 0 else S
@@ -96,8 +96,8 @@ def test_node_sums_then_fold_equal_the_fused_hybrid_kernel_at_full_size(z3, mode
     four node sums, then the fold, against the fused HYBRID_SHARD kernel."""
     w = synth.WORKLOADS["llama7b_hybrid"]
     R, D = w["nodes"], w["D"]
-    plan = z3.zero3_plan([s for _, s in w["tensors"]], D, synth.ALIGN)
-    N, N_pad = plan.N, plan.N_pad
+    plan, ref = checked_plan(z3, [s for _, s in w["tensors"]], D, synth.ALIGN)
+    N, N_pad = ref.N, ref.N_pad
     dt = torch.float32 if mode == 0 else torch.bfloat16
     a = list(state_init(N, N_pad, 3)) + [torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")]
     b = [x.clone() for x in a]

@@ -14,7 +14,7 @@ import torch.distributed as dist
 
 import oracle
 import synth
-from parity_util import assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp
+from parity_util import assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for, oracle_hp
 
 pytestmark = pytest.mark.gpu
 
@@ -43,8 +43,8 @@ def one_rank_group():
 @pytest.mark.parametrize("stage", [3, 2])
 def test_one_rank_group_matches_oracle(z3, one_rank_group, stage):
     from fsdp_sharded_mixed_flat_b200.peer import PeerGroup, PeerZero3Step
-    plan = z3.zero3_plan([(5000,), (77, 3)], 1, 128)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(5000,), (77, 3)], 1, 128)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     grad = torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda")
     p = synth.master_weights(N, N_pad, seed=12, device="cuda")
     m, v = torch.zeros_like(p), torch.zeros_like(p)
@@ -100,8 +100,8 @@ def test_four_ranks_emulated_by_threads_match_oracle(z3, stage, mode):
 
     from fsdp_sharded_mixed_flat_b200.peer import PeerZero3Step
     D = 4
-    plan = z3.zero3_plan([(5000,), (77, 3), (4097,)], D, 128)
-    N, N_pad, S = plan.N, plan.N_pad, plan.S
+    plan, ref = checked_plan(z3, [(5000,), (77, 3), (4097,)], D, 128)
+    N, N_pad, S = ref.N, ref.N_pad, ref.S
     p_full = synth.master_weights(N, N_pad, seed=21, device="cuda")
     grads = [torch.zeros(N_pad, dtype=torch.bfloat16, device="cuda") for _ in range(D)]
     state = [[p_full[r * S:(r + 1) * S].clone(), torch.zeros(S, device="cuda"), torch.zeros(S, device="cuda"),

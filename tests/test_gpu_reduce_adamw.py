@@ -536,13 +536,20 @@ def test_random_hyperparameters_match_oracle(z3):
 @pytest.mark.parametrize("extra", [1, 2, 3, 4, 5, 7])
 def test_four_element_folds_every_tail_residue(z3, extra):
     """The instantiations that take 4 elements per thread (the bf16 fold of 16 ranks,
-    and of 4 and 8 nodes of 8 ranks): single-rank launches whose partition length
+    and of 4 and 8 nodes of 8 ranks; the generic one-node fp32 fold; the generic
+    HYBRID_SHARD fold in both dtypes): single-rank launches whose partition length
     leaves every remainder mod 4 and mod 8 for the scalar tail, owned and full
     layouts, against the oracle."""
     S = 1000 + extra                       # partition length; A = 1 keeps it unpadded
     run_small(z3, [16 * S], 16, 1, 0, z3.Z3_CONTRIB_FULL, 1, steps=2)       # rank 0: aligned at offset 0
     run_small(z3, [16 * S], 16, 1, 11, z3.Z3_CONTRIB_OWNED, 1, steps=2)
+    for D in (3, 12):                      # runtime rank count: one chunk of 8 ranks, and a partial second
+        run_small(z3, [D * S], D, 1, 0, z3.Z3_CONTRIB_FULL, 0, steps=2)
+        run_small(z3, [D * S], D, 1, D - 1, z3.Z3_CONTRIB_OWNED, 0, steps=2)
     from test_gpu_hybrid import run_small as run_hybrid
     for R in (4, 8):
         run_hybrid(z3, [8 * S], R, 8, 1, 0, z3.Z3_CONTRIB_FULL, 1, steps=2)
         run_hybrid(z3, [8 * S], R, 8, 1, 5, z3.Z3_CONTRIB_OWNED, 1, steps=2)
+    for R, D, mode in ((3, 5, 0), (2, 3, 1)):   # runtime node and rank counts
+        run_hybrid(z3, [D * S], R, D, 1, 0, z3.Z3_CONTRIB_FULL, mode, steps=2)
+        run_hybrid(z3, [D * S], R, D, 1, D - 1, z3.Z3_CONTRIB_OWNED, mode, steps=2)

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 import synth
-from parity_util import assert_bf16_parity, assert_f32_parity, f32_host, hp_for, oracle_hp
+from parity_util import assert_bf16_parity, assert_f32_parity, checked_plan, f32_host, hp_for, oracle_hp
 
 pytestmark = pytest.mark.gpu
 
@@ -32,9 +32,9 @@ def owned_contribs(D, S, n_real, seed, step, layer, sigma=1e-3):
 def test_streamed_layers_match_oracle(z3, mode, copy_in):
     from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
     L, D, rank = 7, 4, 2
-    plan = z3.zero3_plan([(300,), (77, 5), (1000,)], D, 8)
-    S = plan.S
-    n_real = max(0, min(S, plan.N - rank * S))
+    plan, ref = checked_plan(z3, [(300,), (77, 5), (1000,)], D, 8)
+    S = ref.S
+    n_real = max(0, min(S, ref.N - rank * S))
     master = synth.master_weights(L * S, L * S, seed=4, device="cuda")
     m, v = torch.zeros_like(master), torch.zeros_like(master)
     w = torch.zeros(L * S, dtype=torch.bfloat16, device="cuda")
@@ -62,9 +62,9 @@ def test_streamed_layers_with_a_fill_refill(z3):
     """The fill hook writes each block's contributions into the transient buffer."""
     from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
     L, D, rank = 5, 4, 1
-    plan = z3.zero3_plan([(4000,)], D, 8)
-    S = plan.S
-    n_real = max(0, min(S, plan.N - rank * S))
+    plan, ref = checked_plan(z3, [(4000,)], D, 8)
+    S = ref.S
+    n_real = max(0, min(S, ref.N - rank * S))
     master = synth.master_weights(L * S, L * S, seed=6, device="cuda")
     m, v = torch.zeros_like(master), torch.zeros_like(master)
     w = torch.zeros(L * S, dtype=torch.bfloat16, device="cuda")
@@ -93,8 +93,8 @@ def test_llama70b_rank_shard_80_layers_sampled(z3):
     from fsdp_sharded_mixed_flat_b200.stream import LayerStreamer
     w_ = synth.WORKLOADS["llama70b_layer"]
     L, D, rank = w_["layers"], w_["D"], 5
-    plan = z3.zero3_plan([s for _, s in w_["tensors"]], D, synth.ALIGN)
-    S = plan.S
+    plan, ref = checked_plan(z3, [s for _, s in w_["tensors"]], D, synth.ALIGN)
+    S = ref.S
     torch.cuda.empty_cache()              # blocks cached by earlier tests count as used
     free, _ = torch.cuda.mem_get_info()
     need = L * S * 14 + 4 * D * S * 2 + (1 << 30)
