@@ -14,7 +14,8 @@
 // The work is split over a pool of host threads that lives for the rest of the
 // process (created on first use, never torn down: its threads may still wait
 // for work when the process exits).  One call runs at a time; a second caller
-// waits for the first to finish.
+// waits for the first to finish.  A child made by fork() starts a pool of its
+// own on its first call.
 #include <algorithm>
 #include <atomic>
 #include <condition_variable>
@@ -24,6 +25,8 @@
 #include <mutex>
 #include <thread>
 #include <vector>
+
+#include <pthread.h>
 
 #include "adamw_scalars.h"
 #include "plan_impl.h"
@@ -77,11 +80,18 @@ void adamw_range(const AdamScalars s, const G* __restrict g, float* __restrict p
 
 // A pool of worker threads; run(n, f) calls f(0) .. f(n-1) spread over the
 // workers and the calling thread and returns when every call has returned.
+class Pool;
+Pool* g_pool = nullptr;  // never destroyed: workers may still wait at exit
+
 class Pool {
   public:
     static Pool& get() {
-        static Pool* pool = new Pool();  // never destroyed: workers may still wait at exit
-        return *pool;
+        static std::once_flag once;
+        std::call_once(once, [] {
+            g_pool = new Pool();
+            pthread_atfork(nullptr, nullptr, &Pool::after_fork_in_child);
+        });
+        return *g_pool;
     }
 
     void run(int workers, int n_tasks, const std::function<void(int)>& f) {
@@ -104,6 +114,12 @@ class Pool {
     }
 
   private:
+    // Only the forking thread lives on in the child: the workers are gone and
+    // a lock of the pool may have been held by one of them.  The child gets a
+    // fresh, empty pool; the old one is left as it is (its thread handles
+    // cannot be destroyed).
+    static void after_fork_in_child() { g_pool = new Pool(); }
+
     void grow(int n) {
         while (int(threads_.size()) < n) {
             const int id = int(threads_.size());

@@ -2,10 +2,14 @@
 against the oracle, on the CPU: bit-exact master / m / v after several steps
 and bf16 weights equal to the oracle's nearest-even cast, for fp32 and bf16
 gradients, ragged sizes, every thread count, random hyper-parameters, the zero
-pad and subnormal gradients; concurrent callers; argument errors."""
+pad and subnormal gradients; concurrent callers; a child forked while another
+thread's call runs; argument errors."""
 import ctypes as C
+import os
 import random
+import signal
 import threading
+import time
 
 import numpy as np
 import pytest
@@ -110,6 +114,59 @@ def test_concurrent_callers_share_the_pool():
         for t in range(1, 4):
             oracle.adamw(f32_of(g), hp_, hm, hv, oracle.hp(step=t))
         check(p, m, v, w, hp_, hm, hv, f"caller {k}")
+
+
+@pytest.mark.filterwarnings("ignore::DeprecationWarning")
+def test_forked_child_gets_a_pool_of_its_own():
+    """fork() while another thread's call holds the pool (its lock taken, a worker
+    busy): the child's own calls run on a fresh pool, since the parent's workers
+    and their locks do not exist in it, and give the oracle's bits."""
+    nb = 16_000_000                        # one call of the busy thread: tens of ms on two threads
+    big = host_state(nb, 7)
+    gbig = grad_of(nb, 7, 1, torch.float32)
+    n = 100_003                            # several tasks: the child's call goes through the pool
+    p, m, v, w = host_state(n, 8)
+    g = grad_of(n, 8, 1, torch.float32)
+    hp_, hm, hv = p.numpy().copy(), np.zeros(n, np.float32), np.zeros(n, np.float32)
+    oracle.adamw(f32_of(g), hp_, hm, hv, oracle.hp(step=1))
+    entering, stop = threading.Event(), threading.Event()
+
+    def busy():
+        t = 1
+        while not stop.is_set():
+            entering.set()
+            z3.zero3_host_adamw(gbig, *big, z3.adamw(step=t), n_threads=2)
+            t += 1
+
+    th = threading.Thread(target=busy)
+    th.start()
+    try:
+        entering.wait()
+        time.sleep(0.005)                  # the busy thread is now inside a call, back to back
+        pid = os.fork()
+        if pid == 0:                       # the child: one call on its own pool, then leave at once
+            code = 1
+            try:
+                z3.zero3_host_adamw(g, p, m, v, w, z3.adamw(step=1), n_threads=4)
+                ok = all(np.array_equal(a.numpy().view(np.uint32), b.view(np.uint32))
+                         for a, b in ((p, hp_), (m, hm), (v, hv)))
+                code = 0 if ok else 2
+            finally:
+                os._exit(code)
+        deadline = time.monotonic() + 60
+        while True:
+            done, status = os.waitpid(pid, os.WNOHANG)
+            if done:
+                break
+            if time.monotonic() > deadline:
+                os.kill(pid, signal.SIGKILL)
+                os.waitpid(pid, 0)
+                pytest.fail("the forked child did not finish its call")
+            time.sleep(0.05)
+        assert os.WIFEXITED(status) and os.WEXITSTATUS(status) == 0, f"child status {status}"
+    finally:
+        stop.set()
+        th.join()
 
 
 P16 = 0x10000  # fake host addresses: the argument checks run before any access
