@@ -10,12 +10,15 @@ memory ledger.
 
 One process per GPU (torchrun for N > 1).  With N = 1 the block's D ranks are
 simulated on the one GPU.  With N > 1 the block is sharded over the N GPUs
-(D = N, strong scaling: one block per step in all): every rank's gradient
-crosses an NCCL all-to-all (the reduce-scatter's data movement), the fused
-kernel updates the rank's own partition, and an NCCL all-gather assembles the
-block (--transport peer: the kernels read the peers' memory through CUDA IPC
-instead); --replicas runs N independent single-GPU replicas instead.  Rank 0
-prints one JSON line.
+(D = N, strong scaling: one block per step in all): the fused kernel on each
+rank reads its partition of every rank's gradient through CUDA IPC mappings
+with plain loads over NVLink (the reduce-scatter's data movement inside the
+optimiser kernel) and updates the rank's state and bf16 shard, and the gather
+kernel reads every rank's shard into the local block.  The line then also
+times the same step with an NCCL all-to-all and all-gather around the fused
+kernel (`baseline_nccl`; --transport nccl makes that form the headline).
+--replicas runs N independent single-GPU replicas instead.  Rank 0 prints one
+JSON line.
 
 Timing: W untimed warm-up steps, then K steps between a barrier plus
 cudaDeviceSynchronize on each side, timed with CUDA events on the launching
@@ -55,6 +58,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "owned params/s for fused reduce+AdamW+cast; achieved HBM GB/s vs ~8 TB/s"
 UNIT = "owned params/s"
+NVLINK_GBS = 770.0   # measured peer copy on this machine's B200s, per direction per GPU (900 GB/s nominal)
 # committed ncu summaries of the fused kernel, by workload (fp32 reduce), with its DRAM traffic
 PROFILE_K1 = {"llama7b_d8": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md"),
               "llama7b_hybrid": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_hybrid_llama7b_4x8.md")}
@@ -102,9 +106,13 @@ def parse_args(argv=None):
     ap.add_argument("--replicas", action="store_true",
                     help="N > 1: run N independent single-GPU replicas (each simulating its own D ranks) instead "
                          "of the real D-GPU step with D = N")
-    ap.add_argument("--transport", choices=["nccl", "peer"], default="nccl",
-                    help="N > 1: how the D-GPU step moves its bytes: NCCL all-to-all and all-gather around the "
-                         "fused kernel, or the kernels' own plain loads of the peers' memory (CUDA IPC)")
+    ap.add_argument("--transport", choices=["nccl", "peer"], default="peer",
+                    help="N > 1: how the D-GPU step moves its bytes: the kernels' own plain loads of the peers' "
+                         "memory through CUDA IPC mappings (the reduce-scatter fused into the optimiser kernel; "
+                         "the default), or NCCL all-to-all and all-gather around the fused kernel (the baseline)")
+    ap.add_argument("--no-nccl-baseline", action="store_true",
+                    help="N > 1 with --transport peer: skip the NCCL form of the same step, which the line "
+                         "otherwise times after the headline as `baseline_nccl`")
     ap.add_argument("--sweep-steps", type=int, default=10,
                     help="timed steps per configuration in the sweep of the target configurations")
     ap.add_argument("--no-sweep", action="store_true",
@@ -1014,7 +1022,8 @@ class CollectiveRunner:
     §5.1).  With transport "peer" the kernels read the peers' gradients and
     shards through CUDA IPC mappings with plain loads instead (peer.py)."""
 
-    def __init__(self, z3, synth, workload, world, rank, reduce_dtype, dev, kernels=None, transport="nccl"):
+    def __init__(self, z3, synth, workload, world, rank, reduce_dtype, dev, kernels=None, transport="nccl",
+                 peer_group=None):
         import torch
         from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
         w = synth.WORKLOADS[workload]
@@ -1032,8 +1041,9 @@ class CollectiveRunner:
         self.transport = transport
         if transport == "peer":
             from fsdp_sharded_mixed_flat_b200.peer import PeerGroup, PeerZero3Step
-            self.stepper = PeerZero3Step(PeerGroup(), plan, self.grad, self.master, self.exp_avg, self.exp_avg_sq,
-                                         self.work, self.flat, reduce_dtype=reduce_dtype, kernels=kernels or z3)
+            self.stepper = PeerZero3Step(peer_group or PeerGroup(), plan, self.grad, self.master, self.exp_avg,
+                                         self.exp_avg_sq, self.work, self.flat, reduce_dtype=reduce_dtype,
+                                         kernels=kernels or z3)
         else:
             self.stepper = CollectiveZero3Step(plan, self.grad, self.master, self.exp_avg, self.exp_avg_sq,
                                                self.work, self.flat, reduce_dtype=reduce_dtype, kernels=kernels or z3)
@@ -1050,26 +1060,23 @@ class CollectiveRunner:
         a = self.synth.ADAMW
         self.step_no += 1
         hp = self.z3.adamw(step=self.step_no, **a)
-        if self.transport == "peer":
-            m0 = self.clock.mark() if timed else None
-            self.stepper.step(hp)
-            if timed:
-                m1 = self.clock.mark()
-                self.marks.append((m0, m0, m1, m1))
-        else:
-            self.stepper.step(hp, mark=self.clock.mark if timed else None, marks=self.marks)
+        self.stepper.step(hp, mark=self.clock.mark if timed else None, marks=self.marks)
+
+    def phases(self) -> dict:
+        """Mean seconds of each phase of the timed steps: the all-to-all, the fused
+        kernel and the all-gather (NCCL); the two fences, the fused kernel reading
+        the peers' gradients and the gather kernel reading their shards (peer)."""
+        names = (("all_to_all", "reduce_adamw", "all_gather") if self.transport == "nccl" else
+                 ("fence_before", "reduce_adamw", "fence_between", "gather"))
+        return {n: statistics.mean(self.clock.seconds(m[k], m[k + 1]) for m in self.marks)
+                for k, n in enumerate(names)}
 
 
-def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, clocks=None, barrier=None):
-    """bench.py --gpus N, N > 1: the real D-GPU step with D = N, the block's
-    ranks on N GPUs (strong scaling: one block's N_pad owned params per step in
-    all, S = N_pad / N per rank).  Returns (the JSON line, the runner); only rank
-    0's line is printed."""
-    import torch
-    mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
-    R = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport=args.transport)
-    barrier = barrier or (lambda: torch.distributed.barrier())
-    for _ in range(args.warmup):
+def time_collective_steps(R, steps: int, warmup: int, world: int, dev, barrier, clocks=None):
+    """Warm-up, then `steps` timed steps bracketed by a barrier and a device
+    synchronisation on both sides; (seconds of this rank, job seconds = the max
+    over ranks, job units, clock record)."""
+    for _ in range(warmup):
         R.step()
     R.clock.sync()
     barrier()
@@ -1077,17 +1084,35 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
         clocks.start()
     t0 = R.clock.mark()
     R.marks.clear()
-    for _ in range(args.steps):
+    for _ in range(steps):
         R.step(timed=True)
     t1 = R.clock.mark()
     R.clock.sync()
     barrier()
     clk = clocks.stop() if clocks is not None else None
     secs = R.clock.seconds(t0, t1)
-    phase = [[R.clock.seconds(m[k], m[k + 1]) for m in R.marks] for k in range(3)]
-    a2a_s, k1_s, ag_s = (statistics.mean(x) for x in phase)
-    job_secs, job_units = aggregate(secs, float(R.units_per_step) * args.steps, world,
-                                    dev if dev.type == "cuda" else None)
+    job_secs, job_units = aggregate(secs, float(R.units_per_step) * steps, world, dev if dev.type == "cuda" else None)
+    return secs, job_secs, job_units, clk
+
+
+def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, clocks=None, barrier=None,
+                   peer_group=None):
+    """bench.py --gpus N, N > 1: the real D-GPU step with D = N, the block's
+    ranks on N GPUs (strong scaling: one block's N_pad owned params per step in
+    all, S = N_pad / N per rank).  The headline is the step as --transport sets
+    it: by default the peer form, whose fused kernel reads every rank's gradient
+    slice over the peer mappings (the reduce-scatter inside the optimiser
+    kernel) and whose gather kernel reads every rank's shard; with it, the NCCL
+    form of the same step is timed afterwards as `baseline_nccl`.  Returns (the
+    JSON line, the headline's runner); only rank 0's line is printed."""
+    import torch
+    mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
+    peer = args.transport == "peer"
+    R = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport=args.transport,
+                         peer_group=peer_group)
+    barrier = barrier or (lambda: torch.distributed.barrier())
+    secs, job_secs, job_units, clk = time_collective_steps(R, args.steps, args.warmup, world, dev, barrier, clocks)
+    ph = R.phases()
 
     # ---- end to end: this rank's gradient from pinned host memory, its new shard back
     pin = dev.type == "cuda"
@@ -1106,8 +1131,35 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
     e2e_secs, e2e_units = aggregate(R.clock.seconds(e0, e1), float(R.units_per_step) * e2e_steps, world,
                                     dev if dev.type == "cuda" else None)
     hbm_peak, peak_kind = measured_peaks()
+    k1_s = ph["reduce_adamw"]
     k1_gbs = R.k1_bytes_per_launch / k1_s / 1e9
     step_s = secs / args.steps
+    kname = f"k_reduce_adamw_vec<{'fp32' if mode == 0 else 'bf16'}, D={world}>"
+    if peer:
+        # the fused kernel pulls 2(D-1) bytes per owned element over NVLink and touches
+        # 28 B of its own HBM (its gradient slice, the state); the link is the bound
+        link_gbs = R.a2a_bytes / k1_s / 1e9
+        roofline = {"bound": "nvlink", "achieved": link_gbs, "peak": NVLINK_GBS, "unit": "GB/s",
+                    "frac": link_gbs / NVLINK_GBS,
+                    "peak_kind": "measured peer copy per direction per GPU on this pool (900 nominal)",
+                    "kernel": kname + " (full layout, peers' gradients through the IPC mappings)",
+                    "nvlink_bytes_in_per_launch": R.a2a_bytes, "hbm_algorithmic_gbs": k1_gbs, "traffic": None}
+        collective = {"fence_ms": 1e3 * (ph["fence_before"] + ph["fence_between"]),
+                      "reduce_adamw_ms": 1e3 * k1_s, "gather_ms": 1e3 * ph["gather"],
+                      "collective_share_of_step": (ph["fence_before"] + ph["fence_between"]) / max(step_s, 1e-12),
+                      "nvlink_bytes_in_per_rank": R.a2a_bytes + R.gather_bytes,
+                      "note": "the reduce-scatter's data movement runs inside the fused kernel and the "
+                              "all-gather's inside the gather kernel; the fences are a stream synchronisation "
+                              "and a group barrier"}
+    else:
+        roofline = {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
+                    "kernel": kname + " (owned layout)", "algorithmic_bytes_per_launch": R.k1_bytes_per_launch,
+                    "traffic": None}
+        collective = {"all_to_all_ms": 1e3 * ph["all_to_all"], "reduce_adamw_ms": 1e3 * k1_s,
+                      "all_gather_ms": 1e3 * ph["all_gather"],
+                      "collective_share_of_step": (ph["all_to_all"] + ph["all_gather"]) / max(step_s, 1e-12),
+                      "all_to_all_bytes_in_per_rank": R.a2a_bytes, "all_gather_bytes_in_per_rank": R.gather_bytes}
     line = {
         "metric": METRIC, "value": job_units / job_secs, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_secs / args.steps, "higher_is_better": True,
@@ -1118,21 +1170,25 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
                           f"AdamW lr=3e-4 b=(0.9,0.95) eps=1e-8 wd=0.1; transport {args.transport}"),
         "per_rank_owned_params_per_s": R.units_per_step / step_s,
         "comm_nranks": world,
-        "collective": {"all_to_all_ms": 1e3 * a2a_s, "reduce_adamw_ms": 1e3 * k1_s, "all_gather_ms": 1e3 * ag_s,
-                       "collective_share_of_step": (a2a_s + ag_s) / max(step_s, 1e-12),
-                       "all_to_all_bytes_in_per_rank": R.a2a_bytes, "all_gather_bytes_in_per_rank": R.gather_bytes,
-                       "note": "with transport peer the whole step is one phase (reduce_adamw_ms holds it)"},
+        "collective": collective,
         "kernels": {"reduce_adamw_ms": 1e3 * k1_s, "reduce_adamw_gbs": k1_gbs},
-        "roofline": {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
-                     "kernel": f"k_reduce_adamw_vec<{'fp32' if mode == 0 else 'bf16'}, D={world}> (owned layout)",
-                     "algorithmic_bytes_per_launch": R.k1_bytes_per_launch, "traffic": None},
+        "roofline": roofline,
         "clocks": clk,
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": 2 * R.N_pad,
                 "d2h_bytes_per_step": 2 * R.S, "steps": e2e_steps},
-        "gpu_launches": args.steps * (1 if args.transport == "nccl" else 2),
+        "gpu_launches": args.steps * (2 if peer else 1),
         "ledger_bytes_per_device": ledger(z3, R.N, R.N_pad, world, R.N_pad),
     }
+    if peer and not args.no_nccl_baseline:
+        B = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport="nccl")
+        _, b_secs, b_units, _ = time_collective_steps(B, args.steps, args.warmup, world, dev, barrier)
+        bph = B.phases()
+        line["baseline_nccl"] = {
+            "value": b_units / b_secs, "unit": UNIT, "ms_per_step": 1e3 * b_secs / args.steps,
+            "all_to_all_ms": 1e3 * bph["all_to_all"], "reduce_adamw_ms": 1e3 * bph["reduce_adamw"],
+            "all_gather_ms": 1e3 * bph["all_gather"],
+            "note": "the same step with NCCL all-to-all and all-gather around the fused kernel (owned layout)"}
+        del B
     return line, R
 
 

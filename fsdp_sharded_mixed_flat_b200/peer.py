@@ -98,16 +98,34 @@ class PeerZero3Step:
         else:
             self.flats = peers.share(flat)                  # D gathered blocks, rank order
 
-    def step(self, hp: "z3.AdamW") -> None:
+    def step(self, hp: "z3.AdamW", mark=None, marks: Optional[list] = None) -> None:
+        """One step.  With mark (a callable returning a time mark, e.g. a CUDA event
+        recorded on the current stream) and marks (a list), the marks around the
+        fences and kernels are appended to marks as one tuple: (before the first
+        fence, after it, after the fused kernel, after the second fence, after the
+        gather) at stage 3; (before the first fence, after it, after the fused
+        kernel, after the last fence) otherwise."""
         k = self.k
+        t = [mark()] if mark else None
         self.peers.fence(self.device)                       # every rank's gradient is complete
+        if t is not None:
+            t.append(mark())
         if self.stage == 3:
             k.zero3_reduce_adamw(self.plan, self.rank, self.grads, self.master, self.exp_avg, self.exp_avg_sq,
                                  self.work, hp, contrib_layout=k.Z3_CONTRIB_FULL, reduce_dtype=self.reduce_dtype)
+            if t is not None:
+                t.append(mark())
             self.peers.fence(self.device)                   # every rank's shard is updated
+            if t is not None:
+                t.append(mark())
             k.zero3_gather_block(self.plan, self.shards, self.flat, None)
         else:
             k.zero3_reduce_adamw_gather(self.plan, self.rank, self.grads, self.master, self.exp_avg,
                                         self.exp_avg_sq, self.work, self.flats, hp,
                                         contrib_layout=k.Z3_CONTRIB_FULL, reduce_dtype=self.reduce_dtype)
+            if t is not None:
+                t.append(mark())
             self.peers.fence(self.device)                   # every rank's pushes have landed
+        if t is not None:
+            t.append(mark())
+            marks.append(tuple(t))

@@ -81,7 +81,32 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"] == bench.contract_config(bench.parse_args([]), 1, 8, 1, 202_383_360)
 
 
-def _collective_worker(rank, world, port, mode, out):
+def _file_peer_group(tmpdir: str, rank: int):
+    """A PeerGroup whose "IPC" is a file every rank maps (host memory shared
+    between the gloo processes): share() moves the tensor's storage into a
+    fresh shared file mapping, so this rank's later writes are seen by every
+    rank that opened it."""
+    import itertools
+
+    import torch
+    from fsdp_sharded_mixed_flat_b200.peer import PeerGroup
+    count = itertools.count()
+
+    def share(t):
+        path = os.path.join(tmpdir, f"rank{rank}_{next(count)}")
+        mapped = torch.from_file(path, shared=True, size=t.numel(), dtype=t.dtype)
+        mapped.copy_(t)
+        t.set_(mapped)
+        return path, t.numel(), t.dtype
+
+    def open_(handle):
+        path, n, dtype = handle
+        return torch.from_file(path, shared=True, size=n, dtype=dtype)
+
+    return PeerGroup(share_fn=share, open_fn=open_, sync_fn=lambda device: None)
+
+
+def _collective_worker(rank, world, port, mode, transport, tmpdir, out):
     import numpy as np
     import torch
 
@@ -91,9 +116,11 @@ def _collective_worker(rank, world, port, mode, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     args = bench.parse_args(["--gpus", str(world), "--workload", "tiny_gpt", "--steps", "2", "--warmup", "1",
-                             "--e2e-steps", "1", "--reduce-dtype", "bf16" if mode else "fp32"])
+                             "--e2e-steps", "1", "--reduce-dtype", "bf16" if mode else "fp32",
+                             "--transport", transport])
+    group = _file_peer_group(tmpdir, rank) if transport == "peer" else None
     line, R = bench.run_collective(args, rank, world, torch.device("cpu"), z3, synth, kernels=OracleKernels(),
-                                   barrier=dist.barrier)
+                                   barrier=dist.barrier, peer_group=group)
     out[rank] = (line, R.master.numpy().copy(), R.exp_avg.numpy().copy(), R.exp_avg_sq.numpy().copy(),
                  R.work.view(torch.int16).numpy().view(np.uint16).copy(),
                  R.flat.view(torch.int16).numpy().view(np.uint16).copy(), R.step_no)
@@ -101,12 +128,15 @@ def _collective_worker(rank, world, port, mode, out):
     dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("transport", ["peer", "nccl"])
 @pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
-def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode):
+def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode, transport, tmp_path):
     """bench.py's N > 1 path (run_collective: the D-GPU step, warm-up, timed
     steps, max-over-ranks aggregation, the end-to-end leg, the JSON line) on two
-    gloo ranks; the oracle stands in for the kernels, the collectives move the
-    real bytes.  Every rank's state equals one oracle run over both ranks."""
+    gloo ranks, in both forms: the peer form over shared host mappings standing
+    in for the IPC mappings (then also the NCCL form as the baseline), and the
+    NCCL form with the collectives moving the real bytes.  The oracle stands in
+    for the kernels.  Every rank's state equals one oracle run over both ranks."""
     import numpy as np
 
     import oracle
@@ -116,7 +146,8 @@ def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode):
     with ctx.Manager() as m:
         out = m.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_collective_worker, args=(r, world, port, mode, out)) for r in range(world)]
+        procs = [ctx.Process(target=_collective_worker, args=(r, world, port, mode, transport, str(tmp_path), out))
+                 for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
@@ -131,6 +162,11 @@ def test_multi_gpu_path_end_to_end_on_two_gloo_ranks(mode):
     assert line["n_gpus"] == 2 and line["comm_nranks"] == 2 and line["scaling"] == "strong"
     assert line["config"]["D"] == 2 and line["value"] > 0 and line["e2e"]["value"] > 0
     assert line["metric"] == bench.METRIC and line["steps"] == 2 and line["warmup"] == 1
+    if transport == "peer":
+        assert line["roofline"]["bound"] == "nvlink" and line["gpu_launches"] == 2 * 2
+        assert line["baseline_nccl"]["value"] > 0 and line["collective"]["gather_ms"] >= 0
+    else:
+        assert line["roofline"]["bound"] == "hbm" and line["gpu_launches"] == 2 and "baseline_nccl" not in line
     w = synth.WORKLOADS["tiny_gpt"]
     numels = [synth.numel(s) for _, s in w["tensors"]]
     _, N, N_pad, S = oracle.plan(numels, world, synth.ALIGN)

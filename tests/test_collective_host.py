@@ -36,6 +36,7 @@ def _bits(t: torch.Tensor) -> np.ndarray:
 class OracleKernels:
     """The kernels' entry points, computed by the oracle on host tensors."""
     Z3_CONTRIB_OWNED = oracle.LAYOUT_OWNED
+    Z3_CONTRIB_FULL = oracle.LAYOUT_FULL
 
     @staticmethod
     def _hp(hp):
@@ -51,11 +52,15 @@ class OracleKernels:
 
     def zero3_reduce_adamw(self, plan, rank, contrib, master, exp_avg, exp_avg_sq, work, hp, contrib_layout,
                            reduce_dtype):
-        assert contrib_layout == oracle.LAYOUT_OWNED
+        assert contrib_layout in (oracle.LAYOUT_OWNED, oracle.LAYOUT_FULL)
         oracle.reduce_adamw([_bits(c) for c in contrib], plan.S, rank, master.numpy(), exp_avg.numpy(),
                             exp_avg_sq.numpy(), _bits(work),
                             oracle.hp(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, hp.step),
-                            layout=oracle.LAYOUT_OWNED, reduce_dtype=reduce_dtype)
+                            layout=contrib_layout, reduce_dtype=reduce_dtype)
+
+    def zero3_gather_block(self, plan, shards, flat, tensor_out=None):
+        assert tensor_out is None
+        _bits(flat)[:] = oracle.all_gather([_bits(x) for x in shards], plan.S)
 
 
 def _worker(rank, world, port, mode, steps, out):

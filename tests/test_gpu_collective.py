@@ -95,16 +95,24 @@ def test_one_rank_nccl_hybrid_step_matches_oracle(z3, nccl_one_rank, mode):
     assert np.array_equal(synth.bf16_bits(flat), hw)
 
 
-def test_bench_multi_gpu_path_on_a_one_rank_nccl_group(z3, nccl_one_rank):
+@pytest.mark.parametrize("transport", ["peer", "nccl"])
+def test_bench_multi_gpu_path_on_a_one_rank_nccl_group(z3, nccl_one_rank, transport):
     """bench.py's N > 1 path (run_collective) on a one-rank NCCL group with the
-    real kernels: CUDA-event timing of the all-to-all, the fused kernel and the
-    all-gather, the end-to-end leg, the JSON line; the rank's state after every
-    step equals the oracle's."""
+    real kernels, in both forms (the peer form, then the NCCL form as its
+    baseline; the NCCL form alone): CUDA-event timing of every phase, the
+    end-to-end leg, the JSON line; the rank's state after every step equals the
+    oracle's."""
     import bench
-    args = bench.parse_args(["--workload", "tiny_gpt", "--steps", "3", "--warmup", "2", "--e2e-steps", "2"])
+    args = bench.parse_args(["--workload", "tiny_gpt", "--steps", "3", "--warmup", "2", "--e2e-steps", "2",
+                             "--transport", transport])
     line, R = bench.run_collective(args, 0, 1, torch.device("cuda", 0), z3, synth)
     assert line["n_gpus"] == 1 and line["comm_nranks"] == 1 and line["value"] > 0 and line["e2e"]["value"] > 0
-    assert line["collective"]["reduce_adamw_ms"] > 0 and line["gpu_launches"] == 3
+    assert line["collective"]["reduce_adamw_ms"] > 0
+    if transport == "peer":
+        assert line["gpu_launches"] == 6 and line["collective"]["gather_ms"] > 0
+        assert line["baseline_nccl"]["value"] > 0 and line["baseline_nccl"]["reduce_adamw_ms"] > 0
+    else:
+        assert line["gpu_launches"] == 3 and "baseline_nccl" not in line
     w = synth.WORKLOADS["tiny_gpt"]
     numels = [synth.numel(s) for _, s in w["tensors"]]
     _, N, N_pad, S = oracle.plan(numels, 1, synth.ALIGN)
