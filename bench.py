@@ -62,7 +62,9 @@ NVLINK_GBS = 770.0   # measured peer copy on this machine's B200s, per direction pe
 # committed ncu summaries of the fused kernel, by workload (fp32 reduce), with its DRAM traffic
 PROFILE_K1 = {"llama7b_d8": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md"),
               "llama7b_hybrid": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_hybrid_llama7b_4x8.md")}
-K1_SOURCE = os.path.join(ROOT, "fsdp_sharded_mixed_flat_b200", "csrc", "reduce_adamw.cu")
+# the sources whose code makes up the fused kernel
+K1_SOURCES = [os.path.join(ROOT, "fsdp_sharded_mixed_flat_b200", "csrc", f)
+              for f in ("reduce_adamw.cu", "step_common.cuh", "adamw_scalars.h")]
 SLOW_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
 
 
@@ -170,19 +172,31 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def code_sha256(paths) -> str:
+    """sha256 of the code in the given C/CUDA sources, with // comments, trailing
+    blanks and empty lines removed: a profile taken on some code stays matched
+    to it through comment edits, and any change of code breaks the match."""
+    lines = []
+    for path in paths:
+        for line in open(path, encoding="utf-8"):
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()
+
+
 def profiled_traffic(workload: str):
     """DRAM bytes per launch from the committed ncu summary of the fused kernel on
-    this workload, if that summary was taken on the current kernel source; else None."""
+    this workload, if that summary was taken on the kernel's current code; else None."""
     path = PROFILE_K1.get(workload)
     if path is None or not os.path.exists(path):
         return None
     text = open(path).read()
-    sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    sha = re.search(r"code_sha256:\s*([0-9a-f]{64})", text)
     tb = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
     if not sha or not tb:
         return None
-    cur = hashlib.sha256(open(K1_SOURCE, "rb").read()).hexdigest()
-    return float(tb.group(1)) if sha.group(1) == cur else None
+    return float(tb.group(1)) if sha.group(1) == code_sha256(K1_SOURCES) else None
 
 
 # ------------------------------------------------------------------ clocks

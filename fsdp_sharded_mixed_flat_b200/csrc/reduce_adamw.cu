@@ -20,11 +20,15 @@
 // elements: one 16-byte load per rank, two per state array, all issued before
 // the arithmetic so that (D + 6) x 16 bytes per thread are in flight; the
 // ranks are folded in order 0..D-1 in chunks (8 ranks, 16 for the bf16 fold at
-// D = 32) to bound registers at large D.  The bf16 fold at D = 16 takes 4
-// elements per thread instead (see k1_elems).  The grid covers the whole range
-// rather than looping over a resident grid: HBM bandwidth does not divide
-// evenly over the SMs, and a resident grid leaves the SMs that finish first
-// idle, while the block scheduler keeps every SM fed until the end.  Stores carry the streaming cache hint: every
+// D = 32) to bound registers at large D.  The folds that did not fit the
+// register cap with 8 take 4 elements per thread instead (see k1_elems).
+// Loading each tile with 1-D bulk copies (cp.async.bulk) into shared memory
+// measured no faster on B200 (7044 against 7049 GB/s at D = 8, with more bytes
+// in flight): the read/write mix of HBM is the bound, not the issue of the
+// loads.  The grid covers the whole range rather than looping over a resident
+// grid: HBM bandwidth does not divide evenly over the SMs, and a resident grid
+// leaves the SMs that finish first idle, while the block scheduler keeps every
+// SM fed until the end.  Stores carry the streaming cache hint: every
 // byte is written exactly once.  Asking for three resident blocks per SM caps
 // the registers at 80 (65,536 / (3 x 256), rounded down to the allocation
 // granularity; left alone the compiler takes up to 128 at D >= 16); measured
@@ -38,7 +42,8 @@
 // Measured ceilings of HBM on the B200s used here, for a full-grid kernel with
 // two or more independent 16-byte vectors per thread: read-only 7.54 TB/s,
 // write-only 7.56 TB/s, copy 6.94 TB/s, two reads per write 7.16 TB/s.  This
-// pass reads 28 B and writes 14 B per element at D = 8, the two-to-one mix.
+// pass reads 28 B and writes 14 B per element at D = 8, the two-to-one mix;
+// the benchmark times torch's kernels of each mix beside it on the same GPU.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 

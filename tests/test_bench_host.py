@@ -225,3 +225,19 @@ def test_config_sweep_records_a_failing_entry_and_goes_on(monkeypatch):
     assert set(out["next4_offload_llama7b_d8"]) == {"host", "state"}
     assert out["next4_offload_llama7b_d8"]["state"]["pcie_bytes_per_param"] == 24
     assert out["next4_offload_llama7b_d8"]["host"]["pcie_bytes_per_param"] == pytest.approx(6.0)
+
+
+def test_committed_k1_profiles_match_the_kernel_code():
+    """The DRAM traffic the bench line reports comes from committed ncu profiles;
+    they must have been taken on the kernel's current code."""
+    for workload in ("llama7b_d8", "llama7b_hybrid"):
+        assert bench.profiled_traffic(workload) is not None, workload
+
+
+def test_code_hash_ignores_comments_only(tmp_path):
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text("// header\nint f(int x) {  // doubled\n    return 2 * x;\n}\n")
+    b.write_text("// another header\n\nint f(int x) {\n    return 2 * x;   \n}\n// end\n")
+    c.write_text("// header\nint f(int x) {\n    return 3 * x;\n}\n")
+    assert bench.code_sha256([a]) == bench.code_sha256([b])
+    assert bench.code_sha256([a]) != bench.code_sha256([c])
