@@ -1037,7 +1037,7 @@ class CollectiveRunner:
     shards through CUDA IPC mappings with plain loads instead (peer.py)."""
 
     def __init__(self, z3, synth, workload, world, rank, reduce_dtype, dev, kernels=None, transport="nccl",
-                 peer_group=None):
+                 peer_group=None, stage=3):
         import torch
         from fsdp_sharded_mixed_flat_b200.collective import CollectiveZero3Step
         w = synth.WORKLOADS[workload]
@@ -1052,12 +1052,12 @@ class CollectiveRunner:
         self.exp_avg, self.exp_avg_sq = torch.zeros_like(self.master), torch.zeros_like(self.master)
         self.work = torch.zeros(S, dtype=torch.bfloat16, device=dev)
         self.flat = torch.zeros(N_pad, dtype=torch.bfloat16, device=dev)
-        self.transport = transport
+        self.transport, self.stage = transport, stage
         if transport == "peer":
             from fsdp_sharded_mixed_flat_b200.peer import PeerGroup, PeerZero3Step
             self.stepper = PeerZero3Step(peer_group or PeerGroup(), plan, self.grad, self.master, self.exp_avg,
-                                         self.exp_avg_sq, self.work, self.flat, reduce_dtype=reduce_dtype,
-                                         kernels=kernels or z3)
+                                         self.exp_avg_sq, self.work, self.flat, stage=stage,
+                                         reduce_dtype=reduce_dtype, kernels=kernels or z3)
         else:
             self.stepper = CollectiveZero3Step(plan, self.grad, self.master, self.exp_avg, self.exp_avg_sq,
                                                self.work, self.flat, reduce_dtype=reduce_dtype, kernels=kernels or z3)
@@ -1079,9 +1079,13 @@ class CollectiveRunner:
     def phases(self) -> dict:
         """Mean seconds of each phase of the timed steps: the all-to-all, the fused
         kernel and the all-gather (NCCL); the two fences, the fused kernel reading
-        the peers' gradients and the gather kernel reading their shards (peer)."""
+        the peers' gradients and the gather kernel reading their shards (peer,
+        stage 3); the two fences around the one kernel that reads the peers'
+        gradients and stores the new shard into every rank's block (peer, stages
+        1 and 2)."""
         names = (("all_to_all", "reduce_adamw", "all_gather") if self.transport == "nccl" else
-                 ("fence_before", "reduce_adamw", "fence_between", "gather"))
+                 ("fence_before", "reduce_adamw", "fence_between", "gather") if self.stage == 3 else
+                 ("fence_before", "reduce_adamw", "fence_between"))
         return {n: statistics.mean(self.clock.seconds(m[k], m[k + 1]) for m in self.marks)
                 for k, n in enumerate(names)}
 
@@ -1122,8 +1126,10 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
     import torch
     mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
     peer = args.transport == "peer"
+    if args.stage != 3 and not peer:
+        raise SystemExit("--stage 1/2 with N > 1 is the peer form's fused kernel (--transport peer)")
     R = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport=args.transport,
-                         peer_group=peer_group)
+                         peer_group=peer_group, stage=args.stage)
     barrier = barrier or (lambda: torch.distributed.barrier())
     secs, job_secs, job_units, clk = time_collective_steps(R, args.steps, args.warmup, world, dev, barrier, clocks)
     ph = R.phases()
@@ -1151,20 +1157,30 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
     kname = f"k_reduce_adamw_vec<{'fp32' if mode == 0 else 'bf16'}, D={world}>"
     if peer:
         # the fused kernel pulls 2(D-1) bytes per owned element over NVLink and touches
-        # 28 B of its own HBM (its gradient slice, the state); the link is the bound
+        # 28 B of its own HBM (its gradient slice, the state); the link is the bound.
+        # At stages 1 and 2 it also pushes 2(D-1) bytes per owned element out (the
+        # new shard into every other rank's block).
         link_gbs = R.a2a_bytes / k1_s / 1e9
+        fences = ph["fence_before"] + ph["fence_between"]
+        if args.stage == 3:
+            kdesc = " (full layout, peers' gradients through the IPC mappings)"
+        else:
+            kdesc = (" with the all-gather's stores fused (zero3_reduce_adamw_gather: peers' gradients read and "
+                     "the new shard stored into every rank's block through the IPC mappings)")
         roofline = {"bound": "nvlink", "achieved": link_gbs, "peak": NVLINK_GBS, "unit": "GB/s",
                     "frac": link_gbs / NVLINK_GBS,
                     "peak_kind": "measured peer copy per direction per GPU on this pool (900 nominal)",
-                    "kernel": kname + " (full layout, peers' gradients through the IPC mappings)",
-                    "nvlink_bytes_in_per_launch": R.a2a_bytes, "hbm_algorithmic_gbs": k1_gbs, "traffic": None}
-        collective = {"fence_ms": 1e3 * (ph["fence_before"] + ph["fence_between"]),
-                      "reduce_adamw_ms": 1e3 * k1_s, "gather_ms": 1e3 * ph["gather"],
-                      "collective_share_of_step": (ph["fence_before"] + ph["fence_between"]) / max(step_s, 1e-12),
+                    "kernel": kname + kdesc, "nvlink_bytes_in_per_launch": R.a2a_bytes,
+                    "hbm_algorithmic_gbs": k1_gbs, "traffic": None}
+        collective = {"fence_ms": 1e3 * fences, "reduce_adamw_ms": 1e3 * k1_s,
+                      "collective_share_of_step": fences / max(step_s, 1e-12),
                       "nvlink_bytes_in_per_rank": R.a2a_bytes + R.gather_bytes,
                       "note": "the reduce-scatter's data movement runs inside the fused kernel and the "
-                              "all-gather's inside the gather kernel; the fences are a stream synchronisation "
-                              "and a group barrier"}
+                              "all-gather's inside the gather kernel (stage 3) or the fused kernel's own "
+                              "stores (stages 1 and 2); the fences are a stream synchronisation and a group "
+                              "barrier"}
+        if args.stage == 3:
+            collective["gather_ms"] = 1e3 * ph["gather"]
     else:
         roofline = {"bound": "hbm", "achieved": k1_gbs, "peak": hbm_peak, "unit": "GB/s",
                     "frac": k1_gbs / hbm_peak, "peak_kind": peak_kind + " (HBM copy, MEASURED_PEAKS.json)",
@@ -1190,7 +1206,7 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
         "clocks": clk,
         "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": 2 * R.N_pad,
                 "d2h_bytes_per_step": 2 * R.S, "steps": e2e_steps},
-        "gpu_launches": args.steps * (2 if peer else 1),
+        "gpu_launches": args.steps * (2 if peer and args.stage == 3 else 1),
         "ledger_bytes_per_device": ledger(z3, R.N, R.N_pad, world, R.N_pad),
     }
     if peer and not args.no_nccl_baseline:

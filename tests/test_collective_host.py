@@ -58,6 +58,13 @@ class OracleKernels:
                             oracle.hp(hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, hp.step),
                             layout=contrib_layout, reduce_dtype=reduce_dtype)
 
+    def zero3_reduce_adamw_gather(self, plan, rank, contrib, master, exp_avg, exp_avg_sq, work, gathered, hp,
+                                  contrib_layout, reduce_dtype):
+        self.zero3_reduce_adamw(plan, rank, contrib, master, exp_avg, exp_avg_sq, work, hp, contrib_layout,
+                                reduce_dtype)
+        for g in gathered:                                  # the new shard into every rank's block
+            _bits(g)[rank * plan.S:(rank + 1) * plan.S] = _bits(work)
+
     def zero3_gather_block(self, plan, shards, flat, tensor_out=None):
         assert tensor_out is None
         _bits(flat)[:] = oracle.all_gather([_bits(x) for x in shards], plan.S)

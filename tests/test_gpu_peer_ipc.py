@@ -93,14 +93,15 @@ def test_two_processes_share_through_cuda_ipc(mode, stage):
         assert np.array_equal(rflat, w), f"gathered block rank {r}"
 
 
-def _bench_worker(rank, world, port, out):
+def _bench_worker(rank, world, port, stage, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
     torch.cuda.set_device(0)
     import bench
     from fsdp_sharded_mixed_flat_b200 import zero3 as z3
     args = bench.parse_args(["--gpus", str(world), "--workload", "tiny_gpt", "--steps", "2", "--warmup", "1",
-                             "--e2e-steps", "1", "--transport", "peer", "--no-nccl-baseline"])
+                             "--e2e-steps", "1", "--transport", "peer", "--no-nccl-baseline",
+                             "--stage", str(stage)])
     line, R = bench.run_collective(args, rank, world, torch.device("cuda", 0), z3, synth, barrier=dist.barrier)
     torch.cuda.synchronize()
     dist.barrier()
@@ -112,23 +113,27 @@ def _bench_worker(rank, world, port, out):
     dist.destroy_process_group()
 
 
-def test_bench_peer_path_in_two_processes_on_one_gpu():
-    """bench.py's N > 1 headline (run_collective, peer form) with its real CUDA IPC
-    mappings and kernels, two ranks as two processes on one GPU (the timings mean
-    nothing here; the NCCL form, which needs a GPU per rank, is left out): the
-    JSON line, and both ranks' state equal to one oracle run over both ranks."""
+@pytest.mark.parametrize("stage", [3, 2])
+def test_bench_peer_path_in_two_processes_on_one_gpu(stage):
+    """bench.py's N > 1 headline (run_collective, peer form; at stage 2 the one
+    kernel that reads the peers' gradients and stores the new shard into every
+    rank's block) with its real CUDA IPC mappings and kernels, two ranks as two
+    processes on one GPU (the timings mean nothing here; the NCCL form, which
+    needs a GPU per rank, is left out): the JSON line, and both ranks' state
+    equal to one oracle run over both ranks."""
     assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
     from fsdp_sharded_mixed_flat_b200 import build
     build.build()
     world = 2
     with mp.get_context("spawn").Manager() as manager:
         out = manager.dict()
-        mp.spawn(_bench_worker, args=(world, _free_port(), out), nprocs=world, join=True)
+        mp.spawn(_bench_worker, args=(world, _free_port(), stage, out), nprocs=world, join=True)
         res = dict(out)
     line = res[0][0]
     assert line["n_gpus"] == 2 and line["comm_nranks"] == 2 and line["value"] > 0 and line["e2e"]["value"] > 0
-    assert line["roofline"]["bound"] == "nvlink" and line["gpu_launches"] == 2 * 2
-    assert line["collective"]["reduce_adamw_ms"] > 0 and line["collective"]["gather_ms"] > 0
+    assert line["roofline"]["bound"] == "nvlink" and line["gpu_launches"] == 2 * (2 if stage == 3 else 1)
+    assert line["collective"]["reduce_adamw_ms"] > 0
+    assert (line["collective"]["gather_ms"] > 0) if stage == 3 else ("gather_ms" not in line["collective"])
     assert "baseline_nccl" not in line
     w = synth.WORKLOADS["tiny_gpt"]
     _, N, N_pad, S = oracle.plan([synth.numel(s) for _, s in w["tensors"]], world, synth.ALIGN)
