@@ -187,6 +187,10 @@ Z3_API int zero3_allgather_bytes(int64_t block_params, int32_t n_blocks, int32_t
  *          launch (state arrays then hold all D partitions back to back).
  *   contrib host array of D device pointers, the ranks' bf16 gradient
  *          contributions in `contrib_layout` (Z3_CONTRIB_OWNED needs rank >= 0).
+ *          A pointer may address any memory this device can read with plain
+ *          loads: its own, or another GPU's mapped through peer access or
+ *          CUDA IPC (the kernel's loads then are the reduce-scatter's data
+ *          movement, [P2] §4), read only, never with TMA.
  *   master, exp_avg, exp_avg_sq  fp32, S elements (N_pad if rank = -1), read
  *          and updated in place.  In device memory, or in page-locked host
  *          memory mapped into the device's address space (the CPU-offload
@@ -392,7 +396,9 @@ Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t
  * [P2] §5.1: full_params = all_gather(local_shard) before the block runs) and
  * the optional unflatten into separate per-tensor buffers.
  *   shards     host array of D device pointers, shard r = rank r's S bf16
- *              working weights.
+ *              working weights.  A pointer may address another GPU's memory
+ *              mapped through peer access or CUDA IPC (plain loads; the
+ *              all-gather done by the receiving GPU's kernel).
  *   flat_out   device bf16, N_pad elements: flat_out[r*S + j] = shards[r][j].
  *              May be NULL when tensor_out is given.  A shard may already
  *              sit in place inside it, shards[r] == flat_out + r*S (a rank's
