@@ -1204,8 +1204,9 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
         "kernels": {"reduce_adamw_ms": 1e3 * k1_s, "reduce_adamw_gbs": k1_gbs},
         "roofline": roofline,
         "clocks": clk,
-        "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": 2 * R.N_pad,
-                "d2h_bytes_per_step": 2 * R.S, "steps": e2e_steps},
+        "e2e": {"value": e2e_units / e2e_secs, "unit": UNIT, "h2d_bytes_per_step": 2 * R.N_pad * world,
+                "d2h_bytes_per_step": 2 * R.S * world, "steps": e2e_steps,
+                "note": "bytes of all ranks: each copies its full gradient in and its new shard out"},
         "gpu_launches": args.steps * (2 if peer and args.stage == 3 else 1),
         "ledger_bytes_per_device": ledger(z3, R.N, R.N_pad, world, R.N_pad),
     }
