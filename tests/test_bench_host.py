@@ -81,44 +81,19 @@ def test_reference_arm_prints_one_contract_line():
     assert d["config"] == bench.contract_config(bench.parse_args([]), 1, 8, 1, 202_383_360)
 
 
-def _file_peer_group(tmpdir: str, rank: int):
-    """A PeerGroup whose "IPC" is a file every rank maps (host memory shared
-    between the gloo processes): share() moves the tensor's storage into a
-    fresh shared file mapping, so this rank's later writes are seen by every
-    rank that opened it."""
-    import itertools
-
-    import torch
-    from fsdp_sharded_mixed_flat_b200.peer import PeerGroup
-    count = itertools.count()
-
-    def share(t):
-        path = os.path.join(tmpdir, f"rank{rank}_{next(count)}")
-        mapped = torch.from_file(path, shared=True, size=t.numel(), dtype=t.dtype)
-        mapped.copy_(t)
-        t.set_(mapped)
-        return path, t.numel(), t.dtype
-
-    def open_(handle):
-        path, n, dtype = handle
-        return torch.from_file(path, shared=True, size=n, dtype=dtype)
-
-    return PeerGroup(share_fn=share, open_fn=open_, sync_fn=lambda device: None)
-
-
 def _collective_worker(rank, world, port, mode, transport, stage, tmpdir, out):
     import numpy as np
     import torch
 
     import synth
     from fsdp_sharded_mixed_flat_b200 import zero3 as z3
-    from test_collective_host import OracleKernels
+    from test_collective_host import OracleKernels, file_peer_group
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     args = bench.parse_args(["--gpus", str(world), "--workload", "tiny_gpt", "--steps", "2", "--warmup", "1",
                              "--e2e-steps", "1", "--reduce-dtype", "bf16" if mode else "fp32",
                              "--transport", transport, "--stage", str(stage)])
-    group = _file_peer_group(tmpdir, rank) if transport == "peer" else None
+    group = file_peer_group(tmpdir, rank) if transport == "peer" else None
     line, R = bench.run_collective(args, rank, world, torch.device("cpu"), z3, synth, kernels=OracleKernels(),
                                    barrier=dist.barrier, peer_group=group)
     out[rank] = (line, R.master.numpy().copy(), R.exp_avg.numpy().copy(), R.exp_avg_sq.numpy().copy(),

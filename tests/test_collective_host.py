@@ -70,6 +70,30 @@ class OracleKernels:
         _bits(flat)[:] = oracle.all_gather([_bits(x) for x in shards], plan.S)
 
 
+def file_peer_group(tmpdir: str, rank: int):
+    """A PeerGroup whose "IPC" is a file every rank maps (host memory shared
+    between the gloo processes): share() moves the tensor's storage into a
+    fresh shared file mapping, so this rank's later writes are seen by every
+    rank that opened it."""
+    import itertools
+
+    from fsdp_sharded_mixed_flat_b200.peer import PeerGroup
+    count = itertools.count()
+
+    def share(t):
+        path = os.path.join(tmpdir, f"rank{rank}_{next(count)}")
+        mapped = torch.from_file(path, shared=True, size=t.numel(), dtype=t.dtype)
+        mapped.copy_(t)
+        t.set_(mapped)
+        return path, t.numel(), t.dtype
+
+    def open_(handle):
+        path, n, dtype = handle
+        return torch.from_file(path, shared=True, size=n, dtype=dtype)
+
+    return PeerGroup(share_fn=share, open_fn=open_, sync_fn=lambda device: None)
+
+
 def _worker(rank, world, port, mode, steps, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -189,7 +213,7 @@ def test_collective_hybrid_step_equals_the_two_level_oracle(R, D, mode):
         assert np.array_equal(rflat, w), f"gathered block rank {g}"
 
 
-def _failing_worker(rank, world, port, how, out):
+def _failing_worker(rank, world, port, how, form, tmpdir, out):
     import time
     from datetime import timedelta
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -202,7 +226,12 @@ def _failing_worker(rank, world, port, how, out):
     master = synth.master_weights(N, N_pad, seed=SEED)[rank * S:(rank + 1) * S].clone()
     m, v = torch.zeros(S), torch.zeros(S)
     work, flat = torch.zeros(S, dtype=torch.bfloat16), torch.zeros(N_pad, dtype=torch.bfloat16)
-    step = CollectiveZero3Step(plan, grad, master, m, v, work, flat, kernels=OracleKernels())
+    if form == "peer":                               # the fused peer-memory step, fences = gloo barriers
+        from fsdp_sharded_mixed_flat_b200.peer import PeerZero3Step
+        step = PeerZero3Step(file_peer_group(tmpdir, rank), plan, grad, master, m, v, work, flat,
+                             kernels=OracleKernels())
+    else:
+        step = CollectiveZero3Step(plan, grad, master, m, v, work, flat, kernels=OracleKernels())
     step.step(z3.adamw(step=1))                      # a whole step with every rank
     if rank == world - 1:                            # the failing rank leaves between steps
         if how == "stall":
@@ -218,18 +247,22 @@ def _failing_worker(rank, world, port, how, out):
     os._exit(0)
 
 
+@pytest.mark.parametrize("form", ["nccl", "peer"])
 @pytest.mark.parametrize("how", ["exit", "stall"])
-def test_collective_step_surfaces_a_lost_rank_as_an_error(how):
+def test_collective_step_surfaces_a_lost_rank_as_an_error(how, form, tmp_path):
     """A rank that exits, or stops answering, between steps: the surviving ranks'
     next step ends with an error from the process group (a closed connection, or
     its 3-second timeout), well before the lost rank would have come back; no rank
-    waits forever.  (Failure detection made on the host, with gloo ranks.)"""
+    waits forever.  Both forms of the step: collectives moving the bytes, and the
+    peer-memory step whose fences are group barriers.  (Failure detection made on
+    the host, with gloo ranks.)"""
     world = 3
     ctx = mp.get_context("spawn")
     with ctx.Manager() as manager:
         out = manager.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_failing_worker, args=(r, world, port, how, out)) for r in range(world)]
+        procs = [ctx.Process(target=_failing_worker, args=(r, world, port, how, form, str(tmp_path), out))
+                 for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
