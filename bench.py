@@ -58,7 +58,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "owned params/s for fused reduce+AdamW+cast; achieved HBM GB/s vs ~8 TB/s"
 UNIT = "owned params/s"
-NVLINK_GBS = 770.0   # measured peer copy on this machine's B200s, per direction per GPU (900 GB/s nominal)
+NVLINK_GBS = 770.0   # measured B200 peer copy over NVLink 5, per direction per GPU (900 GB/s nominal)
 # committed ncu summaries of the fused kernel, by workload (fp32 reduce), with its DRAM traffic
 PROFILE_K1 = {"llama7b_d8": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_llama7b_d8.md"),
               "llama7b_hybrid": os.path.join(ROOT, "profiles", "k_reduce_adamw_vec_hybrid_llama7b_4x8.md")}
@@ -1169,7 +1169,7 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
                      "the new shard stored into every rank's block through the IPC mappings)")
         roofline = {"bound": "nvlink", "achieved": link_gbs, "peak": NVLINK_GBS, "unit": "GB/s",
                     "frac": link_gbs / NVLINK_GBS,
-                    "peak_kind": "measured peer copy per direction per GPU on this pool (900 nominal)",
+                    "peak_kind": "measured B200 peer copy over NVLink 5, per direction per GPU (900 nominal)",
                     "kernel": kname + kdesc, "nvlink_bytes_in_per_launch": R.a2a_bytes,
                     "hbm_algorithmic_gbs": k1_gbs, "traffic": None}
         collective = {"fence_ms": 1e3 * fences, "reduce_adamw_ms": 1e3 * k1_s,
