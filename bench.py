@@ -1126,6 +1126,15 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
     import torch
     mode = z3.Z3_REDUCE_BF16 if args.reduce_dtype == "bf16" else z3.Z3_REDUCE_FP32
     peer = args.transport == "peer"
+    unsupported = [o for o, on in (("--graph", args.graph), ("--unflatten-copy", args.unflatten_copy),
+                                   ("--offload", bool(args.offload)), ("--split", args.split),
+                                   ("--nodes", args.nodes > 1),
+                                   (f"--workload {args.workload}",
+                                    args.workload in ("llama7b_hybrid", "llama70b_shard", "profile_hybrid")))
+                   if on]
+    if unsupported:
+        raise SystemExit(f"N > 1 runs the block step over the N GPUs; {', '.join(unsupported)} is measured on one "
+                         f"GPU only (HYBRID_SHARD across GPUs is collective.CollectiveHybridStep)")
     if args.stage != 3 and not peer:
         raise SystemExit("--stage 1/2 with N > 1 is the peer form's fused kernel (--transport peer)")
     R = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport=args.transport,

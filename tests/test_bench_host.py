@@ -219,3 +219,17 @@ def test_code_hash_ignores_comments_only(tmp_path):
     c.write_text("// header\nint f(int x) {\n    return 3 * x;\n}\n")
     assert bench.code_sha256([a]) == bench.code_sha256([b])
     assert bench.code_sha256([a]) != bench.code_sha256([c])
+
+
+@pytest.mark.parametrize("flags", [["--graph"], ["--offload"], ["--nodes", "4"], ["--workload", "llama7b_hybrid"],
+                                   ["--transport", "nccl", "--stage", "2"]])
+def test_multi_gpu_path_refuses_what_it_does_not_measure(flags):
+    """Options measured on one GPU only are refused at N > 1, before any collective,
+    instead of being silently dropped."""
+    import torch
+
+    import synth
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    args = bench.parse_args(["--gpus", "2"] + flags)
+    with pytest.raises(SystemExit):
+        bench.run_collective(args, 0, 2, torch.device("cpu"), z3, synth)
