@@ -1076,6 +1076,13 @@ class CollectiveRunner:
         hp = self.z3.adamw(step=self.step_no, **a)
         self.stepper.step(hp, mark=self.clock.mark if timed else None, marks=self.marks)
 
+    def close(self) -> None:
+        """Once this rank's kernels are done, release its mappings of the other
+        ranks' memory (peer form)."""
+        self.clock.sync()
+        if self.transport == "peer":
+            self.stepper.peers.close()
+
     def phases(self) -> dict:
         """Mean seconds of each phase of the timed steps: the all-to-all, the fused
         kernel and the all-gather (NCCL); the two fences, the fused kernel reading
@@ -1223,6 +1230,7 @@ def run_collective(args, rank: int, world: int, dev, z3, synth, kernels=None, cl
         B = CollectiveRunner(z3, synth, args.workload, world, rank, mode, dev, kernels=kernels, transport="nccl")
         _, b_secs, b_units, _ = time_collective_steps(B, args.steps, args.warmup, world, dev, barrier)
         bph = B.phases()
+        B.close()
         line["baseline_nccl"] = {
             "value": b_units / b_secs, "unit": UNIT, "ms_per_step": 1e3 * b_secs / args.steps,
             "all_to_all_ms": 1e3 * bph["all_to_all"], "reduce_adamw_ms": 1e3 * bph["reduce_adamw"],
@@ -1261,6 +1269,7 @@ def run_ours(args):
                                  clocks=ClockSampler(f"GPU-{uuid}" if uuid is not None else None))
         if rank == 0:
             print(json.dumps(line), flush=True)
+        R.close()
         del R
         dist.barrier()
         dist.destroy_process_group()

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libzero3.so")
 
-SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "node_fold.cu", "gather.cu", "host_adamw.cpp"]
+SOURCES = ["plan.cpp", "device.cu", "reduce_adamw.cu", "node_fold.cu", "gather.cu", "host_adamw.cpp", "ipc.cpp"]
 # per-source host-compiler flags: the host optimiser must round every operation
 # on its own (no contraction into fused multiply-adds); -fno-math-errno only
 # drops errno bookkeeping around sqrt, so the loop vectorises

@@ -19,9 +19,11 @@ kernels can address the peers' memory with plain loads and stores:
   every rank's gathered block (P2P stores; at most Z3_GATHER_MAX ranks), and a
   final barrier replaces steps 3-4.
 
-Every wait is a host-side stream synchronisation followed by a group barrier,
-so no kernel ever waits on another rank; the barriers take the process group's
-timeout.  The kernels reach the peers' memory with plain loads and stores only (no
+The mappings come from libzero3's IPC entry points, which map each peer
+allocation into the address space of the importing rank's own device with peer
+access enabled, so the kernels launched there can address it.  Every wait is a
+host-side stream synchronisation followed by a group barrier, so no kernel ever
+waits on another rank; the barriers take the process group's timeout.  The kernels reach the peers' memory with plain loads and stores only (no
 TMA), and no library kernel is ever handed a peer's memory: only libzero3.so's
 own kernels touch the mappings.
 """
@@ -36,7 +38,14 @@ from . import zero3 as z3
 
 
 class PeerGroup:
-    """The ranks of a process group, with CUDA IPC sharing of device tensors."""
+    """The ranks of a process group, with CUDA IPC sharing of device tensors.
+
+    By default a rank exports the allocation holding its tensor through
+    libzero3 (zero3_ipc_export) and every other rank maps it into the address
+    space of ITS OWN device (zero3_ipc_import, peer access to the owning GPU
+    enabled as needed), the device its kernels launch on; the mapped view
+    aliases the other rank's memory.  share_fn / open_fn replace the exchange
+    (host tests use stand-ins)."""
 
     def __init__(self, group=None, share_fn: Optional[Callable] = None, open_fn: Optional[Callable] = None,
                  sync_fn: Optional[Callable] = None):
@@ -44,25 +53,38 @@ class PeerGroup:
         self.rank = dist.get_rank(group)
         self.size = dist.get_world_size(group)
         self._sync = sync_fn or (lambda device: torch.cuda.current_stream(device).synchronize())
+        self._device = None
+        self._mappings: List[int] = []
         if share_fn is None or open_fn is None:
-            from torch.multiprocessing.reductions import reduce_tensor
-
-            def share_fn(t):
-                return reduce_tensor(t)
-
-            def open_fn(shared):
-                rebuild, args = shared
-                return rebuild(*args)
+            share_fn, open_fn = self._export, self._import
         self._share, self._open = share_fn, open_fn
+
+    @staticmethod
+    def _export(t: torch.Tensor):
+        handle, offset, size = z3.zero3_ipc_export(t)
+        return handle, offset, size, t.numel(), str(t.dtype).replace("torch.", "")
+
+    def _import(self, shared) -> torch.Tensor:
+        handle, offset, size, numel, dtype = shared
+        view, base = z3.zero3_ipc_import(handle, offset, size, numel, getattr(torch, dtype), self._device)
+        self._mappings.append(base)
+        return view
 
     def share(self, t: torch.Tensor) -> List[torch.Tensor]:
         """Every rank's tensor `t`, in rank order: this rank's own, the others
-        opened through their IPC handles (mapped into this process)."""
+        mapped into this process for the device `t` lives on."""
         if self.size == 1:
             return [t]                              # nobody to share with
         handles = [None] * self.size
         dist.all_gather_object(handles, self._share(t), group=self.group)
+        self._device = t.get_device() if t.is_cuda else None
         return [t if k == self.rank else self._open(h) for k, h in enumerate(handles)]
+
+    def close(self) -> None:
+        """Release this rank's mappings of the other ranks' memory.  Call it once
+        every kernel that reads or writes them has finished (after a fence)."""
+        while self._mappings:
+            z3.zero3_ipc_close(self._mappings.pop(), self._device)
 
     def fence(self, device) -> None:
         """Everything this rank enqueued on its current stream has finished, and so

@@ -87,6 +87,12 @@ def _load() -> C.CDLL:
     L.zero3_reduce_scatter.restype = C.c_int
     L.zero3_host_adamw.argtypes = [i64, vp, i32, vp, vp, vp, vp, C.POINTER(AdamW), i32]
     L.zero3_host_adamw.restype = C.c_int
+    L.zero3_ipc_export.argtypes = [vp, vp, C.POINTER(i64), C.POINTER(i64)]
+    L.zero3_ipc_export.restype = C.c_int
+    L.zero3_ipc_import.argtypes = [vp, i64, C.POINTER(vp), C.POINTER(vp)]
+    L.zero3_ipc_import.restype = C.c_int
+    L.zero3_ipc_close.argtypes = [vp]
+    L.zero3_ipc_close.restype = C.c_int
     return L
 
 
@@ -492,3 +498,54 @@ def zero3_host_adamw(grad: torch.Tensor, master: torch.Tensor, exp_avg: torch.Te
     vp = _host_tensor(exp_avg_sq, torch.float32, n, "exp_avg_sq")
     wp = _host_tensor(work_bf16, torch.bfloat16, n, "work_bf16")
     _check(_lib.zero3_host_adamw(n, gp, gdt, mp, ap, vp, wp, C.byref(hp), n_threads), "zero3_host_adamw")
+
+
+# ------------------------------------------------- peer memory through CUDA IPC
+Z3_IPC_HANDLE_BYTES = 64
+
+
+class _DeviceArray:
+    """A device address range described by the CUDA array interface, so that torch
+    can view it as a tensor without copying (used for imported peer memory)."""
+
+    def __init__(self, ptr: int, numel: int, typestr: str):
+        self.__cuda_array_interface__ = {"shape": (numel,), "typestr": typestr, "data": (ptr, False),
+                                         "strides": None, "version": 2}
+
+
+def zero3_ipc_export(t: torch.Tensor):
+    """(handle bytes, byte offset of t in its allocation, allocation bytes) of a
+    contiguous CUDA tensor, for another process's zero3_ipc_import."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+        raise ValueError("zero3_ipc_export needs a contiguous CUDA tensor")
+    h = (C.c_char * Z3_IPC_HANDLE_BYTES)()
+    off, size = C.c_int64(), C.c_int64()
+    rc = _call_on(t.get_device(), _lib.zero3_ipc_export, t.data_ptr(), h, C.byref(off), C.byref(size))
+    _check(rc, "zero3_ipc_export")
+    return bytes(h), off.value, size.value
+
+
+def zero3_ipc_import(handle: bytes, offset: int, size: int, numel: int, dtype: torch.dtype, device: int):
+    """Map another process's exported allocation into `device`'s address space
+    (peer access to the owning GPU enabled as needed) and view the `numel`
+    elements of `dtype` at `offset` as a tensor.  Returns (tensor, mapping base
+    for zero3_ipc_close).  The tensor aliases the other process's memory; only
+    the library's kernels should touch it, and only until the mapping is closed."""
+    if len(handle) != Z3_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is 64 bytes")
+    itemsize = torch.empty((), dtype=dtype).element_size()
+    if offset < 0 or offset + numel * itemsize > size:
+        raise ValueError(f"{numel} elements at byte {offset} exceed the exported allocation of {size} bytes")
+    buf = (C.c_char * Z3_IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    ptr, base = C.c_void_p(), C.c_void_p()
+    _check(_call_on(device, _lib.zero3_ipc_import, buf, offset, C.byref(ptr), C.byref(base)), "zero3_ipc_import")
+    raw = {2: "<i2", 4: "<f4"}.get(itemsize)
+    if raw is None:
+        raise TypeError(f"no peer view for {dtype}")
+    t = torch.as_tensor(_DeviceArray(ptr.value, numel, raw))
+    return (t.view(dtype) if t.dtype != dtype else t), base.value
+
+
+def zero3_ipc_close(base: int, device: int) -> None:
+    """Release one import of the mapping at `base` (the last release unmaps it)."""
+    _check(_call_on(device, _lib.zero3_ipc_close, base), "zero3_ipc_close")

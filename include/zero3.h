@@ -418,6 +418,39 @@ Z3_API int zero3_reduce_adamw_dev(const z3_plan* p, int32_t rank, const uint16_t
 Z3_API int zero3_gather_block(const z3_plan* p, const uint16_t* const* shards, uint16_t* flat_out,
                               uint16_t* const* tensor_out, void* cuda_stream);
 
+/* ------------------------------------ another process's memory, through CUDA IPC
+ * The D-GPU form of the step ([P2] §4, §5.1): the fused kernel on rank r reads
+ * slice P_r of every rank's gradient, and the gather kernel every rank's shard,
+ * from the other GPUs' memory with plain loads.  Each rank exports the device
+ * allocation that holds a buffer; every other rank imports it, which maps it
+ * into the address space of the importing thread's CURRENT device (the device
+ * its kernels launch on) with peer access to the owning GPU enabled as needed
+ * (cudaIpcMemLazyEnablePeerAccess).
+ *
+ * zero3_ipc_export: for a pointer into device memory from cudaMalloc (e.g.
+ * PyTorch's caching allocator), the IPC handle of the allocation holding it
+ * (Z3_IPC_HANDLE_BYTES bytes written to handle_out), the pointer's byte offset
+ * in the allocation and the allocation's size in bytes.
+ * Errors: Z3_EINVAL (a NULL argument, ptr not inside a device allocation),
+ * Z3_ECUDA (the runtime cannot export the allocation, e.g. virtual-memory
+ * mapped memory).
+ *
+ * zero3_ipc_import: maps the allocation of another process's handle and sets
+ * *ptr_out = mapping + offset and *base_out = the mapping (for zero3_ipc_close).
+ * The caller checks offset against the exporter's size.  Importing a handle
+ * this process holds already returns the same mapping and counts the import.
+ * A handle exported by this same process cannot be imported.
+ * Errors: Z3_EINVAL (a NULL argument, offset < 0), Z3_ECUDA (the runtime
+ * refused the mapping), Z3_ENOMEM (host bookkeeping).
+ *
+ * zero3_ipc_close: releases one import of the mapping at base; the last
+ * release unmaps it.  Nothing the device still has in flight may use it.
+ * Errors: Z3_EINVAL (NULL, or not a mapping from zero3_ipc_import), Z3_ECUDA. */
+#define Z3_IPC_HANDLE_BYTES 64
+Z3_API int zero3_ipc_export(const void* ptr, void* handle_out, int64_t* offset_out, int64_t* size_out);
+Z3_API int zero3_ipc_import(const void* handle, int64_t offset, void** ptr_out, void** base_out);
+Z3_API int zero3_ipc_close(void* base);
+
 #ifdef __cplusplus
 }
 #endif

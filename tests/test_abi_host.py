@@ -11,6 +11,7 @@ import subprocess
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import synth
@@ -36,7 +37,8 @@ def test_library_exports_every_declared_symbol():
                             "zero3_reduce_adamw_hybrid", "zero3_node_sum", "zero3_fold_adamw",
                             "zero3_reduce_adamw_gather",
                             "zero3_step_scalars", "zero3_reduce_adamw_dev", "zero3_gather_block",
-                            "zero3_reduce_scatter", "zero3_host_adamw"]), names
+                            "zero3_reduce_scatter", "zero3_host_adamw", "zero3_ipc_export",
+                            "zero3_ipc_import", "zero3_ipc_close"]), names
     out = subprocess.run(["nm", "-D", "--defined-only", z3.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -418,3 +420,24 @@ def test_gather_block_argument_errors():
 def test_gather_empty_plan_is_a_no_op():
     p = z3.zero3_plan([(0,)], 2, 8)
     assert call_gather(p) == z3.Z3_OK
+
+
+def test_ipc_argument_errors():
+    """The IPC entry points refuse NULL arguments, a negative offset and a base
+    that is not one of their mappings, before any CUDA call."""
+    L, E = z3.lib(), z3.Z3_EINVAL
+    h = (C.c_char * z3.Z3_IPC_HANDLE_BYTES)()
+    off, size = C.c_int64(), C.c_int64()
+    ptr, base = C.c_void_p(), C.c_void_p()
+    assert L.zero3_ipc_export(None, h, C.byref(off), C.byref(size)) == E
+    assert L.zero3_ipc_export(P16, None, C.byref(off), C.byref(size)) == E
+    assert L.zero3_ipc_export(P16, h, None, C.byref(size)) == E
+    assert L.zero3_ipc_export(P16, h, C.byref(off), None) == E
+    assert L.zero3_ipc_import(None, 0, C.byref(ptr), C.byref(base)) == E
+    assert L.zero3_ipc_import(h, -1, C.byref(ptr), C.byref(base)) == E
+    assert L.zero3_ipc_import(h, 0, None, C.byref(base)) == E
+    assert L.zero3_ipc_import(h, 0, C.byref(ptr), None) == E
+    assert L.zero3_ipc_close(None) == E
+    assert L.zero3_ipc_close(P16 * 5) == E                       # never imported
+    with pytest.raises(ValueError):                              # the binding checks the exporter's size
+        z3.zero3_ipc_import(bytes(64), 4096, 4096, 1, torch.float32, 0)

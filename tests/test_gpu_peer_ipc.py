@@ -37,6 +37,21 @@ def _bits(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def test_ipc_export_reports_the_allocation_of_a_view():
+    """Within one process (no mapping, no kernel): two views into one allocation
+    export the same handle, offsets that differ by the views' distance, and an
+    allocation size that holds both."""
+    from fsdp_sharded_mixed_flat_b200 import build
+    build.build()
+    from fsdp_sharded_mixed_flat_b200 import zero3 as z3
+    x = torch.zeros(1 << 20, dtype=torch.float32, device="cuda")
+    h0, off0, size0 = z3.zero3_ipc_export(x)
+    h1, off1, size1 = z3.zero3_ipc_export(x[12345:])
+    assert len(h0) == z3.Z3_IPC_HANDLE_BYTES and h0 == h1 and size0 == size1
+    assert off1 - off0 == 12345 * 4 and off0 >= 0 and off0 + x.numel() * 4 <= size0
+    assert x.data_ptr() - off0 == x[12345:].data_ptr() - off1       # one allocation base
+
+
 def _worker(rank, world, port, mode, stage, steps, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
@@ -58,7 +73,8 @@ def _worker(rank, world, port, mode, stage, steps, out):
     dist.barrier()                 # every rank's last writes into the others' memory have landed
     out[rank] = (master.cpu().numpy().copy(), m.cpu().numpy().copy(), v.cpu().numpy().copy(), _bits(work).copy(),
                  _bits(flat).copy())
-    del step                       # drop the mappings of the other process's memory first
+    step.peers.close()             # unmap the other process's memory (this rank's kernels are done)
+    del step
     torch.cuda.synchronize()
     dist.barrier()
     dist.destroy_process_group()
@@ -107,6 +123,7 @@ def _bench_worker(rank, world, port, stage, out):
     dist.barrier()
     out[rank] = (line, R.master.cpu().numpy().copy(), R.exp_avg.cpu().numpy().copy(),
                  R.exp_avg_sq.cpu().numpy().copy(), _bits(R.work).copy(), _bits(R.flat).copy(), R.step_no)
+    R.close()
     del R
     torch.cuda.synchronize()
     dist.barrier()
