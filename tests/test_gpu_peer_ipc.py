@@ -80,13 +80,13 @@ def _worker(rank, world, port, mode, stage, steps, out):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("stage", [3, 2])
-@pytest.mark.parametrize("mode", [0, 1], ids=["fp32", "bf16"])
-def test_two_processes_share_through_cuda_ipc(mode, stage):
+@pytest.mark.parametrize("world,stage,mode", [(2, 3, 0), (2, 3, 1), (2, 2, 0), (2, 2, 1), (3, 3, 0), (3, 2, 1)])
+def test_processes_share_through_cuda_ipc(world, stage, mode):
+    """world ranks as processes on one GPU (3: the generic rank count's kernel)."""
     assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
     from fsdp_sharded_mixed_flat_b200 import build
     build.build()
-    world, steps = 2, 3
+    steps = 3
     with mp.get_context("spawn").Manager() as manager:
         out = manager.dict()
         mp.spawn(_worker, args=(world, _free_port(), mode, stage, steps, out), nprocs=world, join=True)
